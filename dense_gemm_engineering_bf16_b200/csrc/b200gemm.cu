@@ -1,0 +1,332 @@
+// Host side of the C ABI declared in include/b200gemm.h: argument checks
+// (the correctness contract of "GPU 执行模型", section "正确性契约"),
+// shape-bucket configuration choice (section "编译与 autotune": choices are
+// cached per device and shape class, with no compilation or tuning on the
+// call path), TMA tensor-map encoding ("Modern GPU Programming For MLSys -
+// 书籍总结", section 2.5), and the cluster launch of the persistent kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "b200gemm.h"
+#include "gemm_bf16_sm100.cuh"
+
+namespace {
+
+using b200::DeviceStatus;
+
+// ---------------------------------------------------------------- configs --
+
+using Cfg1x256F32 = b200::GemmBf16Cfg<1, 256, 4, 0>;
+using Cfg1x256B16 = b200::GemmBf16Cfg<1, 256, 4, 1>;
+using Cfg1x128F32 = b200::GemmBf16Cfg<1, 128, 6, 0>;
+using Cfg1x128B16 = b200::GemmBf16Cfg<1, 128, 6, 1>;
+using Cfg2x256F32 = b200::GemmBf16Cfg<2, 256, 6, 0>;
+using Cfg2x256B16 = b200::GemmBf16Cfg<2, 256, 6, 1>;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    bool supported = false;
+    int sm_count = 0;
+    DeviceStatus *status = nullptr;
+    // per (config, out type): smem attribute set, co-resident clusters
+    bool attr_done[GEMM_CFG_COUNT_][2] = {};
+    int max_clusters[GEMM_CFG_COUNT_][2] = {};
+};
+
+std::mutex g_mutex;
+DeviceState g_devices[kMaxDevices];
+std::atomic<int> g_forced{GEMM_CFG_AUTO};
+thread_local int g_last_cuda_error = 0;
+int32_t g_last_where = -1;
+int32_t g_last_block = -1;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+gemm_status_t cuda_fail(cudaError_t e) {
+    g_last_cuda_error = static_cast<int>(e);
+    return GEMM_ERR_LAUNCH;
+}
+
+uint64_t watchdog_ns(int64_t K) {
+    static const uint64_t base = [] {
+        const char *s = std::getenv("B200GEMM_WATCHDOG_MS");
+        const long long ms = s ? std::atoll(s) : 2000;
+        return static_cast<uint64_t>(ms > 0 ? ms : 2000) * 1000000ull;
+    }();
+    // One tile's main loop grows with K; allow ~100 ns per K element on top.
+    return base + static_cast<uint64_t>(K) * 100ull;
+}
+
+// Device of the current thread, checked to be compute capability 10.0, with
+// its status block allocated.
+gemm_status_t current_device(int &dev, DeviceState *&st) {
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        g_last_cuda_error = static_cast<int>(e);
+        return GEMM_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    st = &g_devices[dev];
+    if (!st->ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            return GEMM_ERR_UNSUPPORTED_DEVICE;
+        }
+        st->supported = (major == 10 && minor == 0);
+        if (!st->supported) {
+            st->ready = true;
+            return GEMM_ERR_UNSUPPORTED_DEVICE;
+        }
+        if ((e = cudaDeviceGetAttribute(&st->sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaMalloc(&st->status, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
+        if ((e = cudaMemset(st->status, 0, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        st->ready = true;
+    }
+    return st->supported ? GEMM_OK : GEMM_ERR_UNSUPPORTED_DEVICE;
+}
+
+// [begin, end) byte ranges of a row-major rows x cols matrix with leading dim ld.
+bool overlaps(const void *p, int64_t rows, int64_t cols, int64_t ld, int64_t esize,
+              const void *q, int64_t qrows, int64_t qcols, int64_t qld, int64_t qesize) {
+    if (rows <= 0 || cols <= 0 || qrows <= 0 || qcols <= 0 || !p || !q) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(p);
+    const uintptr_t a1 = a0 + static_cast<uintptr_t>(((rows - 1) * ld + cols) * esize);
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(q);
+    const uintptr_t b1 = b0 + static_cast<uintptr_t>(((qrows - 1) * qld + qcols) * qesize);
+    return a0 < b1 && b0 < a1;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = 0x7FFFFFFF;
+
+// Checks shared by every entry point.  elem sizes in bytes.
+gemm_status_t check_args(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K,
+                         int64_t lda, int64_t ldb, int64_t ldc, int64_t ea, int64_t eb, int64_t ec) {
+    if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_VALUE;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return GEMM_ERR_TOO_LARGE;
+    if (M == 0 || N == 0) return GEMM_OK;
+    if (!C) return GEMM_ERR_INVALID_VALUE;
+    if (ldc < N) return GEMM_ERR_INVALID_VALUE;
+    if (K > 0) {
+        if (!A || !B) return GEMM_ERR_INVALID_VALUE;
+        if (lda < K || ldb < K) return GEMM_ERR_INVALID_VALUE;
+        if (!aligned16(A) || !aligned16(B)) return GEMM_ERR_MISALIGNED;
+        if ((lda * ea) % 16 || (ldb * eb) % 16) return GEMM_ERR_MISALIGNED;
+        if (lda * ea >= (int64_t(1) << 40) || ldb * eb >= (int64_t(1) << 40)) return GEMM_ERR_TOO_LARGE;
+        if (overlaps(C, M, N, ldc, ec, A, M, K, lda, ea) || overlaps(C, M, N, ldc, ec, B, N, K, ldb, eb))
+            return GEMM_ERR_ALIAS;
+    }
+    if (!aligned16(C) || (ldc * ec) % 16) return GEMM_ERR_MISALIGNED;
+    if (ldc * ec >= (int64_t(1) << 40)) return GEMM_ERR_TOO_LARGE;
+    return GEMM_OK;
+}
+
+// ------------------------------------------------------------ tensor maps --
+
+gemm_status_t encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, int64_t inner,
+                        int64_t outer, int64_t ld_bytes, uint32_t box_inner, uint32_t box_outer) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_bytes)};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dtype, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = static_cast<int>(r);
+        return GEMM_ERR_LAUNCH;
+    }
+    return GEMM_OK;
+}
+
+// --------------------------------------------------------------- launches --
+
+gemm_config_t select_config(int64_t M, int64_t N, int64_t /*K*/) {
+    const int forced = g_forced.load(std::memory_order_relaxed);
+    if (forced != GEMM_CFG_AUTO) return static_cast<gemm_config_t>(forced);
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int64_t wide_tiles = ((M + 127) / 128) * ((N + 255) / 256);
+    if (pair_tiles >= 74) return GEMM_CFG_2CTA_256x256;
+    if (wide_tiles >= 148) return GEMM_CFG_1CTA_128x256;
+    return GEMM_CFG_1CTA_128x128;
+}
+
+template <class Cfg>
+gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, const void *B, void *C,
+                          int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                          cudaStream_t stream) {
+    auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
+    const int oi = Cfg::OUT;
+    cudaError_t e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Cfg::CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.blockDim = dim3(Cfg::THREADS, 1, 1);
+    lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    lc.stream = stream;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!st->attr_done[cfg_id][oi]) {
+            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          Cfg::SMEM_BYTES)) != cudaSuccess)
+                return cuda_fail(e);
+            int clusters = st->sm_count / Cfg::CG;
+            if (Cfg::CG > 1) {
+                lc.gridDim = dim3(Cfg::CG * clusters, 1, 1);
+                int n = 0;
+                if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
+                if (n > 0) clusters = n;
+            }
+            st->max_clusters[cfg_id][oi] = clusters;
+            st->attr_done[cfg_id][oi] = true;
+        }
+    }
+    const CUtensorMapDataType cdt = Cfg::OUT == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int64_t ec = Cfg::OUT == 0 ? 4 : 2;
+    alignas(64) CUtensorMap tmA, tmB, tmC;
+    gemm_status_t s;
+    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK, Cfg::BM_CTA)) != GEMM_OK) return s;
+    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::B_ROWS)) != GEMM_OK) return s;
+    // The store map covers the columns that end on a 16-byte granule; the
+    // kernel writes the rest of each row ([n_tma, N)) with plain stores.  If
+    // no whole granule exists the map is a placeholder the kernel never uses.
+    const int64_t n_tma = (N * ec / 16) * 16 / ec;
+    if ((s = encode_2d(&tmC, cdt, C, n_tma > 0 ? n_tma : 16 / ec, M, ldc * ec, Cfg::EPI_COLS, 32)) != GEMM_OK)
+        return s;
+
+    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
+    const int64_t clusters = tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi];
+    lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
+    e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
+                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), st->status, watchdog_ns(K));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GEMM_OK;
+}
+
+template <typename T>
+gemm_status_t launch_zero(void *C, int64_t M, int64_t N, int64_t ldc, int sm_count, cudaStream_t stream) {
+    const int64_t total = M * N;
+    int64_t blocks = (total + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    b200::zero_fill_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<T *>(C), M, N, ldc);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                        int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, cudaStream_t stream) {
+    if (c_type != GEMM_OUT_F32 && c_type != GEMM_OUT_BF16) return GEMM_ERR_INVALID_VALUE;
+    const int64_t ec = c_type == GEMM_OUT_F32 ? 4 : 2;
+    gemm_status_t s = check_args(A, B, C, M, N, K, lda, ldb, ldc, 2, 2, ec);
+    if (s != GEMM_OK || M == 0 || N == 0) return s;
+    int dev;
+    DeviceState *st;
+    if ((s = current_device(dev, st)) != GEMM_OK) return s;
+    if (K == 0) {
+        return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
+                                      : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
+    }
+    const gemm_config_t cfg = select_config(M, N, K);
+    const bool f32 = c_type == GEMM_OUT_F32;
+    switch (cfg) {
+        case GEMM_CFG_1CTA_128x256:
+            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_1CTA_128x128:
+            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_2CTA_256x256:
+            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        default:
+            return GEMM_ERR_INVALID_VALUE;
+    }
+}
+
+gemm_status_t gemm_check_device_status(cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int dev;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GEMM_ERR_UNSUPPORTED_DEVICE;
+    DeviceStatus *status;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        status = g_devices[dev].status;
+    }
+    if (!status) return GEMM_OK;   // nothing ever launched on this device
+    DeviceStatus h;
+    if ((e = cudaMemcpy(&h, status, sizeof(h), cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
+    if (h.code == 0) return GEMM_OK;
+    g_last_where = h.where;
+    g_last_block = h.block;
+    if ((e = cudaMemset(status, 0, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
+    return static_cast<gemm_status_t>(h.code);
+}
+
+void gemm_last_timeout_detail(int32_t *where, int32_t *block) {
+    if (where) *where = g_last_where;
+    if (block) *block = g_last_block;
+}
+
+const char *gemm_status_string(gemm_status_t s) {
+    switch (s) {
+        case GEMM_OK: return "GEMM_OK: success";
+        case GEMM_ERR_INVALID_VALUE: return "GEMM_ERR_INVALID_VALUE: negative size, leading dimension too small, null pointer or bad enum";
+        case GEMM_ERR_MISALIGNED: return "GEMM_ERR_MISALIGNED: pointer or leading dimension not a multiple of 16 bytes";
+        case GEMM_ERR_ALIAS: return "GEMM_ERR_ALIAS: C overlaps an input";
+        case GEMM_ERR_UNSUPPORTED_DEVICE: return "GEMM_ERR_UNSUPPORTED_DEVICE: no CUDA device, or not compute capability 10.0 (B200)";
+        case GEMM_ERR_LAUNCH: return "GEMM_ERR_LAUNCH: a CUDA runtime or driver call failed";
+        case GEMM_ERR_TIMEOUT: return "GEMM_ERR_TIMEOUT: a bounded wait inside a kernel expired (device watchdog)";
+        case GEMM_ERR_TOO_LARGE: return "GEMM_ERR_TOO_LARGE: a dimension or stride exceeds the TMA limits";
+        default: return "unknown gemm_status_t";
+    }
+}
+
+int gemm_last_cuda_error(void) { return g_last_cuda_error; }
+
+gemm_status_t gemm_force_config(gemm_config_t config) {
+    if (static_cast<int>(config) < 0 || static_cast<int>(config) >= GEMM_CFG_COUNT_) return GEMM_ERR_INVALID_VALUE;
+    g_forced.store(static_cast<int>(config), std::memory_order_relaxed);
+    return GEMM_OK;
+}
+
+gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K) { return select_config(M, N, K); }
+
+int gemm_launches_per_call(int64_t M, int64_t N, int64_t K) {
+    (void)K;
+    return (M > 0 && N > 0) ? 1 : 0;
+}
+
+}  // extern "C"

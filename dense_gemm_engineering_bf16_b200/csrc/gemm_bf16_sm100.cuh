@@ -1,0 +1,391 @@
+// Persistent, warp-specialised bf16 GEMM for sm_100a:  C = A . B
+//
+// The construction follows part III of "Modern GPU Programming For MLSys -
+// 书籍总结" (omica.com.cn): a 128 x N output tile (step 1), K-loop
+// accumulation (step 2), tiles spread over CTAs (step 3), TMA loads (step 4),
+// a multi-stage shared-memory ring (step 5), a persistent kernel walking a
+// tile schedule (step 6), warp specialisation into TMA producer / MMA issuer
+// / write-back (step 7) and, for CG == 2, a CTA pair running one
+// cta_group::2 MMA over both CTAs' shared memory with a 256-row tile (step 8).
+//
+// Per CTA (192 threads):
+//   warp 0      TMA producer: waits empty[s], loads the A and B k-tiles of
+//               stage s (128-byte swizzle), completion counted in bytes on
+//               the pair leader's full[s].
+//   warp 1      TMEM owner (alloc / dealloc) and, in the pair leader only, the
+//               MMA issuer: waits full[s], issues BK/16 tcgen05.mma into the
+//               TMEM accumulator, commits to empty[s] (both CTAs); after the
+//               last k-tile of a tile commits to tmem_full[b].
+//   warps 2-5   epilogue: waits tmem_full[b], tcgen05.ld 32 rows x 32 columns
+//               per warp, converts, writes a swizzled staging buffer, and TMA-
+//               stores it; releases tmem_empty[b] (pair leader's barrier)
+//               once the accumulator is read, so tile i+1's main loop runs
+//               while tile i drains (TMEM double buffer, 2 x BN columns).
+//
+// Tails: TMA loads zero-fill outside [0,K) x [0,M) / [0,N) element by
+// element.  TMA stores clip rows exactly but write whole 16-byte granules
+// along a row, so C's tensor map covers only the columns [0, n_tma) that end
+// on a granule boundary; the last < 16 bytes of each row ([n_tma, N)) are
+// written with plain predicated stores.  Every mbarrier wait is bounded.
+#pragma once
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace b200 {
+
+// Device status block (global memory, one per device).  code != 0 records
+// the first expired wait; the host reads and clears it.
+struct DeviceStatus {
+    uint32_t code;
+    int32_t where;
+    int32_t block;
+    uint32_t pad;
+};
+
+constexpr uint32_t kStatusTimeout = 6;   // == GEMM_ERR_TIMEOUT
+
+enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3 };
+enum : int { kBarFull = 1, kBarEmpty = 2, kBarTmemFull = 3, kBarTmemEmpty = 4, kBarTail = 5 };
+
+__host__ __device__ constexpr int pow2_at_least(int v, int lo) {
+    int p = lo;
+    while (p < v) p *= 2;
+    return p;
+}
+
+template <int CG_, int BN_, int STAGES_, int OUT_>
+struct GemmBf16Cfg {
+    static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
+    static constexpr int BN = BN_;                 // tile N == MMA N
+    static constexpr int STAGES = STAGES_;         // shared-memory ring depth
+    static constexpr int OUT = OUT_;               // 0: f32 C, 1: bf16 C
+    static constexpr int BM_CTA = 128;             // accumulator rows per CTA (TMEM lanes)
+    static constexpr int BM = 128 * CG;            // tile M == MMA M
+    static constexpr int BK = 64;                  // 64 bf16 = one 128-byte swizzle row
+    static constexpr int UMMA_K = 16;              // K per tcgen05.mma (kind::f16)
+    static constexpr int B_ROWS = BN / CG;         // B rows this CTA loads per k-tile
+    static constexpr int A_BYTES = BM_CTA * BK * 2;
+    static constexpr int B_BYTES = B_ROWS * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TX_BYTES = STAGE_BYTES * CG;   // bytes landing on the leader's full[s]
+    static constexpr int EPI_COLS = OUT == 0 ? 32 : 64; // columns in one 128-byte staged row
+    static constexpr int EPI_CHUNKS = BN / EPI_COLS;
+    static constexpr int EPI_BUF = 32 * 128;       // one warp's 32 rows x 128 bytes
+    static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
+    static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
+    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
+    static constexpr int THREADS = 192;
+    static constexpr int GROUP_M = 8;              // tile rows per raster group (L2 reuse)
+
+    static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
+    static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows <= 256, whole 8-row swizzle atoms");
+    static_assert(BN % EPI_COLS == 0, "epilogue chunks cover the tile");
+    static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+    static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
+};
+
+// Tile index -> (tile row, tile column), grouped along M so that CTAs
+// running at the same time share A row-panels and B column-panels in L2.
+__device__ __forceinline__ void raster_tile(int tile, int num_m, int num_n, int group_m,
+                                            int &tm, int &tn) {
+    const int group_size = group_m * num_n;
+    const int group = tile / group_size;
+    const int first_m = group * group_m;
+    const int rows = min(group_m, num_m - first_m);
+    const int local = tile - group * group_size;
+    tm = first_m + local % rows;
+    tn = local / rows;
+}
+
+__device__ __forceinline__ void record_timeout(DeviceStatus *status, volatile uint32_t *abort_flag,
+                                               uint32_t abort_smem, int cg, int where) {
+    *abort_flag = 1u;
+    if (cg == 2) store_cluster_u32(map_to_cta(abort_smem, cluster_cta_rank() ^ 1u), 1u);
+    if (atomicCAS(&status->code, 0u, kStatusTimeout) == 0u) {
+        status->where = where;
+        status->block = static_cast<int32_t>(blockIdx.x);
+        __threadfence();
+    }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC,
+                       int M, int N, int K, void *C, int64_t ldc, int n_tma,
+                       DeviceStatus *status, uint64_t timeout_ns) {
+    constexpr int CG = Cfg::CG;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment of the shared-memory window offset (swizzle atoms).
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    const uint32_t base = smem_addr(smem);
+
+    const uint32_t warp = threadIdx.x / 32;
+    const uint32_t lane = threadIdx.x % 32;
+    const uint32_t rank = (CG == 2) ? cluster_cta_rank() : 0u;
+
+    const uint32_t bar0 = base + Cfg::BAR_OFF;
+    auto full_bar = [&](uint32_t s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](uint32_t s) { return bar0 + 8u * (Cfg::STAGES + s); };
+    auto tfull_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + b); };
+    auto tempty_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + b); };
+    const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
+    const uint32_t abort_slot = tmem_slot + 4u;
+    volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
+    volatile uint32_t *abort_flag = tmem_slot_ptr + 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 4 * CG);
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB);
+        tma_prefetch_map(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc<CG>(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish<CG>();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot_ptr;
+
+    const int num_m = (M + Cfg::BM - 1) / Cfg::BM;
+    const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + Cfg::BK - 1) / Cfg::BK;
+    const int cluster_id = static_cast<int>(blockIdx.x) / CG;
+    const int num_clusters = static_cast<int>(gridDim.x) / CG;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            const uint32_t leader_rank = 0;
+            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+                int tm, tn;
+                raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+                const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;
+                const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarEmpty);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = base + stage * Cfg::STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + Cfg::A_BYTES;
+                    const int kx = kb * Cfg::BK;
+                    if constexpr (CG == 1) {
+                        mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
+                        tma_load_2d(a_dst, &tmA, full_bar(stage), kx, a_row);
+                        tma_load_2d(b_dst, &tmB, full_bar(stage), kx, b_row);
+                    } else {
+                        if (rank == leader_rank) mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
+                        const uint32_t bar = map_to_cta(full_bar(stage), leader_rank);
+                        tma_load_2d_pair(a_dst, &tmA, bar, kx, a_row);
+                        tma_load_2d_pair(b_dst, &tmB, bar, kx, b_row);
+                    }
+                    if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // Tail: every stage handed out must be released by the MMA before
+            // this CTA may exit (its empty barriers still receive arrivals).
+            for (int i = 0; ok && i < Cfg::STAGES; ++i) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarTail);
+                    ok = false;
+                }
+                if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // --------------------------------------------------- MMA issuer --
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN);
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            int t = 0;
+            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters, ++t) {
+                const uint32_t buf = static_cast<uint32_t>(t) & 1u;
+                const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
+                if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarTmemEmpty);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + buf * Cfg::BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarFull);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a0 = base + stage * Cfg::STAGE_BYTES;
+                    const uint32_t b0 = a0 + Cfg::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
+                        mma_bf16_ss<CG>(d_tmem, sw128_kmajor_desc(a0 + kk * 32),
+                                        sw128_kmajor_desc(b0 + kk * 32), idesc,
+                                        (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit<CG>(empty_bar(stage), 0x3);
+                    if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit<CG>(tfull_bar(buf), 0x3);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------- epilogue --
+        const uint32_t sub = warp & 3u;            // TMEM lanes [32*sub, 32*sub + 32)
+        const uint32_t ew = warp - 2u;             // staging slot
+        const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
+        uint32_t nstore = 0;
+        int t = 0;
+        for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++t) {
+            int tm, tn;
+            raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+            const uint32_t buf = static_cast<uint32_t>(t) & 1u;
+            const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
+            // One lane waits; the verdict is broadcast so the warp stays
+            // converged for the .sync.aligned TMEM loads below.
+            uint32_t ready = 1;
+            if (lane == 0 && !mbar_wait(tfull_bar(buf), acc_phase, abort_flag, timeout_ns)) {
+                record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarTmemFull);
+                ready = 0;
+            }
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
+            tc_fence_after_sync();
+            const int row0 = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
+            const int col0 = tn * Cfg::BN;
+            const uint32_t tbase = tmem_base + ((sub * 32u) << 16) + buf * Cfg::BN;
+#pragma unroll 1
+            for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
+                uint32_t packed[32];
+                if constexpr (Cfg::OUT == 0) {
+                    tmem_ld_32x32b_x32(tbase + c * 32, packed);
+                    tmem_ld_wait();
+                } else {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_32x32b_x32(tbase + c * 64, v0);
+                    tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+                        packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+                    }
+                }
+                if (c == Cfg::EPI_CHUNKS - 1) {
+                    // This warp has read its whole slice of accumulator `buf`.
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (CG == 1) mbar_arrive_local(tempty_bar(buf));
+                        else mbar_arrive_cluster(map_to_cta(tempty_bar(buf), 0));
+                    }
+                }
+                const int cstart = col0 + c * Cfg::EPI_COLS;
+                if (cstart >= N) continue;                  // chunk wholly right of C
+                if (cstart + Cfg::EPI_COLS > n_tma) {
+                    // Columns [n_tma, N) end C's rows inside a 16-byte granule:
+                    // a TMA store writes whole granules, so these few elements
+                    // (< 16 bytes per row) go out as plain predicated stores.
+                    const int row = row0 + static_cast<int>(lane);
+                    if (row < M) {
+                        uint8_t *crow = static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * (Cfg::OUT == 0 ? 4 : 2);
+#pragma unroll
+                        for (int w = 0; w < Cfg::EPI_COLS; ++w) {
+                            const int col = cstart + w;
+                            if (col >= n_tma && col < N) {
+                                if constexpr (Cfg::OUT == 0) {
+                                    reinterpret_cast<uint32_t *>(crow)[col] = packed[w];
+                                } else {
+                                    reinterpret_cast<uint16_t *>(crow)[col] =
+                                        static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
+                                }
+                            }
+                        }
+                    }
+                    if (cstart >= n_tma) continue;          // nothing left for the TMA store
+                }
+                const uint32_t sbuf = stage_base + (nstore & 1u) * Cfg::EPI_BUF;
+                if (lane == 0) bulk_wait_group_read<1>();   // the store that used sbuf is done reading
+                __syncwarp();
+                // Row `lane` of the 32 x 128-byte box; 16-byte chunk j goes to
+                // chunk slot j ^ (row % 8) -- the TMA 128-byte swizzle.
+                const uint32_t row_addr = sbuf + lane * 128u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4),
+                                 packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmC, sbuf, col0 + c * Cfg::EPI_COLS, row0);
+                    bulk_commit_group();
+                }
+                ++nstore;
+            }
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
+
+    // -------------------------------------------------------- teardown --
+    tc_fence_before_sync();
+    __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();
+    if (*abort_flag) {
+        // A wait expired somewhere: give in-flight TMA copies and MMAs time
+        // to land before the TMEM and shared memory are released.
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+// C = 0 for K == 0 (the empty sum), one element per thread, grid-stride.
+template <typename T>
+__global__ void zero_fill_kernel(T *C, int64_t M, int64_t N, int64_t ldc) {
+    const int64_t total = M * N;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / N;
+        const int64_t c = i - r * N;
+        C[r * ldc + c] = T(0);
+    }
+}
+
+}  // namespace b200

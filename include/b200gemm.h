@@ -1,0 +1,132 @@
+/*
+ * b200gemm -- dense GEMM for NVIDIA B200 (sm_100a), plain C ABI.
+ *
+ *   C = A . B      A: M x K,  B: K x N,  C: M x N
+ *
+ * The operation is the matrix product C_{MxN} = A_{MxK} B_{KxN} of
+ * "GPU 执行模型" (wineandchord.com/llm/systems/gpu-execution/), section
+ * "Tile 的容量约束"; the kernels follow the Blackwell GEMM construction of
+ * "Modern GPU Programming For MLSys - 书籍总结" (omica.com.cn), part III
+ * (steps 1-9: tiling, K loop, TMA, software pipeline, persistent kernel,
+ * warp specialisation, 2-CTA cluster), and the argument contract below
+ * follows the checklist of "GPU 执行模型", section "正确性契约" (shape,
+ * stride, layout, dtype, alignment, tails, accumulation and rounding,
+ * aliasing, stream lifetime, determinism).
+ *
+ * Layouts (all row-major with explicit leading dimensions, in ELEMENTS):
+ *   A  element (i,k) at A[i*lda + k]            (M rows of K)
+ *   B  element (k,j) at B[j*ldb + k]            (stored K-major: N rows of K)
+ *   C  element (i,j) at C[i*ldc + j]            (M rows of N)
+ *   MXFP8 scales: sfa[i*(K/32) + kb], sfb[j*(K/32) + kb], one E8M0 byte per
+ *   32 consecutive K elements (kb = k/32), rows packed (leading dim K/32).
+ *
+ * Ownership: every pointer is a DEVICE pointer owned by the caller, valid
+ * until the work queued on `stream` has finished.  The library keeps one
+ * small per-device status block (allocated on the first call on a device)
+ * and caches per-device launch attributes; nothing else is retained.
+ *
+ * Execution: calls are asynchronous on `stream` (0 = the legacy default
+ * stream) and never synchronise, except gemm_check_device_status().
+ * C is overwritten (no alpha/beta).  Results are deterministic for a given
+ * shape and configuration (fixed per-element accumulation order).
+ *
+ * Errors: every function returns a status and never aborts or throws.
+ * Argument checks run on the host before anything is queued.  A device-side
+ * watchdog bounds every wait inside the kernels; if one expires, the kernel
+ * records GEMM_ERR_TIMEOUT in the status block and exits cleanly, and the
+ * next gemm_check_device_status() reports it.
+ */
+#ifndef B200GEMM_H
+#define B200GEMM_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define B200GEMM_API __attribute__((visibility("default")))
+#else
+#define B200GEMM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GEMM_OK = 0,
+    GEMM_ERR_INVALID_VALUE = 1,     /* negative size, ld too small, bad enum, null pointer */
+    GEMM_ERR_MISALIGNED = 2,        /* pointer or ld*elem_size not a multiple of 16 bytes */
+    GEMM_ERR_ALIAS = 3,             /* C overlaps an input */
+    GEMM_ERR_UNSUPPORTED_DEVICE = 4,/* no device, or not compute capability 10.0 */
+    GEMM_ERR_LAUNCH = 5,            /* a CUDA runtime call failed (see gemm_last_cuda_error) */
+    GEMM_ERR_TIMEOUT = 6,           /* a kernel's bounded wait expired (device watchdog) */
+    GEMM_ERR_TOO_LARGE = 7          /* a dimension exceeds 2^31-1 (TMA coordinates are int32) */
+} gemm_status_t;
+
+typedef enum {
+    GEMM_OUT_F32 = 0,               /* C is float32 */
+    GEMM_OUT_BF16 = 1               /* C is bfloat16, rounded to nearest even */
+} gemm_out_t;
+
+/* Kernel configurations.  GEMM_CFG_AUTO picks by shape; the others force a
+ * configuration (for tests and benchmarks) through gemm_force_config(). */
+typedef enum {
+    GEMM_CFG_AUTO = 0,
+    GEMM_CFG_1CTA_128x256 = 1,      /* one CTA per tile, tile 128 x 256, tcgen05 cta_group::1 */
+    GEMM_CFG_1CTA_128x128 = 2,      /* one CTA per tile, tile 128 x 128 */
+    GEMM_CFG_2CTA_256x256 = 3,      /* CTA pair per tile, tile 256 x 256, cta_group::2 */
+    GEMM_CFG_COUNT_ = 4
+} gemm_config_t;
+
+/*
+ * gemm_bf16: C = A . B with bf16 A and B, fp32 accumulation in tensor memory,
+ * C written as fp32 or bf16 (c_type).
+ *
+ *   A, B     device pointers to bfloat16; C device pointer to c_type
+ *   M, N, K  >= 0.  M == 0 or N == 0: nothing to do (GEMM_OK).
+ *            K == 0 with M, N > 0: C is set to zero (the empty sum).
+ *   lda, ldb >= K, ldc >= N (elements); lda*2, ldb*2 and ldc*sizeof(c_type)
+ *            multiples of 16 bytes; A, B, C 16-byte aligned.
+ *   Tails: any M, N, K are accepted; partial tiles are zero-filled on load
+ *   and clipped on store, so no element outside the M x N (x K) ranges is
+ *   read or written.
+ *   C must not overlap A or B.
+ */
+B200GEMM_API gemm_status_t gemm_bf16(const void *A, const void *B, void *C,
+                        int64_t M, int64_t N, int64_t K,
+                        int64_t lda, int64_t ldb, int64_t ldc,
+                        gemm_out_t c_type, cudaStream_t stream);
+
+/* Synchronises `stream`, then reports and clears the device watchdog status
+ * of the current device: GEMM_OK, or GEMM_ERR_TIMEOUT if a kernel's bounded
+ * wait expired since the last check.  GEMM_ERR_LAUNCH if the stream itself
+ * reports a CUDA error. */
+B200GEMM_API gemm_status_t gemm_check_device_status(cudaStream_t stream);
+
+/* Detail of the last watchdog event read by gemm_check_device_status():
+ * which wait expired (role * 16 + barrier kind) and in which CTA; -1 if none. */
+B200GEMM_API void gemm_last_timeout_detail(int32_t *where, int32_t *block);
+
+/* Static description of a status code. */
+B200GEMM_API const char *gemm_status_string(gemm_status_t status);
+
+/* The CUDA error behind the last GEMM_ERR_LAUNCH on this host thread. */
+B200GEMM_API int gemm_last_cuda_error(void);
+
+/* Force a kernel configuration for subsequent calls in this process
+ * (GEMM_CFG_AUTO restores shape-based selection).  Returns
+ * GEMM_ERR_INVALID_VALUE for an unknown configuration. */
+B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
+
+/* The configuration the next gemm_bf16 call with this shape would use. */
+B200GEMM_API gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K);
+
+/* Number of kernels that gemm_bf16 / gemm_mxfp8 queue per call for this
+ * shape (0 for an empty problem). */
+B200GEMM_API int gemm_launches_per_call(int64_t M, int64_t N, int64_t K);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B200GEMM_H */

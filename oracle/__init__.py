@@ -247,3 +247,29 @@ def smem_estimate_double_buffer(m_tile: int, n_tile: int, k_tile: int, stages: i
     section "Tile 的容量约束" -- read with 2 = bf16 bytes per element and
     s = the number of pipeline stages."""
     return 2 * stages * (m_tile * k_tile + k_tile * n_tile)
+
+
+# ---------------------------------------------------- full-size properties --
+
+def gemm_line_sums_f64(a64: np.ndarray, b64_nk: np.ndarray):
+    """Row and column sums of C = A.B without forming C, for checking every
+    output of a full-size product at once:
+
+        sum_j C[i][j] = sum_k a(i,k) (sum_j b(k,j))     (row sums, length M)
+        sum_i C[i][j] = sum_k (sum_i a(i,k)) b(k,j)     (column sums, length N)
+
+    together with the matching magnitudes sum_j sum_k |a(i,k) b(k,j)| and
+    sum_i sum_k |a(i,k) b(k,j)| that scale the per-element tolerance.
+    All in fp64; each is a plain contraction (library matrix-vector products).
+    """
+    a64 = np.asarray(a64, dtype=np.float64)
+    b64 = np.asarray(b64_nk, dtype=np.float64)
+    b_col = b64.sum(axis=0)               # over j, for each k
+    b_abs = np.abs(b64).sum(axis=0)
+    a_row = a64.sum(axis=0)               # over i, for each k
+    a_abs = np.abs(a64).sum(axis=0)
+    rows = a64 @ b_col
+    rows_mag = np.abs(a64) @ b_abs
+    cols = b64 @ a_row
+    cols_mag = np.abs(b64) @ a_abs
+    return rows, rows_mag, cols, cols_mag

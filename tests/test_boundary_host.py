@@ -1,0 +1,95 @@
+"""The C-ABI boundary on the host: the library loads, exports every symbol
+the public header declares, and rejects bad arguments with the documented
+status before anything is queued.  No kernel is launched here (CPU only)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from dense_gemm_engineering_bf16_b200 import gemm as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
+def _declared():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        names += re.findall(r"^B200GEMM_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_and_library_exports_everything():
+    names = _declared()
+    assert "gemm_bf16" in names and "gemm_check_device_status" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", G.library_path], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in names:
+        assert hasattr(G.lib, n)
+
+
+A = 0x7F0000000000   # never dereferenced: every call below fails validation first
+B = 0x7F0000100000
+C = 0x7F0000200000
+
+
+def _call(A_=A, B_=B, C_=C, M=128, N=128, K=128, lda=None, ldb=None, ldc=None, ct=G.OUT_F32):
+    lda = K if lda is None else lda
+    ldb = K if ldb is None else ldb
+    ldc = N if ldc is None else ldc
+    return G.lib.gemm_bf16(A_, B_, C_, M, N, K, lda, ldb, ldc, ct, 0)
+
+
+def test_rejects_bad_arguments_before_any_launch():
+    assert _call(M=-1) == 1
+    assert _call(K=-5) == 1
+    assert _call(ct=7) == 1
+    assert _call(lda=64) == 1                       # lda < K
+    assert _call(ldb=100) == 1                      # ldb < K
+    assert _call(ldc=64) == 1                       # ldc < N
+    assert _call(C_=0) == 1                         # null C
+    assert _call(A_=0) == 1                         # null A with K > 0
+    assert _call(A_=A + 2) == 2                     # misaligned pointer
+    assert _call(C_=C + 8) == 2
+    assert _call(K=100, lda=100, ldb=104) == 2      # 200-byte row pitch
+    assert _call(N=100, ldc=102) == 2               # 408-byte fp32 pitch
+    assert _call(N=100, ldc=100, ct=G.OUT_BF16) == 2   # 200-byte bf16 pitch
+    assert _call(M=1 << 31) == 7
+    assert _call(C_=A + 4096) == 3                  # C overlaps A
+    assert _call(C_=B) == 3                         # C overlaps B
+
+
+def test_empty_problems_succeed_without_touching_memory():
+    assert _call(M=0) == 0
+    assert _call(N=0) == 0
+    assert _call(M=0, A_=0, B_=0, C_=0) == 0
+    assert G.gemm_launches_per_call(0, 5, 5) == 0
+    assert G.gemm_launches_per_call(5, 5, 0) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_unsupported_device():
+    assert _call() == 4
+    assert G.gemm_check_device_status(stream=0, check=False) in (0, 5)
+
+
+def test_status_strings_and_config_control():
+    for code, name in G.STATUS_NAMES.items():
+        assert G.gemm_status_string(code).startswith(name)
+    assert "unknown" in G.gemm_status_string(99)
+    assert G.lib.gemm_force_config(99) == 1
+    G.gemm_force_config("2cta_256x256")
+    assert G.gemm_select_config(16, 16, 16) == G.CONFIGS["2cta_256x256"]
+    G.gemm_force_config("auto")
+    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256"]
+    assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
+    with pytest.raises(G.GemmError):
+        G.gemm_bf16(A, B, C, -1, 1, 1, 1, 1, 1, stream=0)

@@ -329,3 +329,15 @@ def test_mxfp8_brute_force_tiny():
                     sb = Fraction(2) ** (int(sfb[j, k // 32]) - 127)
                     want += Fraction(float(av[i, k])) * sa * Fraction(float(bv[j, k])) * sb
                 assert Fraction(c[i, j]) == want
+
+
+def test_line_sums_match_full_product():
+    """The row/column-sum identity used for full-size checks agrees with the
+    full oracle product (exactly, on integers)."""
+    a_bits, b_bits = synth.bf16_operands(37, 29, 70, "ints", workload=14)
+    a = oracle.decode_bf16(a_bits)
+    b = oracle.decode_bf16(b_bits)
+    c, s = oracle.gemm_bf16_f64(a_bits, b_bits, with_abs=True)
+    rows, rows_mag, cols, cols_mag = oracle.gemm_line_sums_f64(a, b)
+    assert np.array_equal(rows, c.sum(axis=1)) and np.array_equal(cols, c.sum(axis=0))
+    assert np.array_equal(rows_mag, s.sum(axis=1)) and np.array_equal(cols_mag, s.sum(axis=0))
