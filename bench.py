@@ -176,8 +176,10 @@ def run_reference(args, world, rank):
     from dense_gemm_engineering_bf16_b200 import synth
     M, N, K, dist, wid, desc = WORKLOADS[args.workload]
     a_bits, b_bits = synth.bf16_operands(M, N, K, dist, workload=wid)
-    # each step: a bounded row sample of the workload (about 1-2 s)
-    _, _, R = oracle_sample(a_bits, b_bits, K, budget_s=1.0)
+    # each step: a bounded row sample of the workload, sized so that all
+    # warm-up + timed steps take about two and a half minutes
+    per_step = max(0.05, min(2.0, 150.0 / (args.steps + args.warmup)))
+    _, _, R = oracle_sample(a_bits, b_bits, K, budget_s=per_step)
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
