@@ -241,6 +241,62 @@ gemm_status_t launch_zero(void *C, int64_t M, int64_t N, int64_t ldc, int sm_cou
     return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
 }
 
+// ------------------------------------------------ allocation-free variant --
+//
+// gemm_bf16_noalloc runs the same kernels as gemm_bf16, but the kernels'
+// scratch (the watchdog status block) lives in the file-scope array below
+// instead of memory obtained from cudaMalloc.  The array is part of the
+// library image: every GPU that loads the library holds its
+// kNoAllocScratchBytes until the process exits.  All calls share it.
+
+constexpr size_t kNoAllocScratchBytes = 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Scratch one call needs: the status block, for every shape.
+constexpr size_t noalloc_scratch_bytes() { return sizeof(DeviceStatus); }
+
+DeviceState g_noalloc_devices[kMaxDevices];
+
+// Per-device set-up, once, with the device current: check the device, take
+// the address of the scratch array with cudaGetSymbolAddress (host code may
+// not use the array's name as a device address), and zero it.
+gemm_status_t noalloc_device(int &dev, DeviceState *&st) {
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        g_last_cuda_error = static_cast<int>(e);
+        return GEMM_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    st = &g_noalloc_devices[dev];
+    if (!st->ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return GEMM_ERR_UNSUPPORTED_DEVICE;
+        st->supported = (major == 10 && minor == 0);
+        if (!st->supported) {
+            st->ready = true;
+            return GEMM_ERR_UNSUPPORTED_DEVICE;
+        }
+        if ((e = cudaDeviceGetAttribute(&st->sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        void *scratch = nullptr;
+        if ((e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch)) != cudaSuccess || !scratch)
+            return cuda_fail(e);
+        if ((e = cudaMemset(scratch, 0, kNoAllocScratchBytes)) != cudaSuccess) return cuda_fail(e);
+        st->status = static_cast<DeviceStatus *>(scratch);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        st->ready = true;
+    }
+    return st->supported ? GEMM_OK : GEMM_ERR_UNSUPPORTED_DEVICE;
+}
+
 }  // namespace
 
 extern "C" {
@@ -327,6 +383,41 @@ gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K) { return selec
 int gemm_launches_per_call(int64_t M, int64_t N, int64_t K) {
     (void)K;
     return (M > 0 && N > 0) ? 1 : 0;
+}
+
+gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                                int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type,
+                                cudaStream_t stream) {
+    if (c_type != GEMM_OUT_F32 && c_type != GEMM_OUT_BF16) return GEMM_ERR_INVALID_VALUE;
+    const int64_t ec = c_type == GEMM_OUT_F32 ? 4 : 2;
+    gemm_status_t s = check_args(A, B, C, M, N, K, lda, ldb, ldc, 2, 2, ec);
+    if (s != GEMM_OK || M == 0 || N == 0) return s;
+    if (noalloc_scratch_bytes() > kNoAllocScratchBytes) return GEMM_ERR_TOO_LARGE;
+    int dev;
+    DeviceState *st;
+    if ((s = noalloc_device(dev, st)) != GEMM_OK) return s;
+    if (K == 0) {
+        return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
+                                      : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
+    }
+    // The status word must start at zero for the kernel to record a timeout.
+    cudaError_t e = cudaMemsetAsync(st->status, 0, noalloc_scratch_bytes(), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const gemm_config_t cfg = select_config(M, N, K);
+    const bool f32 = c_type == GEMM_OUT_F32;
+    switch (cfg) {
+        case GEMM_CFG_1CTA_128x256:
+            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_1CTA_128x128:
+            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_2CTA_256x256:
+            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        default:
+            return GEMM_ERR_INVALID_VALUE;
+    }
 }
 
 }  // extern "C"

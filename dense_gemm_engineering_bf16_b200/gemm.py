@@ -42,6 +42,8 @@ _int = ctypes.c_int
 
 lib.gemm_bf16.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp]
 lib.gemm_bf16.restype = _int
+lib.gemm_bf16_noalloc.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp]
+lib.gemm_bf16_noalloc.restype = _int
 lib.gemm_check_device_status.argtypes = [_vp]
 lib.gemm_check_device_status.restype = _int
 lib.gemm_last_timeout_detail.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
@@ -103,6 +105,15 @@ def gemm_bf16(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
     """
     st = lib.gemm_bf16(_ptr(A), _ptr(B), _ptr(C), M, N, K, lda, ldb, ldc, int(c_type), _stream(stream))
     return _check(st, "gemm_bf16", check)
+
+
+def gemm_bf16_noalloc(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
+                      c_type: int = OUT_F32, stream=None, check: bool = True) -> int:
+    """gemm_bf16 without any device allocation: the kernels' scratch is a
+    static array inside the library (see include/b200gemm.h)."""
+    st = lib.gemm_bf16_noalloc(_ptr(A), _ptr(B), _ptr(C), M, N, K, lda, ldb, ldc, int(c_type),
+                               _stream(stream))
+    return _check(st, "gemm_bf16_noalloc", check)
 
 
 def gemm_check_device_status(stream=None, check: bool = True) -> int:

@@ -97,6 +97,37 @@ B200GEMM_API gemm_status_t gemm_bf16(const void *A, const void *B, void *C,
                         int64_t lda, int64_t ldb, int64_t ldc,
                         gemm_out_t c_type, cudaStream_t stream);
 
+/*
+ * gemm_bf16_noalloc: gemm_bf16 for callers that cannot allocate device memory.
+ * (No counterpart in the pages: it is a packaging choice of this library.)
+ *
+ * gemm_bf16 allocates a small status block with cudaMalloc on its first call
+ * on each device.  Some callers cannot allow that: code that runs while a
+ * framework's caching allocator owns the whole device memory, allocator or
+ * memory-pool callbacks that must not re-enter the allocator, and latency-
+ * critical loops where cudaMalloc's implicit device synchronisation is not
+ * allowed.  This entry point computes exactly what gemm_bf16 computes, with
+ * the same arguments, checks, kernels and configuration choice, but it
+ * allocates nothing: the kernels' scratch (the 16-byte watchdog status
+ * block) lives in a static 256-byte device array inside the library, which
+ * every GPU that loads the library holds until the process exits.  A call
+ * that would need more scratch than that array is rejected with
+ * GEMM_ERR_TOO_LARGE (no shape does today: the scratch does not grow with
+ * M, N or K).
+ *
+ * The first call on each device does a one-time set-up with that device
+ * current (it looks up the array's device address and zeroes it); make that
+ * first call before any stream capture.  Each call clears the status word
+ * on `stream` before its kernel.  All calls share the one array, so
+ * calls that overlap on the GPU (different streams, no ordering) race on it.
+ * Watchdog timeouts of this entry point are recorded in that array and are
+ * not reported by gemm_check_device_status().
+ */
+B200GEMM_API gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C,
+                                             int64_t M, int64_t N, int64_t K,
+                                             int64_t lda, int64_t ldb, int64_t ldc,
+                                             gemm_out_t c_type, cudaStream_t stream);
+
 /* Synchronises `stream`, then reports and clears the device watchdog status
  * of the current device: GEMM_OK, or GEMM_ERR_TIMEOUT if a kernel's bounded
  * wait expired since the last check.  GEMM_ERR_LAUNCH if the stream itself

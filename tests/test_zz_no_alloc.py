@@ -1,0 +1,82 @@
+"""gemm_bf16_noalloc, the entry point for callers that cannot allocate device
+memory (a framework's caching allocator owns the device, allocator callbacks
+must not re-enter it, or cudaMalloc's implicit synchronisation is not
+allowed).  Its kernels keep their scratch in a static array inside the
+library instead of cudaMalloc'd memory.
+
+This file is collected last on purpose: it must pass both alone in a fresh
+process and after every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dense_gemm_engineering_bf16_b200 import gemm as G
+from dense_gemm_engineering_bf16_b200 import synth
+
+from gpu_helpers import tolerance, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+# two calls in a row: different shapes through the same kernel instantiation,
+# so the second call cannot trigger a first-use kernel load
+CASES = [(300, 200, 136, G.OUT_F32), (777, 1030, 1000, G.OUT_F32)]
+
+
+def _decode(c, c_type):
+    if c_type == G.OUT_F32:
+        return c.cpu().numpy().astype(np.float64)
+    return oracle.decode_bf16(c.cpu().view(torch.int16).numpy().view(np.uint16))
+
+
+def test_noalloc_matches_gemm_bf16_on_two_calls_in_a_row():
+    G.gemm_force_config("auto")
+    prepared = []
+    for i, (M, N, K, c_type) in enumerate(CASES):
+        lda = K + (-K % 8)
+        a_bits, b_bits = synth.bf16_operands(M, N, K, "normal", workload=70 + i, lda=lda, ldb=lda)
+        dt = torch.float32 if c_type == G.OUT_F32 else torch.bfloat16
+        ldc = N + (-N % 8)
+        prepared.append(dict(M=M, N=N, K=K, c_type=c_type, lda=lda, ldc=ldc, a=a_bits, b=b_bits,
+                             A=to_device_bf16(a_bits), B=to_device_bf16(b_bits),
+                             C_na=torch.full((M, ldc), float("nan"), dtype=dt, device="cuda"),
+                             C_ref=torch.full((M, ldc), float("nan"), dtype=dt, device="cuda")))
+    torch.cuda.synchronize()
+
+    # the allocation-free entry point, twice in a row; the second call must
+    # not change the device's free memory (any cudaMalloc takes >= 2 MiB)
+    free_before = None
+    for i, p in enumerate(prepared):
+        if i == 1:
+            torch.cuda.synchronize()
+            free_before = torch.cuda.mem_get_info()[0]
+        G.gemm_bf16_noalloc(p["A"], p["B"], p["C_na"], p["M"], p["N"], p["K"], p["lda"], p["lda"],
+                            p["ldc"], p["c_type"])
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free_before
+
+    # the existing entry point on the same inputs
+    for p in prepared:
+        G.gemm_bf16(p["A"], p["B"], p["C_ref"], p["M"], p["N"], p["K"], p["lda"], p["lda"],
+                    p["ldc"], p["c_type"])
+    G.gemm_check_device_status()
+
+    for p in prepared:
+        M, N, K = p["M"], p["N"], p["K"]
+        got = _decode(p["C_na"], p["c_type"])
+        ref = _decode(p["C_ref"], p["c_type"])
+        assert np.isnan(got[:, N:]).all(), "wrote past column N"
+        got, ref = got[:, :N], ref[:, :N]
+        c64, s_abs = oracle.gemm_bf16_f64(p["a"], p["b"], K=K, with_abs=True)
+        tol = tolerance(c64, s_abs, p["c_type"])
+        assert np.all(np.abs(got - ref) <= tol), f"{M}x{N}x{K}: differs from gemm_bf16"
+        assert np.all(np.abs(got - c64) <= tol), f"{M}x{N}x{K}: outside the oracle tolerance"
+
+
+def test_noalloc_argument_checks_match():
+    ptr = 0x7F0000000000
+    for args in [(-1, 8, 8, 8, 8, 8, 0), (8, 8, 8, 4, 8, 8, 0), (8, 8, 8, 8, 8, 8, 9)]:
+        M, N, K, lda, ldb, ldc, ct = args
+        assert G.lib.gemm_bf16_noalloc(ptr, ptr + 4096, ptr + 8192, M, N, K, lda, ldb, ldc, ct, 0) == \
+            G.lib.gemm_bf16(ptr, ptr + 4096, ptr + 8192, M, N, K, lda, ldb, ldc, ct, 0)
