@@ -209,6 +209,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="square8192", choices=sorted(WORKLOADS))
+    ap.add_argument("--shape", type=int, nargs=3, metavar=("M", "N", "K"),
+                    help="override the workload's shape (bf16 U[-1,1] inputs), e.g. for profiling")
     ap.add_argument("--config", default="auto")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -234,6 +236,10 @@ def main():
                                 device_id=torch.device("cuda", local))
 
     M, N, K, distname, wid, desc = WORKLOADS[args.workload]
+    if args.shape:
+        M, N, K = args.shape
+        distname, wid = "uniform", 90
+        desc = f"gemm {M}x{N}x{K}, bf16 U[-1,1] in, fp32 out"
     a_bits, b_bits = synth.bf16_operands(M, N, K, distname, workload=wid, base=rank)
     A = torch.from_numpy(a_bits.view(np.int16)).cuda().view(torch.bfloat16)
     B = torch.from_numpy(b_bits.view(np.int16)).cuda().view(torch.bfloat16)
@@ -281,10 +287,23 @@ def main():
         t = torch.tensor([t_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         t_ms = float(t.item())
-    value = world * args.steps * flops / (t_ms * 1e-3) / 1e12
-
     # ------------------------------------------- end to end, host buffers --
-    e2e_steps = max(1, args.e2e_steps)
+    e2e_steps = args.e2e_steps
+    e2e_value = None
+    if e2e_steps > 0:
+        e2e_value = run_e2e(torch, dist, G, a_bits, b_bits, A, B, C, M, N, K, flops, e2e_steps,
+                            stream, world, barrier)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    _report(args, G, M, N, K, desc, cfg_name, flops, in_out_bytes, world, t_ms, per_launch_ms,
+            sampler, e2e_value, e2e_steps, a_bits, b_bits)
+
+
+def run_e2e(torch, dist, G, a_bits, b_bits, A, B, C, M, N, K, flops, e2e_steps, stream, world, barrier):
+    """Same metric through the C ABI with pinned host buffers: H2D of A and B,
+    the GEMM, D2H of C, all inside the timed region."""
     A_h = torch.from_numpy(a_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     B_h = torch.from_numpy(b_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     C_h = torch.empty((M, N), dtype=torch.float32).pin_memory()
@@ -314,13 +333,12 @@ def main():
         e2e_ms = float(t.item())
     barrier()
     G.gemm_check_device_status(stream)
-    e2e_value = world * e2e_steps * flops / (e2e_ms * 1e-3) / 1e12
+    return world * e2e_steps * flops / (e2e_ms * 1e-3) / 1e12
 
-    if world > 1:
-        dist.destroy_process_group()
-    if rank != 0:
-        return
 
+def _report(args, G, M, N, K, desc, cfg_name, flops, in_out_bytes, world, t_ms, per_launch_ms,
+            sampler, e2e_value, e2e_steps, a_bits, b_bits):
+    value = world * args.steps * flops / (t_ms * 1e-3) / 1e12
     # ------------------------------------------------------------ roofline --
     peaks, peak_src = load_peaks()
     mean_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
@@ -352,8 +370,9 @@ def main():
                    if in_out_bytes > L2_BYTES else "inputs fit in L2 (not flushed)",
                    "launch_ms_median": statistics.median(per_launch_ms),
                    "launch_ms_p90": float(np.percentile(per_launch_ms, 90))},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * (M * K + N * K),
-                "d2h_bytes_per_step": 4 * M * N, "steps": e2e_steps},
+        "e2e": None if e2e_value is None else
+        {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * (M * K + N * K),
+         "d2h_bytes_per_step": 4 * M * N, "steps": e2e_steps},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clocks,
