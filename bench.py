@@ -376,7 +376,7 @@ def _report(args, G, M, N, K, desc, cfg_name, flops, in_out_bytes, world, t_ms, 
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clocks,
-        "gpu_launches": args.steps * G.gemm_launches_per_call(M, N, K) * world,
+        "gpu_launches": args.steps * G.gemm_launches_per_call(M, N, K, False) * world,
     }
     print(json.dumps(line), flush=True)
 

@@ -15,6 +15,7 @@
 
 #include "b200gemm.h"
 #include "gemm_bf16_sm100.cuh"
+#include "gemm_mxfp8_sm100.cuh"
 
 namespace {
 
@@ -28,6 +29,7 @@ using Cfg1x128F32 = b200::GemmBf16Cfg<1, 128, 6, 0>;
 using Cfg1x128B16 = b200::GemmBf16Cfg<1, 128, 6, 1>;
 using Cfg2x256F32 = b200::GemmBf16Cfg<2, 256, 6, 0>;
 using Cfg2x256B16 = b200::GemmBf16Cfg<2, 256, 6, 1>;
+using CfgMxf8 = b200::GemmMxf8Cfg<3>;
 
 constexpr int kMaxDevices = 64;
 
@@ -39,6 +41,10 @@ struct DeviceState {
     // per (config, out type): smem attribute set, co-resident clusters
     bool attr_done[GEMM_CFG_COUNT_][2] = {};
     int max_clusters[GEMM_CFG_COUNT_][2] = {};
+    // block-scaled path: kernel attribute set, repacked-scale workspace
+    bool mx_attr_done = false;
+    uint8_t *mx_ws = nullptr;
+    size_t mx_ws_bytes = 0;
 };
 
 std::mutex g_mutex;
@@ -297,6 +303,85 @@ gemm_status_t noalloc_device(int &dev, DeviceState *&st) {
     return st->supported ? GEMM_OK : GEMM_ERR_UNSUPPORTED_DEVICE;
 }
 
+// ------------------------------------------------------ block-scaled path --
+
+// Bytes of repacked scales for an M x N x K problem: 512 per (128-row block,
+// 128-wide K block) of A, and of B padded to whole 256-row tiles.
+size_t mx_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    const int64_t kb = (K + 127) / 128;
+    const int64_t a_blocks = (M + 127) / 128;
+    const int64_t b_blocks = 2 * ((N + 255) / 256);
+    return static_cast<size_t>((a_blocks + b_blocks) * kb * 512);
+}
+
+// Grows the device's workspace on demand.  cudaFree waits for the device to
+// go idle, so work still using the old buffer has finished before it goes.
+gemm_status_t mx_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (st->mx_ws_bytes < bytes) {
+        cudaError_t e;
+        if (st->mx_ws) {
+            if ((e = cudaFree(st->mx_ws)) != cudaSuccess) return cuda_fail(e);
+            st->mx_ws = nullptr;
+            st->mx_ws_bytes = 0;
+        }
+        const size_t want = bytes < (size_t(1) << 20) ? (size_t(1) << 20) : bytes;
+        if ((e = cudaMalloc(&st->mx_ws, want)) != cudaSuccess) return cuda_fail(e);
+        st->mx_ws_bytes = want;
+    }
+    ws = st->mx_ws;
+    return GEMM_OK;
+}
+
+gemm_status_t launch_mxf8(DeviceState *st, const void *A, const uint8_t *sfa, const void *B,
+                          const uint8_t *sfb, void *C, int64_t M, int64_t N, int64_t K, int64_t lda,
+                          int64_t ldb, int64_t ldc, cudaStream_t stream) {
+    using Cfg = CfgMxf8;
+    auto kernel = b200::gemm_mxf8_sm100_kernel<Cfg>;
+    cudaError_t e;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!st->mx_attr_done) {
+            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          Cfg::SMEM_BYTES)) != cudaSuccess)
+                return cuda_fail(e);
+            st->mx_attr_done = true;
+        }
+    }
+    uint8_t *ws = nullptr;
+    gemm_status_t s;
+    if ((s = mx_workspace(st, mx_workspace_bytes(M, N, K), ws)) != GEMM_OK) return s;
+    const int64_t kb = (K + 127) / 128;
+    const int64_t a_blocks = (M + 127) / 128;
+    const int64_t b_blocks = 2 * ((N + 255) / 256);
+
+    // 1. scales -> TMEM-ready 512-byte chunks
+    const int64_t words = (a_blocks + b_blocks) * kb * 128;
+    int64_t blocks = (words + 255) / 256;
+    if (blocks > static_cast<int64_t>(st->sm_count) * 16) blocks = static_cast<int64_t>(st->sm_count) * 16;
+    b200::mxf8_repack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        sfa, M, a_blocks, sfb, N, b_blocks, K / 32, kb, reinterpret_cast<uint32_t *>(ws));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+
+    // 2. the block-scaled GEMM
+    alignas(64) CUtensorMap tmA, tmB, tmC;
+    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, lda, Cfg::BK, Cfg::BM)) != GEMM_OK) return s;
+    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, ldb, Cfg::BK, Cfg::BN)) != GEMM_OK) return s;
+    const int64_t n_tma = (N * 2 / 16) * 16 / 2;
+    if ((s = encode_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, n_tma > 0 ? n_tma : 8, M, ldc * 2,
+                       Cfg::EPI_COLS, 32)) != GEMM_OK)
+        return s;
+    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
+    const int64_t grid = tiles < st->sm_count ? tiles : st->sm_count;
+    const uint8_t *sfa_chunks = ws;
+    const uint8_t *sfb_chunks = ws + a_blocks * kb * 512;
+    kernel<<<static_cast<unsigned>(grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+        tmA, tmB, tmC, sfa_chunks, sfb_chunks, static_cast<int>(M), static_cast<int>(N),
+        static_cast<int>(K), C, ldc, static_cast<int>(n_tma), st->status, watchdog_ns(K));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    return GEMM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -329,6 +414,25 @@ gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_
         default:
             return GEMM_ERR_INVALID_VALUE;
     }
+}
+
+gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const uint8_t *sfb, void *C,
+                         int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                         cudaStream_t stream) {
+    gemm_status_t s = check_args(A, B, C, M, N, K, lda, ldb, ldc, 1, 1, 2);
+    if (s != GEMM_OK || M == 0 || N == 0) return s;
+    if (K % 32) return GEMM_ERR_INVALID_VALUE;
+    if (K > 0) {
+        if (!sfa || !sfb) return GEMM_ERR_INVALID_VALUE;
+        if (overlaps(C, M, N, ldc, 2, sfa, 1, M * (K / 32), M * (K / 32), 1) ||
+            overlaps(C, M, N, ldc, 2, sfb, 1, N * (K / 32), N * (K / 32), 1))
+            return GEMM_ERR_ALIAS;
+    }
+    int dev;
+    DeviceState *st;
+    if ((s = current_device(dev, st)) != GEMM_OK) return s;
+    if (K == 0) return launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
+    return launch_mxf8(st, A, sfa, B, sfb, C, M, N, K, lda, ldb, ldc, stream);
 }
 
 gemm_status_t gemm_check_device_status(cudaStream_t stream) {
@@ -380,9 +484,9 @@ gemm_status_t gemm_force_config(gemm_config_t config) {
 
 gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K) { return select_config(M, N, K); }
 
-int gemm_launches_per_call(int64_t M, int64_t N, int64_t K) {
-    (void)K;
-    return (M > 0 && N > 0) ? 1 : 0;
+int gemm_launches_per_call(int64_t M, int64_t N, int64_t K, int block_scaled) {
+    if (M <= 0 || N <= 0) return 0;
+    return (block_scaled && K > 0) ? 2 : 1;
 }
 
 gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,

@@ -1,0 +1,327 @@
+// Block-scaled MXFP8 GEMM for sm_100a:
+//
+//   C[i][j] = sum_k (a_ik 2^(sfa[i][k/32]-127)) (b_kj 2^(sfb[j][k/32]-127))
+//
+// with FP8 E4M3 A (M x K) and K-major B (N x K), one E8M0 scale per 32
+// consecutive K elements of every row, fp32 accumulation in TMEM and bf16 C.
+// This is the block-scaled MMA of "Modern GPU Programming For MLSys - 书籍总结"
+// (omica.com.cn), sections 2.4 and 2.6: the scale factors live in tensor
+// memory and the tensor core applies them inside the MMA.
+//
+// Two kernels:
+//   mxf8_repack_scales_kernel  turns the row-major scale bytes into 512-byte
+//       chunks, one per (128-row block, 128-wide K block), laid out the way
+//       tcgen05.cp 32x128b.warpx4 places them in TMEM: chunk byte
+//       r*16 + q*4 + j holds the scale of row 32q + r for the j-th 32-wide
+//       K step.  Padding rows and K steps get 127 (2^0), so zero-filled
+//       operand tails stay zero.
+//   gemm_mxf8_sm100_kernel  persistent, warp-specialised, one CTA per
+//       128 x 256 tile, BK = 128 (one 128-byte swizzle row of E4M3):
+//       warp 0 loads A and B by TMA and the scale chunks by 1-D bulk copy;
+//       warp 1 copies the stage's scales into TMEM (tcgen05.cp, two slots
+//       alternating) and issues 4 block-scaled MMAs (K = 32 each, the byte of
+//       the scale column chosen in the instruction descriptor); warps 2-5
+//       drain the accumulator as bf16 into a full-tile swizzled staging area,
+//       release TMEM at once, and write C with TMA stores.
+//
+// TMEM: accumulator columns [0, 256); scale slot s at 256 + 32 s (A: 4
+// columns) and 256 + 32 s + 16 (B: 8 columns).  Every scale sits in lane
+// (row % 32) of each 32-lane quarter, column (row / 32), byte j.
+#pragma once
+#include <cstdint>
+
+#include "gemm_bf16_sm100.cuh"
+#include "ptx.cuh"
+
+namespace b200 {
+
+template <int STAGES_>
+struct GemmMxf8Cfg {
+    static constexpr int STAGES = STAGES_;
+    static constexpr int BM = 128;
+    static constexpr int BN = 256;
+    static constexpr int BK = 128;                 // E4M3 elements (bytes) per k-tile
+    static constexpr int UMMA_K = 32;              // K per block-scaled MMA
+    static constexpr int MMAS = BK / UMMA_K;       // 4, one scale byte each
+    static constexpr int A_BYTES = BM * BK;
+    static constexpr int B_BYTES = BN * BK;
+    static constexpr int SF_CHUNK = 512;           // scales of 128 rows x 4 K steps
+    static constexpr int SFA_BYTES = SF_CHUNK;
+    static constexpr int SFB_BYTES = 2 * SF_CHUNK;
+    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGE_BYTES = ((TX_BYTES + 1023) / 1024) * 1024;
+    static constexpr int EPI_COLS = 64;            // bf16 columns per 128-byte staged row
+    static constexpr int EPI_CHUNKS = BN / EPI_COLS;
+    static constexpr int EPI_BUF = 32 * 128;       // one 32-row x 128-byte box
+    static constexpr int EPI_BYTES = 4 * EPI_CHUNKS * EPI_BUF;  // each warp stages its whole 32 x 256 slice
+    static constexpr int NUM_BARS = 2 * STAGES + 2;
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SF_COL0 = 256;
+    static constexpr int THREADS = 192;
+    static constexpr int GROUP_M = 8;
+    static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
+};
+
+// Row-major scales [rows][K/32] -> chunks [row block][K block][512], for
+// a_blocks row blocks of A followed by b_blocks row blocks of B; rows past
+// M (or N) and K steps past k32 read as 127.  One thread per 32-bit word.
+__global__ void mxf8_repack_scales_kernel(const uint8_t *__restrict__ sfa, int64_t M, int64_t a_blocks,
+                                          const uint8_t *__restrict__ sfb, int64_t N, int64_t b_blocks,
+                                          int64_t k32, int64_t kblocks, uint32_t *__restrict__ out) {
+    const int64_t words_per_chunk = 128;
+    const int64_t total = (a_blocks + b_blocks) * kblocks * words_per_chunk;
+    for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < total;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t chunk = w / words_per_chunk;
+        const int64_t word = w - chunk * words_per_chunk;     // = r * 4 + q
+        const int64_t r = word >> 2;
+        const int64_t q = word & 3;
+        int64_t rb = chunk / kblocks;
+        const int64_t kb = chunk - rb * kblocks;
+        const uint8_t *src = sfa;
+        int64_t rows = M;
+        if (rb >= a_blocks) {
+            rb -= a_blocks;
+            src = sfb;
+            rows = N;
+        }
+        const int64_t row = rb * 128 + q * 32 + r;
+        uint32_t v = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t ks = kb * 4 + j;
+            const uint32_t byte = (row < rows && ks < k32) ? src[row * k32 + ks] : 127u;
+            v |= byte << (8 * j);
+        }
+        out[w] = v;
+    }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC, const uint8_t *sfa_chunks,
+                       const uint8_t *sfb_chunks, int M, int N, int K, void *C, int64_t ldc, int n_tma,
+                       DeviceStatus *status, uint64_t timeout_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    const uint32_t base = smem_addr(smem);
+    const uint32_t warp = threadIdx.x / 32;
+    const uint32_t lane = threadIdx.x % 32;
+
+    const uint32_t bar0 = base + Cfg::BAR_OFF;
+    auto full_bar = [&](uint32_t s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](uint32_t s) { return bar0 + 8u * (Cfg::STAGES + s); };
+    const uint32_t tfull_bar = bar0 + 8u * (2 * Cfg::STAGES);
+    const uint32_t tempty_bar = tfull_bar + 8u;
+    const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
+    const uint32_t abort_slot = tmem_slot + 4u;
+    volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
+    volatile uint32_t *abort_flag = tmem_slot_ptr + 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(tfull_bar, 1);
+        mbar_init(tempty_bar, 4);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB);
+        tma_prefetch_map(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc<1>(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish<1>();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot_ptr;
+
+    const int num_m = (M + Cfg::BM - 1) / Cfg::BM;
+    const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + Cfg::BK - 1) / Cfg::BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                int tm, tn;
+                raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+                const uint8_t *sfa_row = sfa_chunks + static_cast<int64_t>(tm) * num_kb * Cfg::SF_CHUNK;
+                const uint8_t *sfb_row0 = sfb_chunks + static_cast<int64_t>(2 * tn) * num_kb * Cfg::SF_CHUNK;
+                const uint8_t *sfb_row1 = sfb_row0 + static_cast<int64_t>(num_kb) * Cfg::SF_CHUNK;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarEmpty);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = base + stage * Cfg::STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + Cfg::A_BYTES;
+                    const uint32_t sfa_dst = b_dst + Cfg::B_BYTES;
+                    const uint32_t sfb_dst = sfa_dst + Cfg::SFA_BYTES;
+                    const uint32_t fb = full_bar(stage);
+                    mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
+                    tma_load_2d(a_dst, &tmA, fb, kb * Cfg::BK, tm * Cfg::BM);
+                    tma_load_2d(b_dst, &tmB, fb, kb * Cfg::BK, tn * Cfg::BN);
+                    const int64_t off = static_cast<int64_t>(kb) * Cfg::SF_CHUNK;
+                    bulk_load_1d(sfa_dst, sfa_row + off, Cfg::SF_CHUNK, fb);
+                    bulk_load_1d(sfb_dst, sfb_row0 + off, Cfg::SF_CHUNK, fb);
+                    bulk_load_1d(sfb_dst + Cfg::SF_CHUNK, sfb_row1 + off, Cfg::SF_CHUNK, fb);
+                    if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            for (int i = 0; ok && i < Cfg::STAGES; ++i) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarTail);
+                    ok = false;
+                }
+                if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------- scale copy + MMA issuer --
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, sf_slot = 0;
+            bool ok = true;
+            int t = 0;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++t) {
+                if (!mbar_wait(tempty_bar, (static_cast<uint32_t>(t) & 1u) ^ 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarTmemEmpty);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarFull);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a0 = base + stage * Cfg::STAGE_BYTES;
+                    const uint32_t b0 = a0 + Cfg::A_BYTES;
+                    const uint32_t sfa_smem = b0 + Cfg::B_BYTES;
+                    const uint32_t sfb_smem = sfa_smem + Cfg::SFA_BYTES;
+                    const uint32_t sfa_t = tmem_base + Cfg::SF_COL0 + 32u * sf_slot;
+                    const uint32_t sfb_t = sfa_t + 16u;
+                    // tcgen05.cp and tcgen05.mma issued by one thread execute in
+                    // issue order, so the MMAs below see these scales.
+                    tmem_cp_32x128b_warpx4(sfa_t, rows16_desc(sfa_smem));
+                    tmem_cp_32x128b_warpx4(sfb_t, rows16_desc(sfb_smem));
+                    tmem_cp_32x128b_warpx4(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+#pragma unroll
+                    for (int j = 0; j < Cfg::MMAS; ++j) {
+                        mma_mxf8_ss(tmem_base, sw128_kmajor_desc(a0 + j * 32), sw128_kmajor_desc(b0 + j * 32),
+                                    idesc_mxf8_e8m0(Cfg::BM, Cfg::BN, static_cast<uint32_t>(j),
+                                                    static_cast<uint32_t>(j)),
+                                    sfa_t, sfb_t, (kb | j) != 0 ? 1u : 0u);
+                    }
+                    mma_commit<1>(empty_bar(stage), 0);
+                    sf_slot ^= 1u;
+                    if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit<1>(tfull_bar, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------- epilogue --
+        const uint32_t sub = warp & 3u;
+        const uint32_t ew = warp - 2u;
+        const uint32_t sbuf = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * Cfg::EPI_CHUNKS * Cfg::EPI_BUF;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+            int tm, tn;
+            raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+            uint32_t ready = 1;
+            if (lane == 0 && !mbar_wait(tfull_bar, static_cast<uint32_t>(t) & 1u, abort_flag, timeout_ns)) {
+                record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
+                ready = 0;
+            }
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
+            tc_fence_after_sync();
+            // Drain the accumulator into this warp's staging slice (four
+            // 32 x 128-byte boxes, 128-byte swizzle), then hand TMEM back so
+            // the next tile's MMAs start while the stores drain.
+            const uint32_t tbase = tmem_base + ((sub * 32u) << 16);
+            const int row0 = tm * Cfg::BM + static_cast<int>(sub) * 32;
+            const int col0 = tn * Cfg::BN;
+            const int row = row0 + static_cast<int>(lane);
+            if (lane == 0) bulk_wait_group_read<0>();   // last tile's stores are done reading
+            __syncwarp();
+#pragma unroll 1
+            for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
+                uint32_t v0[32], v1[32], packed[32];
+                tmem_ld_32x32b_x32(tbase + c * 64, v0);
+                tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+                    packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+                }
+                const int cstart = col0 + c * Cfg::EPI_COLS;
+                if (cstart < N && cstart + Cfg::EPI_COLS > n_tma && row < M) {
+                    // the row's last partial 16-byte granule: plain stores
+                    uint16_t *crow = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(C) +
+                                                                  static_cast<int64_t>(row) * ldc * 2);
+#pragma unroll
+                    for (int w = 0; w < Cfg::EPI_COLS; ++w) {
+                        const int col = cstart + w;
+                        if (col >= n_tma && col < N)
+                            crow[col] = static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
+                    }
+                }
+                const uint32_t row_addr = sbuf + c * Cfg::EPI_BUF + lane * 128u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4),
+                                 packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                }
+            }
+            tc_fence_before_sync();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_local(tempty_bar);
+                for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
+                    const int cstart = col0 + c * Cfg::EPI_COLS;
+                    if (cstart < n_tma) tma_store_2d(&tmC, sbuf + c * Cfg::EPI_BUF, cstart, row0);
+                }
+                bulk_commit_group();
+            }
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc<1>(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace b200

@@ -245,6 +245,33 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 1-D bulk copy global -> this CTA's shared memory, completion counted in
+// bytes on `bar`.  Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Shared memory -> TMEM copy of 32 rows x 128 bits, written to lanes 0-31 of
+// every 32-lane quarter (warpx4 broadcast): 4 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
+// Block-scaled MMA, FP8 E4M3 x E4M3 with one E8M0 scale per 32 K elements,
+// f32 accumulator in TMEM; scale factors read from TMEM.
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate),
+                   "r"(sfa_tmem), "r"(sfb_tmem)
+                 : "memory");
+}
+
 // ------------------------------------------------------------ descriptors --
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
@@ -273,6 +300,29 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) |
            (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Descriptor of an unswizzled K-major block of rows of 16 bytes (the
+// scale-factor chunk read by tcgen05.cp 32x128b): core matrices of 8 rows x
+// 16 bytes (128 contiguous bytes), stacked along the rows every 128 bytes
+// (stride byte offset), one 16-byte unit along K (leading byte offset unused),
+// version 1, no swizzle.
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t smem) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(128 >> 4) << 16;
+    d |= static_cast<uint64_t>(128 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    return d;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A and B E4M3 (format
+// 0, bits 7-9 / 10-12), K-major, N >> 3 (17-22), scale format E8M0 (bit 23),
+// M >> 4 (24-28), and which byte of the 32-bit scale column each operand's
+// scales come from: B (bits 4-5), A (bits 29-30).  Dense, K = 32 per MMA.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e8m0(int m, int n, uint32_t a_sf_id, uint32_t b_sf_id) {
+    return (b_sf_id << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(m >> 4) << 24) | (a_sf_id << 29);
 }
 
 // ----------------------------------------------------------- conversions --

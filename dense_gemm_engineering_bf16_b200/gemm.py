@@ -44,6 +44,8 @@ lib.gemm_bf16.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _in
 lib.gemm_bf16.restype = _int
 lib.gemm_bf16_noalloc.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp]
 lib.gemm_bf16_noalloc.restype = _int
+lib.gemm_mxfp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]
+lib.gemm_mxfp8.restype = _int
 lib.gemm_check_device_status.argtypes = [_vp]
 lib.gemm_check_device_status.restype = _int
 lib.gemm_last_timeout_detail.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
@@ -56,7 +58,7 @@ lib.gemm_force_config.argtypes = [_int]
 lib.gemm_force_config.restype = _int
 lib.gemm_select_config.argtypes = [_i64, _i64, _i64]
 lib.gemm_select_config.restype = _int
-lib.gemm_launches_per_call.argtypes = [_i64, _i64, _i64]
+lib.gemm_launches_per_call.argtypes = [_i64, _i64, _i64, _int]
 lib.gemm_launches_per_call.restype = _int
 
 
@@ -107,6 +109,15 @@ def gemm_bf16(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
     return _check(st, "gemm_bf16", check)
 
 
+def gemm_mxfp8(A, sfa, B, sfb, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
+               stream=None, check: bool = True) -> int:
+    """Block-scaled C = (sa.A).(sb.B): E4M3 A (M x lda bytes), E4M3 B stored
+    N x ldb, E8M0 scales sfa (M x K/32) and sfb (N x K/32), bf16 C (M x ldc)."""
+    st = lib.gemm_mxfp8(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(C), M, N, K, lda, ldb, ldc,
+                        _stream(stream))
+    return _check(st, "gemm_mxfp8", check)
+
+
 def gemm_bf16_noalloc(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
                       c_type: int = OUT_F32, stream=None, check: bool = True) -> int:
     """gemm_bf16 without any device allocation: the kernels' scratch is a
@@ -137,5 +148,5 @@ def gemm_select_config(M: int, N: int, K: int) -> int:
     return int(lib.gemm_select_config(M, N, K))
 
 
-def gemm_launches_per_call(M: int, N: int, K: int) -> int:
-    return int(lib.gemm_launches_per_call(M, N, K))
+def gemm_launches_per_call(M: int, N: int, K: int, block_scaled: bool = False) -> int:
+    return int(lib.gemm_launches_per_call(M, N, K, int(bool(block_scaled))))

@@ -98,6 +98,35 @@ B200GEMM_API gemm_status_t gemm_bf16(const void *A, const void *B, void *C,
                         gemm_out_t c_type, cudaStream_t stream);
 
 /*
+ * gemm_mxfp8: block-scaled C = (sa . A) . (sb . B) with FP8 E4M3 A and B and
+ * one E8M0 scale per 32 consecutive K elements of every row of A and of the
+ * K-major B -- the block-scaled MMA with its scale factors in tensor memory
+ * of "Modern GPU Programming For MLSys - 书籍总结", sections 2.4 and 2.6:
+ *
+ *   C[i][j] = sum_k (a_ik 2^(sfa[i][k/32]-127)) (b_kj 2^(sfb[j][k/32]-127))
+ *
+ * fp32 accumulation, C written as bf16 (round to nearest even).
+ *   A   M x lda bytes of E4M3 codes (row i, element k at A[i*lda + k])
+ *   B   N x ldb bytes of E4M3 codes (stored K-major: b(k,j) at B[j*ldb + k])
+ *   sfa M x (K/32) E8M0 bytes, rows packed: sfa[i*(K/32) + k/32]
+ *   sfb N x (K/32) E8M0 bytes, rows packed: sfb[j*(K/32) + k/32]
+ *   C   M x ldc bf16
+ * K must be a multiple of 32; lda and ldb multiples of 16; ldc*2 a multiple
+ * of 16; A, B and C 16-byte aligned (the scales need no alignment).  C must
+ * not overlap A, B, sfa or sfb.  M == 0 or N == 0: nothing to do; K == 0:
+ * C = 0.  An E8M0 byte 0xFF (NaN) makes its block NaN.
+ * Each call queues two kernels: a repack of the scales into a per-device
+ * workspace of 512 bytes per (128 rows x 128 K) block of A and of B, which
+ * the library allocates on first use and grows when a larger problem needs
+ * it (cudaMalloc; growing waits for the device to go idle), then the GEMM.
+ * Calls on streams that are not ordered with each other share that
+ * workspace and must not overlap.
+ */
+B200GEMM_API gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const uint8_t *sfb,
+                                      void *C, int64_t M, int64_t N, int64_t K,
+                                      int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream);
+
+/*
  * gemm_bf16_noalloc: gemm_bf16 for callers that cannot allocate device memory.
  * (No counterpart in the pages: it is a packaging choice of this library.)
  *
@@ -152,9 +181,10 @@ B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
 /* The configuration the next gemm_bf16 call with this shape would use. */
 B200GEMM_API gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K);
 
-/* Number of kernels that gemm_bf16 / gemm_mxfp8 queue per call for this
- * shape (0 for an empty problem). */
-B200GEMM_API int gemm_launches_per_call(int64_t M, int64_t N, int64_t K);
+/* Number of kernels that one call queues for this shape: gemm_bf16 /
+ * gemm_bf16_noalloc (block_scaled = 0) or gemm_mxfp8 (block_scaled = 1);
+ * 0 for an empty problem. */
+B200GEMM_API int gemm_launches_per_call(int64_t M, int64_t N, int64_t K, int block_scaled);
 
 #ifdef __cplusplus
 }

@@ -129,3 +129,23 @@ def sample_indices(n: int, tile: int, extra: int, seed: int) -> np.ndarray:
     rng = np.random.default_rng(seed + 1)
     extra_idx = rng.integers(0, n, size=extra).tolist()
     return np.array(sorted(set(idx) | set(extra_idx)), dtype=np.int64)
+
+
+def run_mxfp8(a_codes: np.ndarray, sfa: np.ndarray, b_codes: np.ndarray, sfb: np.ndarray,
+              M: int, N: int, K: int, ldc: int | None = None):
+    """Run the block-scaled GEMM through the C ABI; returns the GuardedC (bf16)."""
+    lda = a_codes.shape[1] if a_codes.size else 16
+    ldb = b_codes.shape[1] if b_codes.size else 16
+    if ldc is None:
+        ldc = N + (-N % 8)
+
+    def dev(x):
+        x = np.ascontiguousarray(x, dtype=np.uint8)
+        return torch.from_numpy(x).cuda() if x.size else torch.empty(16, dtype=torch.uint8, device="cuda")
+
+    A, B, SA, SB = dev(a_codes), dev(b_codes), dev(sfa), dev(sfb)
+    C = GuardedC(M, N, ldc, G.OUT_BF16)
+    G.gemm_mxfp8(A, SA, B, SB, C.ptr, M, N, K, lda, ldb, ldc)
+    G.gemm_check_device_status()
+    torch.cuda.synchronize()
+    return C

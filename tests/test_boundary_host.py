@@ -67,12 +67,25 @@ def test_rejects_bad_arguments_before_any_launch():
     assert _call(C_=B) == 3                         # C overlaps B
 
 
+def test_mxfp8_rejects_bad_arguments_before_any_launch():
+    f = G.lib.gemm_mxfp8
+    sa, sb = 0x7F0000300000, 0x7F0000400000
+    assert f(A, sa, B, sb, C, 64, 64, 48, 48, 48, 64, 0) == 1          # K % 32
+    assert f(A, sa, B, sb, C, 64, 64, 64, 40, 64, 64, 0) == 1          # lda < K
+    assert f(A, sa, B, sb, C, 64, 64, 96, 104, 96, 64, 0) == 2         # lda not 16-byte multiple
+    assert f(A, 0, B, sb, C, 64, 64, 64, 64, 64, 64, 0) == 1           # null scales
+    assert f(A, sa, B, sb, sa, 64, 64, 64, 64, 64, 64, 0) == 3         # C overlaps sfa
+    assert f(A, sa, B, sb, C, 0, 64, 64, 64, 64, 64, 0) == 0           # empty
+
+
 def test_empty_problems_succeed_without_touching_memory():
     assert _call(M=0) == 0
     assert _call(N=0) == 0
     assert _call(M=0, A_=0, B_=0, C_=0) == 0
     assert G.gemm_launches_per_call(0, 5, 5) == 0
     assert G.gemm_launches_per_call(5, 5, 0) == 1
+    assert G.gemm_launches_per_call(5, 5, 64, block_scaled=True) == 2
+    assert G.gemm_launches_per_call(5, 5, 0, block_scaled=True) == 1
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
