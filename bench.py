@@ -1,25 +1,26 @@
 """Benchmark: bf16 GEMM TFLOP/s at 8192^3 on B200 (C = A.B, bf16 in, fp32 accumulate and out).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload square8192|square4096|ragged|skinny1000|skinny16]
+                    [--workload square8192|square4096|ragged|skinny1000|skinny16|mxfp8_8192]
+                    [--shape M N K] [--config auto|1cta_128x128|1cta_128x256|2cta_256x256]
 
-One step = one gemm_bf16 call over the whole M x N x K problem, inputs
+One step = one library call over the whole M x N x K problem with the inputs
 resident in HBM.  Multi-GPU runs (torchrun, one process per GPU) are
 independent replicas: every rank multiplies its own seeded matrices, no data
 crosses GPUs, and value = FLOPs of all ranks / the slowest rank's time.
 
 Printed (rank 0): one JSON line with the metric, the device-timed value,
-`e2e` (same metric through the C ABI with host buffers, copies included),
-`roofline` of the GEMM kernel, `cpu_baseline` (the CPU oracle on a bounded
-sample of the same workload), clocks sampled during the timed region and the
-number of kernel launches.  `--impl reference` times the oracle alone as the
-reference arm.
+`e2e` (the same metric through the C ABI with host buffers, copies inside
+the timed region), `roofline` of the GEMM kernel, `cpu_baseline` (the CPU
+oracle on a bounded sample of the same workload), clocks sampled during the
+timed region and the number of kernel launches.  `--impl reference` times
+the oracle alone, as the reference arm.
 """
 from __future__ import annotations
 
 import argparse
-import hashlib
 import glob
+import hashlib
 import json
 import os
 import statistics
@@ -33,19 +34,25 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "bf16 GEMM TFLOP/s at 8192³ on 1 B200 (fraction of dense BF16 tensor peak)"
+METRIC_MXFP8 = "MXFP8 block-scaled GEMM TFLOP/s at 8192³ on 1 B200"
 UNIT = "TFLOP/s"
 
+# name: (M, N, K, kind, distribution, workload id, description)
 WORKLOADS = {
-    # name: (M, N, K, distribution, workload id, description)
-    "square8192": (8192, 8192, 8192, "uniform", 3, "gemm 8192x8192x8192, bf16 U[-1,1] in, fp32 accumulate + out"),
-    "square4096": (4096, 4096, 4096, "normal_scaled", 2, "gemm 4096x4096x4096, bf16 N(0,1)/sqrt(K) in, fp32 out"),
-    "ragged": (4000, 3000, 2000, "normal", 4, "gemm 4000x3000x2000, bf16 N(0,1) in, fp32 out"),
-    "skinny1000": (1000, 8192, 8192, "normal", 5, "gemm 1000x8192x8192, bf16 N(0,1) in, fp32 out"),
-    "skinny16": (16, 8192, 8192, "normal", 6, "gemm 16x8192x8192, bf16 N(0,1) in, fp32 out"),
+    "square8192": (8192, 8192, 8192, "bf16", "uniform", 3,
+                   "gemm 8192x8192x8192, bf16 U[-1,1] in, fp32 accumulate + out"),
+    "square4096": (4096, 4096, 4096, "bf16", "normal_scaled", 2,
+                   "gemm 4096x4096x4096, bf16 N(0,1)/sqrt(K) in, fp32 out"),
+    "ragged": (4000, 3000, 2000, "bf16", "normal", 4, "gemm 4000x3000x2000, bf16 N(0,1) in, fp32 out"),
+    "skinny1000": (1000, 8192, 8192, "bf16", "normal", 5, "gemm 1000x8192x8192, bf16 N(0,1) in, fp32 out"),
+    "skinny16": (16, 8192, 8192, "bf16", "normal", 6, "gemm 16x8192x8192, bf16 N(0,1) in, fp32 out"),
+    "mxfp8_8192": (8192, 8192, 8192, "mxfp8", "uniform", 8,
+                   "block-scaled gemm 8192^3, E4M3 U[-1,1], E8M0 per 32 (exp U{-4..4}), bf16 out"),
 }
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 
 def kernel_source_hash() -> str:
@@ -60,8 +67,7 @@ def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            p = json.load(f)
-        return p, "measured"
+            return json.load(f), "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
 
@@ -69,9 +75,8 @@ def load_peaks():
 def profile_traffic(workload: str, config_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        with open(path) as f:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
@@ -81,6 +86,24 @@ def profile_traffic(workload: str, config_name: str):
     return entry.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------ multi-rank --
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The maximum of x over all ranks (x itself when world == 1)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step: float, steps: int, world: int, slowest_ms: float) -> float:
+    """Replicas: every rank did `steps` steps; the job took the slowest rank's time."""
+    return world * steps * flops_per_step / (slowest_ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle samples every 100 ms while running."""
 
@@ -88,7 +111,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str | None):
+    def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
         self.lines = []
@@ -116,44 +139,100 @@ class ClockSampler:
         self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return summarize_clocks(self.lines)
 
 
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.gpus > 1 and world == 1:
-        raise SystemExit("--gpus N > 1 needs torchrun: python -m torch.distributed.run "
-                         "--nproc-per-node N --master-addr 127.0.0.1 bench.py --gpus N")
-    return world, rank, local
+def summarize_clocks(lines):
+    """Median SM clock, max clock, median power and the throttle reasons seen."""
+    sm, smax, power, reasons = [], [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for name, val in zip(names, parts[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    # "under load": samples drawing at least 60 % of the highest power seen
+    # (the sampler brackets the timed region by a few hundred ms of idle)
+    pmax = max(power)
+    loaded = [i for i, pw in enumerate(power) if pw >= 0.6 * pmax] or list(range(len(sm)))
+    return {"sm_mhz": statistics.median(sm[i] for i in loaded), "sm_max_mhz": max(smax),
+            "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded),
+            "power_w_median_under_load": statistics.median(power[i] for i in loaded)}
 
 
-def oracle_sample(a_bits, b_bits, K, budget_s):
-    """Time the CPU oracle on the first R rows of A (all of B), R sized so
-    the run takes about budget_s.  Returns (flops, seconds, R)."""
-    import oracle
+# -------------------------------------------------------------- workloads --
+
+class Problem:
+    """Host operands of one workload and the library call that runs it."""
+
+    def __init__(self, name, shape, rank):
+        from dense_gemm_engineering_bf16_b200 import synth
+        M, N, K, kind, dist, wid, desc = WORKLOADS[name]
+        if shape:
+            M, N, K = shape
+            dist, wid = "uniform", 90
+            desc = (f"gemm {M}x{N}x{K}, bf16 U[-1,1] in, fp32 out" if kind == "bf16" else
+                    f"block-scaled gemm {M}x{N}x{K}, E4M3 U[-1,1], E8M0 per 32, bf16 out")
+        self.name, self.M, self.N, self.K, self.kind, self.desc = name, M, N, K, kind, desc
+        self.flops = 2.0 * M * N * K
+        if kind == "bf16":
+            self.a, self.b = synth.bf16_operands(M, N, K, dist, workload=wid, base=rank)
+            self.host = [self.a, self.b]
+            self.in_bytes = 2 * (M * K + N * K)
+            self.out_bytes = 4 * M * N
+        else:
+            self.a, self.sfa, self.b, self.sfb = synth.mxfp8_operands(M, N, K, workload=wid, base=rank)
+            self.host = [self.a, self.sfa, self.b, self.sfb]
+            self.in_bytes = M * K + N * K + (M + N) * (K // 32)
+            self.out_bytes = 2 * M * N
+
+    def device_arrays(self, torch):
+        if self.kind == "bf16":
+            return [torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) for x in self.host]
+        return [torch.from_numpy(np.ascontiguousarray(x)).cuda() for x in self.host]
+
+    def empty_out(self, torch, pinned=False):
+        dt = torch.float32 if self.kind == "bf16" else torch.bfloat16
+        if pinned:
+            return torch.empty((self.M, self.N), dtype=dt).pin_memory()
+        return torch.empty((self.M, self.N), dtype=dt, device="cuda")
+
+    def call(self, G, dev, C, stream):
+        M, N, K = self.M, self.N, self.K
+        if self.kind == "bf16":
+            A, B = dev
+            G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_F32, stream=stream)
+        else:
+            A, SA, B, SB = dev
+            G.gemm_mxfp8(A, SA, B, SB, C, M, N, K, K, K, N, stream=stream)
+
+    def launches(self, G):
+        return G.gemm_launches_per_call(self.M, self.N, self.K, self.kind == "mxfp8")
+
+    def oracle_rows(self, rows):
+        import oracle
+        if self.kind == "bf16":
+            return oracle.gemm_bf16_f64(self.a[:rows], self.b, K=self.K)
+        return oracle.gemm_mxfp8_f64(self.a[:rows], self.sfa[:rows], self.b, self.sfb, K=self.K)
+
+
+def oracle_sample(problem: Problem, budget_s: float):
+    """Time the CPU oracle on the first R rows of A (all of B), R sized so the
+    run takes about budget_s.  Returns (flops, seconds, R)."""
 
     def timed(rows):
         t0 = time.perf_counter()
-        oracle.gemm_bf16_f64(a_bits[:rows], b_bits, K=K)
+        problem.oracle_rows(rows)
         return time.perf_counter() - t0
 
     # each call decodes all of B once, then spends a fixed time per row of A:
@@ -161,42 +240,37 @@ def oracle_sample(a_bits, b_bits, K, budget_s):
     t4, t16 = timed(4), timed(16)
     per_row = max((t16 - t4) / 12.0, 1e-6)
     fixed = max(t4 - 4 * per_row, 0.0)
-    R = int(max(4, min(a_bits.shape[0], (budget_s - fixed) / per_row)))
-    t0 = time.perf_counter()
-    oracle.gemm_bf16_f64(a_bits[:R], b_bits, K=K)
-    dt = time.perf_counter() - t0
-    return 2.0 * R * b_bits.shape[0] * K, dt, R
+    R = int(max(4, min(problem.M, (budget_s - fixed) / per_row)))
+    dt = timed(R)
+    return 2.0 * R * problem.N * problem.K, dt, R
 
 
-def run_reference(args, world, rank):
+def run_reference(args, rank):
     """Reference arm: the CPU oracle, as it stands, on the host cores."""
     if rank != 0:
         return
     import oracle
-    from dense_gemm_engineering_bf16_b200 import synth
-    M, N, K, dist, wid, desc = WORKLOADS[args.workload]
-    a_bits, b_bits = synth.bf16_operands(M, N, K, dist, workload=wid)
-    # each step: a bounded row sample of the workload, sized so that all
-    # warm-up + timed steps take about two and a half minutes
+    p = Problem(args.workload, args.shape, 0)
+    # each step: a bounded row sample, sized so all warm-up + timed steps take
+    # about two and a half minutes
     per_step = max(0.05, min(2.0, 150.0 / (args.steps + args.warmup)))
-    _, _, R = oracle_sample(a_bits, b_bits, K, budget_s=per_step)
+    _, _, R = oracle_sample(p, per_step)
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        oracle.gemm_bf16_f64(a_bits[:R], b_bits, K=K)
-        dt = time.perf_counter() - t0
+        p.oracle_rows(R)
         if i >= args.warmup:
-            times.append(dt)
+            times.append(time.perf_counter() - t0)
     total = sum(times)
-    value = 2.0 * R * N * K * len(times) / total / 1e12
+    value = 2.0 * R * p.N * p.K * len(times) / total / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": desc, "M": M, "N": N, "K": K,
-                                        "sample_rows_per_step": R},
+        "impl": "reference", "metric": METRIC if p.kind == "bf16" else METRIC_MXFP8, "value": value,
+        "unit": UNIT, "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": p.desc, "M": p.M, "N": p.N, "K": p.K, "sample_rows_per_step": R},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"rows 0..{R - 1} of A against all of B ({R}x{N}x{K}) per step"},
+                         "sample": f"rows 0..{R - 1} of A against all of B ({R}x{p.N}x{p.K}) per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -205,29 +279,33 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="square8192", choices=sorted(WORKLOADS))
     ap.add_argument("--shape", type=int, nargs=3, metavar=("M", "N", "K"),
-                    help="override the workload's shape (bf16 U[-1,1] inputs), e.g. for profiling")
+                    help="override the workload's shape (U[-1,1] inputs), e.g. for profiling")
     ap.add_argument("--config", default="auto")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=5, help="0 skips the end-to-end leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    world, rank, local = dist_setup(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus > 1 and world == 1:
+        raise SystemExit("--gpus N > 1 needs torchrun: python -m torch.distributed.run "
+                         "--nproc-per-node N --master-addr 127.0.0.1 bench.py --gpus N")
     if args.impl == "reference":
-        run_reference(args, world, rank)
+        run_reference(args, rank)
         return
 
     import torch
     import torch.distributed as dist
 
     from dense_gemm_engineering_bf16_b200 import gemm as G
-    from dense_gemm_engineering_bf16_b200 import synth
 
     torch.cuda.set_device(local)
     if world > 1:
@@ -235,31 +313,20 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    M, N, K, distname, wid, desc = WORKLOADS[args.workload]
-    if args.shape:
-        M, N, K = args.shape
-        distname, wid = "uniform", 90
-        desc = f"gemm {M}x{N}x{K}, bf16 U[-1,1] in, fp32 out"
-    a_bits, b_bits = synth.bf16_operands(M, N, K, distname, workload=wid, base=rank)
-    A = torch.from_numpy(a_bits.view(np.int16)).cuda().view(torch.bfloat16)
-    B = torch.from_numpy(b_bits.view(np.int16)).cuda().view(torch.bfloat16)
-    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
-    G.gemm_force_config(args.config)
-    cfg_id = G.gemm_select_config(M, N, K)
-    cfg_name = {v: k for k, v in G.CONFIGS.items()}[cfg_id]
-    stream = torch.cuda.current_stream()
-    flops = 2.0 * M * N * K
-    in_out_bytes = 2 * (M * K + N * K) + 4 * M * N
-
-    def step():
-        G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_F32, stream=stream)
-
     def barrier():
         if world > 1:
             dist.barrier()
 
+    p = Problem(args.workload, args.shape, rank)
+    dev = p.device_arrays(torch)
+    C = p.empty_out(torch)
+    G.gemm_force_config(args.config)
+    cfg_name = "mxfp8_128x256" if p.kind == "mxfp8" else \
+        {v: k for k, v in G.CONFIGS.items()}[G.gemm_select_config(p.M, p.N, p.K)]
+    stream = torch.cuda.current_stream()
+
     for _ in range(args.warmup):
-        step()
+        p.call(G, dev, C, stream)
     G.gemm_check_device_status(stream)
 
     # ---------------------------------------------------- timed region --
@@ -275,108 +342,96 @@ def main():
     torch.cuda.synchronize()
     ev[0].record(stream)
     for i in range(args.steps):
-        step()
+        p.call(G, dev, C, stream)
         ev[i + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
     sampler.stop()
     G.gemm_check_device_status(stream)
-    per_launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    t_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        t = torch.tensor([t_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_ms = float(t.item())
+    per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    t_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, "cuda")
+
     # ------------------------------------------- end to end, host buffers --
-    e2e_steps = args.e2e_steps
-    e2e_value = None
-    if e2e_steps > 0:
-        e2e_value = run_e2e(torch, dist, G, a_bits, b_bits, A, B, C, M, N, K, flops, e2e_steps,
-                            stream, world, barrier)
+    e2e = None
+    if args.e2e_steps > 0:
+        host = [torch.from_numpy(np.ascontiguousarray(x).view(np.int16 if x.dtype == np.uint16 else np.uint8))
+                .pin_memory() for x in p.host]
+        dev_e = [torch.empty_like(d) for d in dev]
+        C_h = p.empty_out(torch, pinned=True)
+        C_e = p.empty_out(torch)
+
+        def e2e_step():
+            for d, h in zip(dev_e, host):
+                d.view(h.dtype).copy_(h, non_blocking=True)
+            p.call(G, dev_e, C_e, stream)
+            C_h.copy_(C_e, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+        barrier()
+        G.gemm_check_device_status(stream)
+        e2e = {"value": whole_job_tflops(p.flops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": p.in_bytes, "d2h_bytes_per_step": p.out_bytes, "steps": args.e2e_steps}
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return
-    _report(args, G, M, N, K, desc, cfg_name, flops, in_out_bytes, world, t_ms, per_launch_ms,
-            sampler, e2e_value, e2e_steps, a_bits, b_bits)
 
-
-def run_e2e(torch, dist, G, a_bits, b_bits, A, B, C, M, N, K, flops, e2e_steps, stream, world, barrier):
-    """Same metric through the C ABI with pinned host buffers: H2D of A and B,
-    the GEMM, D2H of C, all inside the timed region."""
-    A_h = torch.from_numpy(a_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    B_h = torch.from_numpy(b_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    C_h = torch.empty((M, N), dtype=torch.float32).pin_memory()
-    A_d = torch.empty_like(A)
-    B_d = torch.empty_like(B)
-    C_d = torch.empty_like(C)
-
-    def e2e_step():
-        A_d.copy_(A_h, non_blocking=True)
-        B_d.copy_(B_h, non_blocking=True)
-        G.gemm_bf16(A_d, B_d, C_d, M, N, K, K, K, N, G.OUT_F32, stream=stream)
-        C_h.copy_(C_d, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    barrier()
-    G.gemm_check_device_status(stream)
-    return world * e2e_steps * flops / (e2e_ms * 1e-3) / 1e12
-
-
-def _report(args, G, M, N, K, desc, cfg_name, flops, in_out_bytes, world, t_ms, per_launch_ms,
-            sampler, e2e_value, e2e_steps, a_bits, b_bits):
-    value = world * args.steps * flops / (t_ms * 1e-3) / 1e12
-    # ------------------------------------------------------------ roofline --
+    value = whole_job_tflops(p.flops, args.steps, world, t_ms)
     peaks, peak_src = load_peaks()
-    mean_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
-    achieved = flops / (mean_launch_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    traffic = profile_traffic(args.workload, cfg_name)
+    # per-step event time: for bf16 the step is the one GEMM launch; for
+    # MXFP8 it also holds the small scale-repack launch, so `achieved` is a
+    # lower bound for the GEMM kernel alone
+    mean_step_ms = sum(per_step_ms) / len(per_step_ms)
+    achieved = p.flops / (mean_step_ms * 1e-3) / 1e12
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ratio = 1.0 if p.kind == "bf16" else FP8_OVER_BF16
+    peak = bf16_peak * ratio
+    peak_note = (f"{peak_src} bf16_tflops (burst, cuBLAS 8192^3)" if p.kind == "bf16" else
+                 f"{peak_src} bf16_tflops x {FP8_OVER_BF16:g} (nominal fp8/bf16 dense ratio)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16_tflops (burst, cuBLAS 8192^3)",
-                "algorithmic_flops_per_launch": flops,
-                "min_bytes_per_launch": in_out_bytes}
+                "frac": achieved / peak, "traffic": profile_traffic(p.name, cfg_name),
+                "peak_source": peak_note,
+                "frac_of_sustained_peak": achieved / (sustained * ratio),
+                "algorithmic_flops_per_launch": p.flops,
+                "min_bytes_per_launch": p.in_bytes + p.out_bytes}
 
     cpu = None
     if not args.no_cpu_baseline:
         import oracle
-        fl, dt, R = oracle_sample(a_bits, b_bits, K, budget_s=args.cpu_budget)
+        fl, dt, R = oracle_sample(p, args.cpu_budget)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-               "sample": f"rows 0..{R - 1} of A against all of B ({R}x{N}x{K}), fp64 triple loop, "
+               "sample": f"rows 0..{R - 1} of A against all of B ({R}x{p.N}x{p.K}), fp64 triple loop, "
                          f"{dt:.1f} s"}
 
-    clocks = sampler.summary()
+    traffic_bytes = p.in_bytes + p.out_bytes
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": desc, "M": M, "N": N, "K": K, "kernel_config": cfg_name,
+        "metric": METRIC if p.kind == "bf16" else METRIC_MXFP8, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if p.kind == "bf16" else "e4m3",
+        "data": "synthetic",
+        "config": {"workload": p.desc, "M": p.M, "N": p.N, "K": p.K, "kernel_config": cfg_name,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"no flush: inputs+output {in_out_bytes / 2**20:.0f} MiB > 126 MiB L2"
-                   if in_out_bytes > L2_BYTES else "inputs fit in L2 (not flushed)",
-                   "launch_ms_median": statistics.median(per_launch_ms),
-                   "launch_ms_p90": float(np.percentile(per_launch_ms, 90))},
-        "e2e": None if e2e_value is None else
-        {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * (M * K + N * K),
-         "d2h_bytes_per_step": 4 * M * N, "steps": e2e_steps},
+                   "l2": (f"no flush: inputs+output {traffic_bytes / 2**20:.0f} MiB > 126 MiB L2"
+                          if traffic_bytes > L2_BYTES else "inputs fit in L2 (not flushed)"),
+                   "step_ms_median": statistics.median(per_step_ms),
+                   "step_ms_p90": float(np.percentile(per_step_ms, 90))},
+        "e2e": e2e,
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "clocks": clocks,
-        "gpu_launches": args.steps * G.gemm_launches_per_call(M, N, K, False) * world,
+        "clocks": sampler.summary(),
+        "gpu_launches": args.steps * p.launches(G) * world,
     }
     print(json.dumps(line), flush=True)
 

@@ -75,6 +75,18 @@ uint64_t watchdog_ns(int64_t K) {
     return base + static_cast<uint64_t>(K) * 100ull;
 }
 
+// Tile rows per raster group: tiles are walked column by column inside
+// groups of this many tile rows, so the CTAs running at the same time share A
+// row-panels and B column-panels in L2.  B200GEMM_GROUP_M overrides it.
+int raster_group_m() {
+    static const int g = [] {
+        const char *s = std::getenv("B200GEMM_GROUP_M");
+        const int v = s ? std::atoi(s) : 8;
+        return v > 0 ? v : 8;
+    }();
+    return g;
+}
+
 // Device of the current thread, checked to be compute capability 10.0, with
 // its status block allocated.
 gemm_status_t current_device(int &dev, DeviceState *&st) {
@@ -231,7 +243,8 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
     const int64_t clusters = tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi];
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
-                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), st->status, watchdog_ns(K));
+                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
+                           watchdog_ns(K));
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -377,7 +390,8 @@ gemm_status_t launch_mxf8(DeviceState *st, const void *A, const uint8_t *sfa, co
     const uint8_t *sfb_chunks = ws + a_blocks * kb * 512;
     kernel<<<static_cast<unsigned>(grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
         tmA, tmB, tmC, sfa_chunks, sfb_chunks, static_cast<int>(M), static_cast<int>(N),
-        static_cast<int>(K), C, ldc, static_cast<int>(n_tma), st->status, watchdog_ns(K));
+        static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
+                           watchdog_ns(K));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }

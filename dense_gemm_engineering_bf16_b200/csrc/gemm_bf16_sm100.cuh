@@ -78,7 +78,6 @@ struct GemmBf16Cfg {
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
     static constexpr int THREADS = 192;
-    static constexpr int GROUP_M = 8;              // tile rows per raster group (L2 reuse)
 
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
@@ -118,7 +117,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC,
-                       int M, int N, int K, void *C, int64_t ldc, int n_tma,
+                       int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m,
                        DeviceStatus *status, uint64_t timeout_ns) {
     constexpr int CG = Cfg::CG;
     extern __shared__ uint8_t smem_raw[];
@@ -183,7 +182,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t leader_rank = 0;
             for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
                 int tm, tn;
-                raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+                raster_tile(tile, num_m, num_n, group_m, tm, tn);
                 const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;
                 const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
                 for (int kb = 0; kb < num_kb; ++kb) {
@@ -268,7 +267,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         int t = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++t) {
             int tm, tn;
-            raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+            raster_tile(tile, num_m, num_n, group_m, tm, tn);
             const uint32_t buf = static_cast<uint32_t>(t) & 1u;
             const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
             // One lane waits; the verdict is broadcast so the warp stays

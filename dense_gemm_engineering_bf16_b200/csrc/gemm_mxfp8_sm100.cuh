@@ -60,7 +60,6 @@ struct GemmMxf8Cfg {
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL0 = 256;
     static constexpr int THREADS = 192;
-    static constexpr int GROUP_M = 8;
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
 };
 
@@ -104,7 +103,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC, const uint8_t *sfa_chunks,
                        const uint8_t *sfb_chunks, int M, int N, int K, void *C, int64_t ldc, int n_tma,
-                       DeviceStatus *status, uint64_t timeout_ns) {
+                       int group_m, DeviceStatus *status, uint64_t timeout_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -158,7 +157,7 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
                 int tm, tn;
-                raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+                raster_tile(tile, num_m, num_n, group_m, tm, tn);
                 const uint8_t *sfa_row = sfa_chunks + static_cast<int64_t>(tm) * num_kb * Cfg::SF_CHUNK;
                 const uint8_t *sfb_row0 = sfb_chunks + static_cast<int64_t>(2 * tn) * num_kb * Cfg::SF_CHUNK;
                 const uint8_t *sfb_row1 = sfb_row0 + static_cast<int64_t>(num_kb) * Cfg::SF_CHUNK;
@@ -247,7 +246,7 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         int t = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
             int tm, tn;
-            raster_tile(tile, num_m, num_n, Cfg::GROUP_M, tm, tn);
+            raster_tile(tile, num_m, num_n, group_m, tm, tn);
             uint32_t ready = 1;
             if (lane == 0 && !mbar_wait(tfull_bar, static_cast<uint32_t>(t) & 1u, abort_flag, timeout_ns)) {
                 record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
