@@ -15,6 +15,7 @@
 
 #include "b200gemm.h"
 #include "gemm_bf16_sm100.cuh"
+#include "gemm_bf16_skinny_sm100.cuh"
 #include "gemm_mxfp8_sm100.cuh"
 
 namespace {
@@ -29,7 +30,17 @@ using Cfg1x128F32 = b200::GemmBf16Cfg<1, 128, 6, 0>;
 using Cfg1x128B16 = b200::GemmBf16Cfg<1, 128, 6, 1>;
 using Cfg2x256F32 = b200::GemmBf16Cfg<2, 256, 6, 0>;
 using Cfg2x256B16 = b200::GemmBf16Cfg<2, 256, 6, 1>;
+using Cfg2x256F32C = b200::GemmBf16Cfg<2, 256, 6, 0, true>;
+using Cfg2x256B16C = b200::GemmBf16Cfg<2, 256, 6, 1, true>;
+using Cfg1x256F32C = b200::GemmBf16Cfg<1, 256, 4, 0, true>;
+using Cfg1x256B16C = b200::GemmBf16Cfg<1, 256, 4, 1, true>;
 using CfgMxf8 = b200::GemmMxf8Cfg<3>;
+using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
+using CfgSk64B16 = b200::GemmSkinnyCfg<64, 8, 1>;
+using CfgSk128F32 = b200::GemmSkinnyCfg<128, 6, 0>;
+using CfgSk128B16 = b200::GemmSkinnyCfg<128, 6, 1>;
+using CfgSk256F32 = b200::GemmSkinnyCfg<256, 4, 0>;
+using CfgSk256B16 = b200::GemmSkinnyCfg<256, 4, 1>;
 
 constexpr int kMaxDevices = 64;
 
@@ -45,6 +56,11 @@ struct DeviceState {
     bool mx_attr_done = false;
     uint8_t *mx_ws = nullptr;
     size_t mx_ws_bytes = 0;
+    // skinny path: kernel attributes (per template), split-tile workspace
+    bool sk_attr_done[6] = {};
+    uint8_t *sk_ws = nullptr;
+    size_t sk_ws_bytes = 0;
+    uint32_t sk_epoch = 0;
 };
 
 std::mutex g_mutex;
@@ -186,7 +202,11 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t /*K*/) {
     if (forced != GEMM_CFG_AUTO) return static_cast<gemm_config_t>(forced);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int64_t wide_tiles = ((M + 127) / 128) * ((N + 255) / 256);
+    // two or more waves of pair tiles: Cluster Launch Control evens out the
+    // tail; a single wave: the static persistent schedule
+    if (pair_tiles >= 148) return GEMM_CFG_2CTA_256x256_CLC;
     if (pair_tiles >= 74) return GEMM_CFG_2CTA_256x256;
+    if (M <= 256) return GEMM_CFG_SKINNY;          // too few tiles to fill the SMs: stream-K
     if (wide_tiles >= 148) return GEMM_CFG_1CTA_128x256;
     return GEMM_CFG_1CTA_128x128;
 }
@@ -216,7 +236,7 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
                                           Cfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
             int clusters = st->sm_count / Cfg::CG;
-            if (Cfg::CG > 1) {
+            if (Cfg::CG > 1 && !Cfg::CLC) {
                 lc.gridDim = dim3(Cfg::CG * clusters, 1, 1);
                 int n = 0;
                 if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
@@ -240,13 +260,112 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
         return s;
 
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
-    const int64_t clusters = tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi];
+    // Static schedule: as many clusters as fit at once, each striding over
+    // the tiles.  CLC: one cluster per tile; running clusters claim the rest.
+    const int64_t clusters = Cfg::CLC ? tiles
+                                      : (tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi]);
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
                            static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
                            watchdog_ns(K));
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
+}
+
+// ------------------------------------------------------------ skinny path --
+
+// Workspace of the skinny path: per persistent CTA `slots` partial tiles of
+// 128 x MP fp32, then one 64-bit arrival counter per 128-row tile of B.
+struct SkinnyLayout {
+    int64_t grid, slots, tiles, partial_bytes, counter_bytes;
+};
+
+template <class Cfg>
+SkinnyLayout skinny_layout(int64_t N, int64_t K, int sm_count) {
+    SkinnyLayout l;
+    const int64_t kb = (K + Cfg::BK - 1) / Cfg::BK;
+    l.tiles = (N + Cfg::TILE_N - 1) / Cfg::TILE_N;
+    const int64_t total = l.tiles * kb;
+    // at least kMinIters K blocks per CTA: a CTA with fewer barely fills its
+    // pipeline, and a tile cut into many slivers costs a long fix-up
+    constexpr int64_t kMinIters = 8;
+    const int64_t want = (total + kMinIters - 1) / kMinIters;
+    l.grid = want < sm_count ? want : sm_count;
+    const int64_t per = (total + l.grid - 1) / l.grid;
+    l.slots = (per + kb - 1) / kb + 1;
+    l.partial_bytes = l.grid * l.slots * Cfg::TILE_N * Cfg::MP * 4;
+    l.counter_bytes = l.tiles * 8;
+    return l;
+}
+
+// Grows the skinny workspace on demand (counters start at zero; cudaFree
+// waits for the device to go idle before the old buffer goes).
+gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (st->sk_ws_bytes < bytes) {
+        cudaError_t e;
+        if (st->sk_ws) {
+            if ((e = cudaFree(st->sk_ws)) != cudaSuccess) return cuda_fail(e);
+            st->sk_ws = nullptr;
+            st->sk_ws_bytes = 0;
+        }
+        const size_t want = bytes < (size_t(4) << 20) ? (size_t(4) << 20) : bytes;
+        if ((e = cudaMalloc(&st->sk_ws, want)) != cudaSuccess) return cuda_fail(e);
+        if ((e = cudaMemset(st->sk_ws, 0, want)) != cudaSuccess) return cuda_fail(e);
+        st->sk_ws_bytes = want;
+    }
+    ws = st->sk_ws;
+    return GEMM_OK;
+}
+
+template <class Cfg>
+gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const void *B, void *C, int64_t M,
+                            int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream) {
+    auto kernel = b200::gemm_bf16_skinny_sm100_kernel<Cfg>;
+    cudaError_t e;
+    uint32_t epoch;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!st->sk_attr_done[attr_slot]) {
+            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          Cfg::SMEM_BYTES)) != cudaSuccess)
+                return cuda_fail(e);
+            st->sk_attr_done[attr_slot] = true;
+        }
+        epoch = ++st->sk_epoch;
+        if (epoch == 0) epoch = ++st->sk_epoch;
+    }
+    const SkinnyLayout l = skinny_layout<Cfg>(N, K, st->sm_count);
+    uint8_t *ws = nullptr;
+    gemm_status_t s;
+    if ((s = sk_workspace(st, static_cast<size_t>(l.partial_bytes + l.counter_bytes), ws)) != GEMM_OK) return s;
+    const int64_t mpad = (M + 15) / 16 * 16;
+    alignas(64) CUtensorMap tmB, tmA;
+    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N)) != GEMM_OK)
+        return s;
+    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK,
+                       static_cast<uint32_t>(mpad))) != GEMM_OK)
+        return s;
+    float *partials = reinterpret_cast<float *>(ws);
+    unsigned long long *counters = reinterpret_cast<unsigned long long *>(ws + l.partial_bytes);
+    kernel<<<static_cast<unsigned>(l.grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+        tmB, tmA, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(mpad), C, ldc,
+        partials, counters, static_cast<int>(l.slots), epoch, st->status, watchdog_ns(K));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    return GEMM_OK;
+}
+
+gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const void *B, void *C, int64_t M,
+                                int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream) {
+    if (M > 256) return GEMM_ERR_INVALID_VALUE;
+    if (M <= 64)
+        return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                   : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream);
+    if (M <= 128)
+        return f32 ? launch_skinny<CfgSk128F32>(st, 2, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                   : launch_skinny<CfgSk128B16>(st, 3, A, B, C, M, N, K, lda, ldb, ldc, stream);
+    return f32 ? launch_skinny<CfgSk256F32>(st, 4, A, B, C, M, N, K, lda, ldb, ldc, stream)
+               : launch_skinny<CfgSk256B16>(st, 5, A, B, C, M, N, K, lda, ldb, ldc, stream);
 }
 
 template <typename T>
@@ -425,6 +544,14 @@ gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_
         case GEMM_CFG_2CTA_256x256:
             return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
                        : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_SKINNY:
+            return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_2CTA_256x256_CLC:
+            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        case GEMM_CFG_1CTA_128x256_CLC:
+            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
+                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
         default:
             return GEMM_ERR_INVALID_VALUE;
     }
@@ -521,7 +648,10 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
     // The status word must start at zero for the kernel to record a timeout.
     cudaError_t e = cudaMemsetAsync(st->status, 0, noalloc_scratch_bytes(), stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    const gemm_config_t cfg = select_config(M, N, K);
+    // The skinny kernel needs a workspace; without one, small-M shapes run on
+    // the one-CTA 128 x 128 kernel instead.
+    gemm_config_t cfg = select_config(M, N, K);
+    if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128;
     const bool f32 = c_type == GEMM_OUT_F32;
     switch (cfg) {
         case GEMM_CFG_1CTA_128x256:

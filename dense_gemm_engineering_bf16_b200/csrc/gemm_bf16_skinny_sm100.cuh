@@ -1,0 +1,396 @@
+// Skinny bf16 GEMM for sm_100a (small M): C = A . B with M <= 256.
+//
+// For a handful of rows of A the product is bound by streaming B from HBM
+// (the roofline of "Modern GPU Programming For MLSys - 书籍总结", section 2.2:
+// 16 x 8192 x 8192 has an arithmetic intensity of ~16 FLOP/B).  The kernel
+// is laid out so that every SM streams an equal share of B:
+//
+//  * swap A and B: the MMA computes C^T = B . A^T, so 128 rows of B fill the
+//    MMA's M = 128 and the (padded) rows of A are its N (16 .. 256, a
+//    multiple of 16).  No tensor-core work is spent on padding M up to 128.
+//  * stream-K: the iterations (128-row tile of B, 64-wide K block) are
+//    flattened and cut into gridDim.x equal contiguous ranges, one per
+//    persistent CTA.  A CTA's range crosses at most a few tile boundaries; a
+//    tile split across CTAs is finished by whichever contributor arrives
+//    last: every contributor writes its fp32 partial to a workspace, bumps
+//    the tile's arrival counter, and the last one sums the partials in
+//    contributor order (deterministic) and writes C.  A tile owned by one CTA
+//    is written directly.  Split-K is in the search space of "GPU 执行模型",
+//    section "编译与 autotune".
+//
+// Roles per CTA (192 threads) as in the square kernel: warp 0 TMA producer,
+// warp 1 TMEM owner and MMA issuer, warps 2-5 epilogue (TMEM lane = row of
+// B = column n of C).  C rows are written with plain coalesced stores: for a
+// fixed m, the 32 lanes of a warp hold 32 consecutive n.
+//
+// Arrival counters are 64-bit: (epoch << 32) | arrivals.  Each call passes a
+// new epoch, so a counter left behind by an earlier, aborted call is simply
+// restarted and no reset pass is needed; the last contributor also returns
+// its tile's count to zero, so replaying a captured launch (same epoch) works.
+#pragma once
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "gemm_bf16_sm100.cuh"
+#include "ptx.cuh"
+
+namespace b200 {
+
+template <int MP_, int STAGES_, int OUT_>
+struct GemmSkinnyCfg {
+    static constexpr int MP = MP_;                 // max padded rows of A (MMA N)
+    static constexpr int STAGES = STAGES_;
+    static constexpr int OUT = OUT_;               // 0: f32 C, 1: bf16 C
+    static constexpr int TILE_N = 128;             // rows of B per tile (MMA M)
+    static constexpr int BK = 64;
+    static constexpr int UMMA_K = 16;
+    static constexpr int B_BYTES = TILE_N * BK * 2;
+    static constexpr int A_BYTES = MP * BK * 2;
+    static constexpr int STAGE_BYTES = B_BYTES + A_BYTES;
+    static constexpr int TMEM_COLS = pow2_at_least(2 * MP, 32);
+    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
+    static constexpr int THREADS = 192;
+    static_assert(MP % 16 == 0 && MP >= 16 && MP <= 256, "MMA N for M = 128");
+    static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+    static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
+    static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
+};
+
+// First iteration of CTA c's range when `total` iterations are cut into `g`.
+__device__ __forceinline__ int64_t range_begin(int64_t c, int64_t total, int64_t g) {
+    return (c * total) / g;
+}
+
+// The CTA whose range holds iteration `it`.
+__device__ __forceinline__ int64_t range_owner(int64_t it, int64_t total, int64_t g) {
+    return ((it + 1) * g + total - 1) / total - 1;
+}
+
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_c(void *C, int64_t ldc, int m, int n, float v) {
+    if constexpr (OUT == 0) {
+        static_cast<float *>(C)[static_cast<int64_t>(m) * ldc + n] = v;
+    } else {
+        static_cast<__nv_bfloat16 *>(C)[static_cast<int64_t>(m) * ldc + n] = __float2bfloat16_rn(v);
+    }
+}
+
+// The last contributor of a split tile sums the contributors' fp32 partials
+// ([m][128] each) in contributor order and writes C rows [0, M) x the tile's
+// 128 columns.  Thread t handles four consecutive columns (t % 32) * 4 of
+// rows m = 4 j + t / 32; per round every thread has 8 rows x 2 contributors
+// of float4 loads in flight, and each element is summed c_lo, c_lo+1, ...
+// exactly as a sequential loop would.
+template <int OUT>
+__device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_elems, int slots_per_cta,
+                                           int64_t c_lo, int64_t c_hi, int64_t t, int64_t total, int64_t g,
+                                           int64_t kb_per_tile, int M, int N, void *C, int64_t ldc,
+                                           uint32_t epi_tid) {
+    constexpr int ROWS = 8;                      // rows per round for this thread
+    const int n4 = static_cast<int>(epi_tid & 31u) * 4;
+    const int msub = static_cast<int>(epi_tid >> 5);
+    const int n = static_cast<int>(t) * 128 + n4;
+    auto slot_ptr = [&](int64_t cc) {
+        const int64_t cc_first = ((cc * total) / g) / kb_per_tile;
+        return partials + (cc * slots_per_cta + (t - cc_first)) * slot_elems + n4;
+    };
+    for (int m0 = msub; m0 < M; m0 += 4 * ROWS) {
+        float4 acc[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        int64_t cc = c_lo;
+        for (; cc <= c_hi; cc += 2) {
+            const bool two = cc + 1 <= c_hi;
+            const float *p0 = slot_ptr(cc);
+            const float *p1 = two ? slot_ptr(cc + 1) : p0;
+            float4 v0[ROWS], v1[ROWS];
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const int m = m0 + 4 * r;
+                const bool in = m < M;
+                v0[r] = in ? __ldcg(reinterpret_cast<const float4 *>(p0 + static_cast<int64_t>(m) * 128))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                v1[r] = (in && two) ? __ldcg(reinterpret_cast<const float4 *>(p1 + static_cast<int64_t>(m) * 128))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                acc[r].x += v0[r].x; acc[r].y += v0[r].y; acc[r].z += v0[r].z; acc[r].w += v0[r].w;
+                if (two) {
+                    acc[r].x += v1[r].x; acc[r].y += v1[r].y; acc[r].z += v1[r].z; acc[r].w += v1[r].w;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            const int m = m0 + 4 * r;
+            if (m >= M || n >= N) continue;
+            const float vals[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
+            if (n + 4 <= N) {
+                if constexpr (OUT == 0) {
+                    *reinterpret_cast<float4 *>(static_cast<float *>(C) + static_cast<int64_t>(m) * ldc + n) = acc[r];
+                } else {
+                    const uint32_t lo = pack_bf16x2(vals[0], vals[1]);
+                    const uint32_t hi = pack_bf16x2(vals[2], vals[3]);
+                    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(C) + static_cast<int64_t>(m) * ldc + n) =
+                        make_uint2(lo, hi);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (n + q < N) store_c<OUT>(C, ldc, m, n + q, vals[q]);
+            }
+        }
+    }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as N x K, box 64 x 128
+                              const __grid_constant__ CUtensorMap tmA,   // A as M x K, box 64 x mpad
+                              int M, int N, int K, int mpad, void *C, int64_t ldc,
+                              float *partials, unsigned long long *counters, int slots_per_cta,
+                              uint32_t epoch, DeviceStatus *status, uint64_t timeout_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    const uint32_t base = smem_addr(smem);
+    const uint32_t warp = threadIdx.x / 32;
+    const uint32_t lane = threadIdx.x % 32;
+
+    const uint32_t bar0 = base + Cfg::BAR_OFF;
+    auto full_bar = [&](uint32_t s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](uint32_t s) { return bar0 + 8u * (Cfg::STAGES + s); };
+    auto tfull_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + b); };
+    auto tempty_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + b); };
+    const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
+    const uint32_t abort_slot = tmem_slot + 4u;
+    volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
+    volatile uint32_t *abort_flag = tmem_slot_ptr + 1;
+    volatile uint32_t *last_flag = tmem_slot_ptr + 2;
+    volatile uint32_t *ready_flag = tmem_slot_ptr + 3;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 4);
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc<1>(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish<1>();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot_ptr;
+
+    const int64_t kb_per_tile = (K + Cfg::BK - 1) / Cfg::BK;
+    const int64_t tiles = (N + Cfg::TILE_N - 1) / Cfg::TILE_N;
+    const int64_t total = tiles * kb_per_tile;
+    const int64_t g = gridDim.x;
+    const int64_t c = blockIdx.x;
+    const int64_t it_begin = range_begin(c, total, g);
+    const int64_t it_end = range_begin(c + 1, total, g);
+    const int64_t first_tile = it_begin / kb_per_tile;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            const uint32_t tx = static_cast<uint32_t>(Cfg::B_BYTES + mpad * Cfg::BK * 2);
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int64_t it = it_begin; it < it_end; ++it) {
+                const int t = static_cast<int>(it / kb_per_tile);
+                const int kb = static_cast<int>(it - static_cast<int64_t>(t) * kb_per_tile);
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarEmpty);
+                    ok = false;
+                    break;
+                }
+                const uint32_t b_dst = base + stage * Cfg::STAGE_BYTES;
+                const uint32_t a_dst = b_dst + Cfg::B_BYTES;
+                mbar_arrive_expect_tx(full_bar(stage), tx);
+                tma_load_2d(b_dst, &tmB, full_bar(stage), kb * Cfg::BK, t * Cfg::TILE_N);
+                tma_load_2d(a_dst, &tmA, full_bar(stage), kb * Cfg::BK, 0);
+                if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+            }
+            for (int i = 0; ok && i < Cfg::STAGES; ++i) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarTail);
+                    ok = false;
+                }
+                if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // --------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(Cfg::TILE_N, mpad);
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            int seg = 0;
+            int64_t it = it_begin;
+            while (ok && it < it_end) {
+                const int64_t t = it / kb_per_tile;
+                const int64_t seg_end = min(it_end, (t + 1) * kb_per_tile);
+                const uint32_t buf = static_cast<uint32_t>(seg) & 1u;
+                if (!mbar_wait(tempty_bar(buf), ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u, abort_flag,
+                               timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarTmemEmpty);
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + buf * Cfg::MP;
+                for (int64_t j = it; j < seg_end; ++j) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarFull);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t b0 = base + stage * Cfg::STAGE_BYTES;
+                    const uint32_t a0 = b0 + Cfg::B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
+                        mma_bf16_ss<1>(d_tmem, sw128_kmajor_desc(b0 + kk * 32), sw128_kmajor_desc(a0 + kk * 32),
+                                       idesc, (j != it || kk != 0) ? 1u : 0u);
+                    }
+                    mma_commit<1>(empty_bar(stage), 0);
+                    if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit<1>(tfull_bar(buf), 0);
+                it = seg_end;
+                ++seg;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------- epilogue --
+        const uint32_t sub = warp & 3u;
+        const int n_local = static_cast<int>(sub * 32u + lane);
+        const uint32_t epi_tid = threadIdx.x - 64u;          // 0..127
+        const int64_t slot_elems = static_cast<int64_t>(Cfg::TILE_N) * Cfg::MP;
+        int seg = 0;
+        int64_t it = it_begin;
+        while (it < it_end) {
+            const int64_t t = it / kb_per_tile;
+            const int64_t seg_end = min(it_end, (t + 1) * kb_per_tile);
+            const uint32_t buf = static_cast<uint32_t>(seg) & 1u;
+            const int64_t c_lo = range_owner(t * kb_per_tile, total, g);
+            const int64_t c_hi = range_owner((t + 1) * kb_per_tile - 1, total, g);
+            const bool shared_tile = c_hi > c_lo;
+            // One thread waits; all 128 epilogue threads take its verdict, so
+            // they stay in step for the named barriers below.
+            if (epi_tid == 0) {
+                uint32_t ok = 1;
+                if (!mbar_wait(tfull_bar(buf), (static_cast<uint32_t>(seg) >> 1) & 1u, abort_flag, timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
+                    ok = 0;
+                }
+                *ready_flag = ok;
+            }
+            named_barrier_sync(1, 128);
+            if (!*ready_flag) break;
+            tc_fence_after_sync();
+            const int n = static_cast<int>(t) * Cfg::TILE_N + n_local;
+            float *my_partial = partials + (c * slots_per_cta + (t - first_tile)) * slot_elems;
+            const uint32_t tbase = tmem_base + ((sub * 32u) << 16) + buf * Cfg::MP;
+            for (int m0 = 0; m0 < mpad; m0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(m0), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + i;
+                    if (m < M) {
+                        const float x = __uint_as_float(v[i]);
+                        if (shared_tile) my_partial[static_cast<int64_t>(m) * Cfg::TILE_N + n_local] = x;
+                        else if (n < N) store_c<Cfg::OUT>(C, ldc, m, n, x);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(tempty_bar(buf));
+
+            if (shared_tile) {
+                // Publish this partial, count the arrival; the last of the
+                // tile's contributors sums all partials in contributor order.
+                // The barrier orders the 128 threads' partial stores before
+                // thread 0's gpu-scope fence, which (being cumulative) makes
+                // them visible before its counter update.
+                named_barrier_sync(1, 128);
+                if (epi_tid == 0) {
+                    __threadfence();
+                    unsigned long long *ctr = counters + t;
+                    const unsigned long long tag = static_cast<unsigned long long>(epoch) << 32;
+                    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(ctr), seen;
+                    unsigned long long want;
+                    do {
+                        seen = old;
+                        want = ((seen & 0xFFFFFFFF00000000ull) == tag) ? seen + 1ull : (tag | 1ull);
+                        old = atomicCAS(ctr, seen, want);
+                    } while (old != seen);
+                    *last_flag = ((want & 0xFFFFFFFFull) == static_cast<unsigned long long>(c_hi - c_lo + 1)) ? 1u : 0u;
+                }
+                named_barrier_sync(1, 128);
+                if (*last_flag) {
+                    __threadfence();
+                    fixup_tile<Cfg::OUT>(partials, slot_elems, slots_per_cta, c_lo, c_hi, t, total, g,
+                                         kb_per_tile, M, N, C, ldc, epi_tid);
+                    // every contributor has arrived: leave the counter at zero
+                    // arrivals so a replay of this launch (same epoch, e.g.
+                    // from a CUDA graph) starts from a clean count
+                    if (epi_tid == 0) counters[t] = static_cast<unsigned long long>(epoch) << 32;
+                }
+                named_barrier_sync(1, 128);
+            }
+            it = seg_end;
+            ++seg;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc<1>(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace b200

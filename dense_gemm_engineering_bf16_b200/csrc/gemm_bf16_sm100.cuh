@@ -22,6 +22,13 @@
 //               once the accumulator is read, so tile i+1's main loop runs
 //               while tile i drains (TMEM double buffer, 2 x BN columns).
 //
+//   warp 6      (CLC builds only) scheduler, in the pair leader: claims tiles
+//               of clusters that have not started with
+//               clusterlaunchcontrol.try_cancel ("Modern GPU Programming For
+//               MLSys - 书籍总结", section 2.9: fast CTAs pull more work instead
+//               of idling) and hands the tile id to every role of both CTAs
+//               through a 2-deep shared-memory ring.
+//
 // Tails: TMA loads zero-fill outside [0,K) x [0,M) / [0,N) element by
 // element.  TMA stores clip rows exactly but write whole 16-byte granules
 // along a row, so C's tensor map covers only the columns [0, n_tma) that end
@@ -45,8 +52,9 @@ struct DeviceStatus {
 
 constexpr uint32_t kStatusTimeout = 6;   // == GEMM_ERR_TIMEOUT
 
-enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3 };
-enum : int { kBarFull = 1, kBarEmpty = 2, kBarTmemFull = 3, kBarTmemEmpty = 4, kBarTail = 5 };
+enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleScheduler = 4 };
+enum : int { kBarFull = 1, kBarEmpty = 2, kBarTmemFull = 3, kBarTmemEmpty = 4, kBarTail = 5, kBarSched = 6,
+             kBarClc = 7 };
 
 __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     int p = lo;
@@ -54,8 +62,9 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     return p;
 }
 
-template <int CG_, int BN_, int STAGES_, int OUT_>
+template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false>
 struct GemmBf16Cfg {
+    static constexpr bool CLC = CLC_;              // tiles from Cluster Launch Control, not a fixed stride
     static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
     static constexpr int BN = BN_;                 // tile N == MMA N
     static constexpr int STAGES = STAGES_;         // shared-memory ring depth
@@ -74,10 +83,13 @@ struct GemmBf16Cfg {
     static constexpr int EPI_BUF = 32 * 128;       // one warp's 32 rows x 128 bytes
     static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
     static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
-    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    // full[S], empty[S], tmem_full[2], tmem_empty[2] (+ clc[2], sched_full[2], sched_empty[2])
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + (CLC ? 6 : 0);
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
-    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
-    static constexpr int THREADS = 192;
+    // after the barriers: TMEM address, abort flag, 2 tile ids, 2 CLC answers
+    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 64;
+    static constexpr int THREADS = CLC ? 224 : 192;        // + one scheduler warp
+    static constexpr int SCHED_CONSUMERS = CG == 1 ? 6 : 11;  // arrivals that free a tile slot
 
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
@@ -135,10 +147,16 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     auto empty_bar = [&](uint32_t s) { return bar0 + 8u * (Cfg::STAGES + s); };
     auto tfull_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + b); };
     auto tempty_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + b); };
+    auto clc_bar = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 4 + i); };
+    auto sched_full = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 6 + i); };
+    auto sched_empty = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 8 + i); };
     const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
     const uint32_t abort_slot = tmem_slot + 4u;
+    const uint32_t tile_ids = tmem_slot + 8u;              // int32 [2]
+    const uint32_t clc_resp = tmem_slot + 16u;             // 16-byte answers [2]
     volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
     volatile uint32_t *abort_flag = tmem_slot_ptr + 1;
+    volatile int32_t *tile_id_ptr = reinterpret_cast<volatile int32_t *>(tmem_slot_ptr + 2);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -148,6 +166,13 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
             mbar_init(tempty_bar(b), 4 * CG);
+        }
+        if constexpr (Cfg::CLC) {
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(clc_bar(i), 1);
+                mbar_init(sched_full(i), 1);
+                mbar_init(sched_empty(i), Cfg::SCHED_CONSUMERS);
+            }
         }
         *abort_flag = 0u;
         fence_barrier_init();
@@ -174,13 +199,38 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     const int cluster_id = static_cast<int>(blockIdx.x) / CG;
     const int num_clusters = static_cast<int>(gridDim.x) / CG;
 
+    // The tile sequence every role of this CTA (and of its pair) walks.
+    // Static: cluster_id, + num_clusters, ...  CLC: the first tile is the
+    // cluster's own; the j-th later tile is read from ring slot j % 2, which
+    // the scheduler warp fills, and the slot is handed back to the leader.
+    auto next_tile = [&](int tile, uint32_t j, bool &ok) -> int {
+        if constexpr (!Cfg::CLC) {
+            (void)j;
+            (void)ok;
+            const int n = tile + num_clusters;
+            return n < num_tiles ? n : -1;
+        } else {
+            (void)tile;
+            const uint32_t slot = j & 1u;
+            if (!mbar_wait(sched_full(slot), (j >> 1) & 1u, abort_flag, timeout_ns)) {
+                ok = false;
+                return -1;
+            }
+            const int n = tile_id_ptr[slot];
+            if constexpr (CG == 1) mbar_arrive_local(sched_empty(slot));
+            else mbar_arrive_cluster(map_to_cta(sched_empty(slot), 0));
+            return n;
+        }
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             const uint32_t leader_rank = 0;
-            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+            uint32_t fetched = 0;
+            for (int tile = cluster_id; ok && tile >= 0;) {
                 int tm, tn;
                 raster_tile(tile, num_m, num_n, group_m, tm, tn);
                 const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;
@@ -206,6 +256,9 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
+                if (!ok) break;
+                tile = next_tile(tile, fetched++, ok);
+                if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarSched);
             }
             // Tail: every stage handed out must be released by the MMA before
             // this CTA may exit (its empty barriers still receive arrivals).
@@ -225,7 +278,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             int t = 0;
-            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters, ++t) {
+            for (int tile = cluster_id; ok && tile >= 0; ++t) {
                 const uint32_t buf = static_cast<uint32_t>(t) & 1u;
                 const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
                 if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, timeout_ns)) {
@@ -255,6 +308,39 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 if (!ok) break;
                 mma_commit<CG>(tfull_bar(buf), 0x3);
+                tile = next_tile(tile, static_cast<uint32_t>(t), ok);
+                if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarSched);
+            }
+        }
+        __syncwarp();
+    } else if (Cfg::CLC && warp == 6) {
+        // ------------------------------------------- CLC scheduler (leader) --
+        if constexpr (Cfg::CLC) {
+            if (rank == 0 && lane == 0) {
+                for (uint32_t j = 0;; ++j) {
+                    const uint32_t slot = j & 1u, ph = (j >> 1) & 1u;
+                    if (!mbar_wait(sched_empty(slot), ph ^ 1u, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleScheduler * 16 + kBarSched);
+                        break;
+                    }
+                    mbar_arrive_expect_tx(clc_bar(slot), 16);
+                    clc_try_cancel(clc_resp + 16u * slot, clc_bar(slot));
+                    if (!mbar_wait(clc_bar(slot), ph, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleScheduler * 16 + kBarClc);
+                        break;
+                    }
+                    uint32_t first_x = 0;
+                    const bool got = clc_query(clc_resp + 16u * slot, first_x);
+                    fence_proxy_async_smem();   // the slot's answer is rewritten by a later request
+                    const int next = got ? static_cast<int>(first_x) / CG : -1;
+                    tile_id_ptr[slot] = next;
+                    mbar_arrive_local(sched_full(slot));
+                    if constexpr (CG == 2) {
+                        store_cluster_s32(map_to_cta(tile_ids + 4u * slot, 1), next);
+                        mbar_arrive_cluster(map_to_cta(sched_full(slot), 1));
+                    }
+                    if (next < 0) break;   // no cluster left: no further requests
+                }
             }
         }
         __syncwarp();
@@ -265,7 +351,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
         uint32_t nstore = 0;
         int t = 0;
-        for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++t) {
+        for (int tile = cluster_id; tile >= 0; ++t) {
             int tm, tn;
             raster_tile(tile, num_m, num_n, group_m, tm, tn);
             const uint32_t buf = static_cast<uint32_t>(t) & 1u;
@@ -352,6 +438,14 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 ++nstore;
             }
+            // next tile: one lane fetches it, the warp follows
+            int nt = -1;
+            if (lane == 0) {
+                bool ok = true;
+                nt = next_tile(tile, static_cast<uint32_t>(t), ok);
+                if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarSched);
+            }
+            tile = __shfl_sync(0xffffffffu, nt, 0);
         }
         if (lane == 0) bulk_wait_group<0>();
         __syncwarp();

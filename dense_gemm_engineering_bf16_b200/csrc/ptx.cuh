@@ -272,6 +272,35 @@ __device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, ui
                  : "memory");
 }
 
+// ------------------------------------------------ cluster launch control --
+
+// Ask the hardware scheduler to cancel one cluster of this grid that has not
+// started yet; the 16-byte answer lands in this CTA's shared memory at
+// `resp` and completes 16 transaction bytes on `bar`.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+    asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+                 ::"r"(resp), "r"(bar) : "memory");
+}
+
+// Decode an answer: true and the first CTA index (x) of the cancelled
+// cluster, or false when no cluster was left to cancel.
+__device__ __forceinline__ bool clc_query(uint32_t resp, uint32_t &first_ctaid_x) {
+    uint32_t ok, x;
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+                 "ld.shared.b128 r, [%2];\n\t"
+                 "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t"
+                 "mov.u32 %1, 0;\n\t"
+                 "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+                 : "=r"(ok), "=r"(x) : "r"(resp) : "memory");
+    first_ctaid_x = x;
+    return ok != 0;
+}
+
+__device__ __forceinline__ void store_cluster_s32(uint32_t cluster_addr, int32_t v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // ------------------------------------------------------------ descriptors --
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA

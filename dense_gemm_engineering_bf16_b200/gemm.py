@@ -28,6 +28,9 @@ CONFIGS = {
     "1cta_128x256": 1,
     "1cta_128x128": 2,
     "2cta_256x256": 3,
+    "skinny": 4,
+    "2cta_256x256_clc": 5,
+    "1cta_128x256_clc": 6,
 }
 
 STATUS_NAMES = {

@@ -75,7 +75,13 @@ typedef enum {
     GEMM_CFG_1CTA_128x256 = 1,      /* one CTA per tile, tile 128 x 256, tcgen05 cta_group::1 */
     GEMM_CFG_1CTA_128x128 = 2,      /* one CTA per tile, tile 128 x 128 */
     GEMM_CFG_2CTA_256x256 = 3,      /* CTA pair per tile, tile 256 x 256, cta_group::2 */
-    GEMM_CFG_COUNT_ = 4
+    GEMM_CFG_SKINNY = 4,            /* M <= 256: swap A/B (128 rows of B per MMA), stream-K over
+                                       all SMs, deterministic fix-up of split tiles; uses a
+                                       library-owned workspace (cudaMalloc on first use) */
+    GEMM_CFG_2CTA_256x256_CLC = 5,  /* as 2CTA_256x256, tiles handed out by Cluster Launch Control:
+                                       one cluster per tile, running pairs claim pending ones */
+    GEMM_CFG_1CTA_128x256_CLC = 6,  /* as 1CTA_128x256 with Cluster Launch Control */
+    GEMM_CFG_COUNT_ = 7
 } gemm_config_t;
 
 /*
