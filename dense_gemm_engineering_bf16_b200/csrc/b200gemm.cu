@@ -103,6 +103,14 @@ int raster_group_m() {
     return g;
 }
 
+// Test-only: B200GEMM_INJECT_TIMEOUT=1 makes the next square-kernel launches
+// drop one pipeline arrival in CTA 0 so the device watchdog fires (read at
+// every launch, so a test can switch it on and off inside one process).
+uint32_t inject_flags() {
+    const char *s = std::getenv("B200GEMM_INJECT_TIMEOUT");
+    return (s && s[0] == '1') ? b200::kInjectDropFirstStage : 0u;
+}
+
 // Device of the current thread, checked to be compute capability 10.0, with
 // its status block allocated.
 gemm_status_t current_device(int &dev, DeviceState *&st) {
@@ -267,7 +275,7 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
                            static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
-                           watchdog_ns(K));
+                           watchdog_ns(K), inject_flags());
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -509,8 +517,7 @@ gemm_status_t launch_mxf8(DeviceState *st, const void *A, const uint8_t *sfa, co
     const uint8_t *sfb_chunks = ws + a_blocks * kb * 512;
     kernel<<<static_cast<unsigned>(grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
         tmA, tmB, tmC, sfa_chunks, sfb_chunks, static_cast<int>(M), static_cast<int>(N),
-        static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
-                           watchdog_ns(K));
+        static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status, watchdog_ns(K));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }

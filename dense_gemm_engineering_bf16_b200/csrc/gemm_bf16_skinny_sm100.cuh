@@ -230,7 +230,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
             for (int64_t it = it_begin; it < it_end; ++it) {
                 const int t = static_cast<int>(it / kb_per_tile);
                 const int kb = static_cast<int>(it - static_cast<int64_t>(t) * kb_per_tile);
-                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarEmpty);
                     ok = false;
                     break;
@@ -243,7 +243,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
             }
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
-                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarTail);
                     ok = false;
                 }
@@ -264,7 +264,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 const int64_t seg_end = min(it_end, (t + 1) * kb_per_tile);
                 const uint32_t buf = static_cast<uint32_t>(seg) & 1u;
                 if (!mbar_wait(tempty_bar(buf), ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u, abort_flag,
-                               timeout_ns)) {
+                               3 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarTmemEmpty);
                     break;
                 }
@@ -313,7 +313,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
             // they stay in step for the named barriers below.
             if (epi_tid == 0) {
                 uint32_t ok = 1;
-                if (!mbar_wait(tfull_bar(buf), (static_cast<uint32_t>(seg) >> 1) & 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(tfull_bar(buf), (static_cast<uint32_t>(seg) >> 1) & 1u, abort_flag, 3 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
                     ok = 0;
                 }

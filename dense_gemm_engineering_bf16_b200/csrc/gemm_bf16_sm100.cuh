@@ -52,6 +52,11 @@ struct DeviceStatus {
 
 constexpr uint32_t kStatusTimeout = 6;   // == GEMM_ERR_TIMEOUT
 
+// Test-only fault injection (host side: B200GEMM_INJECT_TIMEOUT): CTA 0 skips
+// its first k-tile, leaving that stage's full barrier unarmed, so the MMA
+// warp's bounded wait expires and the abort path runs.  Nothing faults.
+constexpr uint32_t kInjectDropFirstStage = 1u;
+
 enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleScheduler = 4 };
 enum : int { kBarFull = 1, kBarEmpty = 2, kBarTmemFull = 3, kBarTmemEmpty = 4, kBarTail = 5, kBarSched = 6,
              kBarClc = 7 };
@@ -113,15 +118,20 @@ __device__ __forceinline__ void raster_tile(int tile, int num_m, int num_n, int 
     tn = local / rows;
 }
 
+// A bounded wait failed.  If it failed because this CTA was already told to
+// abort, someone else has recorded the cause: just leave.  Otherwise record
+// the first expired wait of the grid (role, barrier, CTA), then tell this CTA
+// and its pair partner to abort.
 __device__ __forceinline__ void record_timeout(DeviceStatus *status, volatile uint32_t *abort_flag,
                                                uint32_t abort_smem, int cg, int where) {
-    *abort_flag = 1u;
-    if (cg == 2) store_cluster_u32(map_to_cta(abort_smem, cluster_cta_rank() ^ 1u), 1u);
+    if (*abort_flag) return;
     if (atomicCAS(&status->code, 0u, kStatusTimeout) == 0u) {
         status->where = where;
         status->block = static_cast<int32_t>(blockIdx.x);
         __threadfence();
     }
+    *abort_flag = 1u;
+    if (cg == 2) store_cluster_u32(map_to_cta(abort_smem, cluster_cta_rank() ^ 1u), 1u);
 }
 
 template <class Cfg>
@@ -130,7 +140,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC,
                        int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m,
-                       DeviceStatus *status, uint64_t timeout_ns) {
+                       DeviceStatus *status, uint64_t timeout_ns, uint32_t inject) {
     constexpr int CG = Cfg::CG;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-memory window offset (swizzle atoms).
@@ -212,7 +222,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         } else {
             (void)tile;
             const uint32_t slot = j & 1u;
-            if (!mbar_wait(sched_full(slot), (j >> 1) & 1u, abort_flag, timeout_ns)) {
+            if (!mbar_wait(sched_full(slot), (j >> 1) & 1u, abort_flag, 3 * timeout_ns)) {
                 ok = false;
                 return -1;
             }
@@ -236,7 +246,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;
                 const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarEmpty);
                         ok = false;
                         break;
@@ -244,6 +254,12 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t a_dst = base + stage * Cfg::STAGE_BYTES;
                     const uint32_t b_dst = a_dst + Cfg::A_BYTES;
                     const int kx = kb * Cfg::BK;
+                    if ((inject & kInjectDropFirstStage) && blockIdx.x == 0 && fetched == 0 && kb == 0) {
+                        // Failure-detection test: this stage's full barrier is
+                        // never armed, so the MMA's bounded wait on it expires.
+                        if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
                     if constexpr (CG == 1) {
                         mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
                         tma_load_2d(a_dst, &tmA, full_bar(stage), kx, a_row);
@@ -263,7 +279,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             // Tail: every stage handed out must be released by the MMA before
             // this CTA may exit (its empty barriers still receive arrivals).
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
-                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarTail);
                     ok = false;
                 }
@@ -281,7 +297,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int tile = cluster_id; ok && tile >= 0; ++t) {
                 const uint32_t buf = static_cast<uint32_t>(t) & 1u;
                 const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
-                if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, 3 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarTmemEmpty);
                     ok = false;
                     break;
@@ -319,13 +335,13 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             if (rank == 0 && lane == 0) {
                 for (uint32_t j = 0;; ++j) {
                     const uint32_t slot = j & 1u, ph = (j >> 1) & 1u;
-                    if (!mbar_wait(sched_empty(slot), ph ^ 1u, abort_flag, timeout_ns)) {
+                    if (!mbar_wait(sched_empty(slot), ph ^ 1u, abort_flag, 3 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleScheduler * 16 + kBarSched);
                         break;
                     }
                     mbar_arrive_expect_tx(clc_bar(slot), 16);
                     clc_try_cancel(clc_resp + 16u * slot, clc_bar(slot));
-                    if (!mbar_wait(clc_bar(slot), ph, abort_flag, timeout_ns)) {
+                    if (!mbar_wait(clc_bar(slot), ph, abort_flag, 3 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleScheduler * 16 + kBarClc);
                         break;
                     }
@@ -359,7 +375,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             // One lane waits; the verdict is broadcast so the warp stays
             // converged for the .sync.aligned TMEM loads below.
             uint32_t ready = 1;
-            if (lane == 0 && !mbar_wait(tfull_bar(buf), acc_phase, abort_flag, timeout_ns)) {
+            if (lane == 0 && !mbar_wait(tfull_bar(buf), acc_phase, abort_flag, 3 * timeout_ns)) {
                 record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarTmemFull);
                 ready = 0;
             }

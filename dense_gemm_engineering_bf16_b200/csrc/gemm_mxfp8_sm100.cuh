@@ -162,7 +162,7 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                 const uint8_t *sfb_row0 = sfb_chunks + static_cast<int64_t>(2 * tn) * num_kb * Cfg::SF_CHUNK;
                 const uint8_t *sfb_row1 = sfb_row0 + static_cast<int64_t>(num_kb) * Cfg::SF_CHUNK;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarEmpty);
                         ok = false;
                         break;
@@ -183,7 +183,7 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                 }
             }
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
-                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarTail);
                     ok = false;
                 }
@@ -198,7 +198,7 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             bool ok = true;
             int t = 0;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++t) {
-                if (!mbar_wait(tempty_bar, (static_cast<uint32_t>(t) & 1u) ^ 1u, abort_flag, timeout_ns)) {
+                if (!mbar_wait(tempty_bar, (static_cast<uint32_t>(t) & 1u) ^ 1u, abort_flag, 3 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarTmemEmpty);
                     ok = false;
                     break;
@@ -248,7 +248,7 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             int tm, tn;
             raster_tile(tile, num_m, num_n, group_m, tm, tn);
             uint32_t ready = 1;
-            if (lane == 0 && !mbar_wait(tfull_bar, static_cast<uint32_t>(t) & 1u, abort_flag, timeout_ns)) {
+            if (lane == 0 && !mbar_wait(tfull_bar, static_cast<uint32_t>(t) & 1u, abort_flag, 3 * timeout_ns)) {
                 record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
                 ready = 0;
             }
