@@ -19,7 +19,6 @@ the oracle alone, as the reference arm.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -55,12 +54,27 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 
-def kernel_source_hash() -> str:
+# The device sources each kernel is compiled from; an ncu traffic figure is
+# valid only while these files are unchanged.
+KERNEL_SOURCES = {
+    "bf16": ["ptx.cuh", "gemm_bf16_sm100.cuh"],
+    "skinny": ["ptx.cuh", "gemm_bf16_sm100.cuh", "gemm_bf16_skinny_sm100.cuh"],
+    "mxfp8": ["ptx.cuh", "gemm_bf16_sm100.cuh", "gemm_mxfp8_sm100.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str = "bf16") -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "dense_gemm_engineering_bf16_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "dense_gemm_engineering_bf16_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def kernel_family(config_name: str) -> str:
+    if config_name.startswith("mxfp8"):
+        return "mxfp8"
+    return "skinny" if config_name == "skinny" else "bf16"
 
 
 def load_peaks():
@@ -81,7 +95,7 @@ def profile_traffic(workload: str, config_name: str):
     except (OSError, ValueError):
         return None
     entry = t.get(f"{workload}:{config_name}")
-    if not entry or entry.get("kernel_source_hash") != kernel_source_hash():
+    if not entry or entry.get("kernel_source_hash") != kernel_source_hash(kernel_family(config_name)):
         return None
     return entry.get("dram_bytes_per_launch")
 
