@@ -34,7 +34,7 @@ using Cfg2x256F32C = b200::GemmBf16Cfg<2, 256, 6, 0, true>;
 using Cfg2x256B16C = b200::GemmBf16Cfg<2, 256, 6, 1, true>;
 using Cfg1x256F32C = b200::GemmBf16Cfg<1, 256, 4, 0, true>;
 using Cfg1x256B16C = b200::GemmBf16Cfg<1, 256, 4, 1, true>;
-using CfgMxf8 = b200::GemmMxf8Cfg<3>;
+using CfgMxf8 = b200::GemmMxf8Cfg<4>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
 using CfgSk64B16 = b200::GemmSkinnyCfg<64, 8, 1>;
 using CfgSk128F32 = b200::GemmSkinnyCfg<128, 6, 0>;
@@ -496,28 +496,22 @@ gemm_status_t launch_mxf8(DeviceState *st, const void *A, const uint8_t *sfa, co
     const int64_t b_blocks = 2 * ((N + 255) / 256);
 
     // 1. scales -> TMEM-ready 512-byte chunks
-    const int64_t words = (a_blocks + b_blocks) * kb * 128;
-    int64_t blocks = (words + 255) / 256;
-    if (blocks > static_cast<int64_t>(st->sm_count) * 16) blocks = static_cast<int64_t>(st->sm_count) * 16;
+    const int64_t blocks = (a_blocks + b_blocks) * ((kb + b200::kRepackKb - 1) / b200::kRepackKb);
     b200::mxf8_repack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         sfa, M, a_blocks, sfb, N, b_blocks, K / 32, kb, reinterpret_cast<uint32_t *>(ws));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
 
     // 2. the block-scaled GEMM
-    alignas(64) CUtensorMap tmA, tmB, tmC;
+    alignas(64) CUtensorMap tmA, tmB;
     if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, lda, Cfg::BK, Cfg::BM)) != GEMM_OK) return s;
     if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, ldb, Cfg::BK, Cfg::BN)) != GEMM_OK) return s;
-    const int64_t n_tma = (N * 2 / 16) * 16 / 2;
-    if ((s = encode_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, n_tma > 0 ? n_tma : 8, M, ldc * 2,
-                       Cfg::EPI_COLS, 32)) != GEMM_OK)
-        return s;
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     const int64_t grid = tiles < st->sm_count ? tiles : st->sm_count;
     const uint8_t *sfa_chunks = ws;
     const uint8_t *sfb_chunks = ws + a_blocks * kb * 512;
     kernel<<<static_cast<unsigned>(grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
-        tmA, tmB, tmC, sfa_chunks, sfb_chunks, static_cast<int>(M), static_cast<int>(N),
-        static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status, watchdog_ns(K));
+        tmA, tmB, sfa_chunks, sfb_chunks, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), C, ldc,
+        raster_group_m(), st->status, watchdog_ns(K));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }

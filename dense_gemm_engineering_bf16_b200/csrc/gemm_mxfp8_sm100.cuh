@@ -21,8 +21,8 @@
 //       warp 1 copies the stage's scales into TMEM (tcgen05.cp, two slots
 //       alternating) and issues 4 block-scaled MMAs (K = 32 each, the byte of
 //       the scale column chosen in the instruction descriptor); warps 2-5
-//       drain the accumulator as bf16 into a full-tile swizzled staging area,
-//       release TMEM at once, and write C with TMA stores.
+//       drain the accumulator to registers, release TMEM once the last
+//       columns are read, and write bf16 C with 16-byte global stores.
 //
 // TMEM: accumulator columns [0, 256); scale slot s at 256 + 32 s (A: 4
 // columns) and 256 + 32 s + 16 (B: 8 columns).  Every scale sits in lane
@@ -50,12 +50,10 @@ struct GemmMxf8Cfg {
     static constexpr int SFB_BYTES = 2 * SF_CHUNK;
     static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int STAGE_BYTES = ((TX_BYTES + 1023) / 1024) * 1024;
-    static constexpr int EPI_COLS = 64;            // bf16 columns per 128-byte staged row
+    static constexpr int EPI_COLS = 64;            // accumulator columns drained per step
     static constexpr int EPI_CHUNKS = BN / EPI_COLS;
-    static constexpr int EPI_BUF = 32 * 128;       // one 32-row x 128-byte box
-    static constexpr int EPI_BYTES = 4 * EPI_CHUNKS * EPI_BUF;  // each warp stages its whole 32 x 256 slice
     static constexpr int NUM_BARS = 2 * STAGES + 2;
-    static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL0 = 256;
@@ -65,45 +63,78 @@ struct GemmMxf8Cfg {
 
 // Row-major scales [rows][K/32] -> chunks [row block][K block][512], for
 // a_blocks row blocks of A followed by b_blocks row blocks of B; rows past
-// M (or N) and K steps past k32 read as 127.  One thread per 32-bit word.
-__global__ void mxf8_repack_scales_kernel(const uint8_t *__restrict__ sfa, int64_t M, int64_t a_blocks,
-                                          const uint8_t *__restrict__ sfb, int64_t N, int64_t b_blocks,
-                                          int64_t k32, int64_t kblocks, uint32_t *__restrict__ out) {
-    const int64_t words_per_chunk = 128;
-    const int64_t total = (a_blocks + b_blocks) * kblocks * words_per_chunk;
-    for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < total;
-         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t chunk = w / words_per_chunk;
-        const int64_t word = w - chunk * words_per_chunk;     // = r * 4 + q
-        const int64_t r = word >> 2;
-        const int64_t q = word & 3;
-        int64_t rb = chunk / kblocks;
-        const int64_t kb = chunk - rb * kblocks;
-        const uint8_t *src = sfa;
-        int64_t rows = M;
-        if (rb >= a_blocks) {
-            rb -= a_blocks;
-            src = sfb;
-            rows = N;
+// M (or N) and K steps past k32 read as 127.
+//
+// One CTA (256 threads) per (row block, group of kRepackKb K blocks): it
+// reads the 128 rows x (4 kRepackKb) scale bytes coalesced into shared
+// memory, then writes kRepackKb consecutive 512-byte chunks with 16-byte
+// stores (thread r of a chunk writes the four words of rows r, r+32, r+64,
+// r+96).
+constexpr int kRepackKb = 32;
+
+__global__ void __launch_bounds__(256)
+mxf8_repack_scales_kernel(const uint8_t *__restrict__ sfa, int64_t M, int64_t a_blocks,
+                          const uint8_t *__restrict__ sfb, int64_t N, int64_t b_blocks,
+                          int64_t k32, int64_t kblocks, uint32_t *__restrict__ out) {
+    __shared__ __align__(16) uint8_t tile[128][4 * kRepackKb];
+    const int64_t groups = (kblocks + kRepackKb - 1) / kRepackKb;
+    int64_t rb = static_cast<int64_t>(blockIdx.x) / groups;
+    const int64_t g = static_cast<int64_t>(blockIdx.x) - rb * groups;
+    const int64_t out_rb = rb;
+    const uint8_t *src = sfa;
+    int64_t rows = M;
+    if (rb >= a_blocks) {
+        rb -= a_blocks;
+        src = sfb;
+        rows = N;
+    }
+    const int64_t kb0 = g * kRepackKb;
+    const int64_t col0 = kb0 * 4;                      // first scale column of this group
+    // load: 128 rows x 128 bytes.  16-byte loads when every row starts on a
+    // 16-byte boundary (then a 16-byte piece is either wholly inside the row
+    // or wholly past it), else byte loads; consecutive threads read
+    // consecutive pieces of a row.
+    const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) && (k32 % 16 == 0);
+    if (vec) {
+        constexpr int kPieces = 4 * kRepackKb / 16;
+        for (int i = threadIdx.x; i < 128 * kPieces; i += blockDim.x) {
+            const int r = i / kPieces;
+            const int v = i - r * kPieces;
+            const int64_t row = rb * 128 + r;
+            const int64_t col = col0 + 16 * v;
+            uint4 x = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+            if (row < rows && col < k32) x = __ldg(reinterpret_cast<const uint4 *>(src + row * k32 + col));
+            *reinterpret_cast<uint4 *>(&tile[r][16 * v]) = x;
         }
-        const int64_t row = rb * 128 + q * 32 + r;
-        uint32_t v = 0;
+    } else {
+        for (int i = threadIdx.x; i < 128 * 4 * kRepackKb; i += blockDim.x) {
+            const int r = i / (4 * kRepackKb);
+            const int cidx = i - r * (4 * kRepackKb);
+            const int64_t row = rb * 128 + r;
+            const int64_t col = col0 + cidx;
+            tile[r][cidx] = (row < rows && col < k32) ? src[row * k32 + col] : static_cast<uint8_t>(127);
+        }
+    }
+    __syncthreads();
+    // store: chunk j of the group = 32 x 16-byte rows
+    const int nkb = static_cast<int>(kblocks - kb0 < kRepackKb ? kblocks - kb0 : kRepackKb);
+    for (int i = threadIdx.x; i < nkb * 32; i += blockDim.x) {
+        const int j = i / 32;
+        const int r = i - j * 32;
+        uint32_t w[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t ks = kb * 4 + j;
-            const uint32_t byte = (row < rows && ks < k32) ? src[row * k32 + ks] : 127u;
-            v |= byte << (8 * j);
-        }
-        out[w] = v;
+        for (int q = 0; q < 4; ++q)
+            w[q] = *reinterpret_cast<const uint32_t *>(&tile[32 * q + r][4 * j]);
+        uint4 *dst = reinterpret_cast<uint4 *>(out) + ((out_rb * kblocks + kb0 + j) * 32 + r);
+        *dst = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ CUtensorMap tmC, const uint8_t *sfa_chunks,
-                       const uint8_t *sfb_chunks, int M, int N, int K, void *C, int64_t ldc, int n_tma,
-                       int group_m, DeviceStatus *status, uint64_t timeout_ns) {
+                       const uint8_t *sfa_chunks, const uint8_t *sfb_chunks, int M, int N, int K, void *C,
+                       int64_t ldc, int group_m, DeviceStatus *status, uint64_t timeout_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -134,7 +165,6 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmB);
-        tma_prefetch_map(&tmC);
     }
     if (warp == 1) {
         tmem_alloc<1>(tmem_slot, Cfg::TMEM_COLS);
@@ -240,9 +270,11 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         __syncwarp();
     } else {
         // ----------------------------------------------------- epilogue --
+        // TMEM -> registers -> bf16 -> global, 16-byte stores: thread `lane`
+        // of warp `sub` owns row 32*sub + lane of the tile.  No shared-memory
+        // staging, so the whole SMEM budget goes to the operand ring; TMEM is
+        // handed back as soon as the last columns are in registers.
         const uint32_t sub = warp & 3u;
-        const uint32_t ew = warp - 2u;
-        const uint32_t sbuf = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * Cfg::EPI_CHUNKS * Cfg::EPI_BUF;
         int t = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
             int tm, tn;
@@ -255,59 +287,43 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             ready = __shfl_sync(0xffffffffu, ready, 0);
             if (!ready) break;
             tc_fence_after_sync();
-            // Drain the accumulator into this warp's staging slice (four
-            // 32 x 128-byte boxes, 128-byte swizzle), then hand TMEM back so
-            // the next tile's MMAs start while the stores drain.
             const uint32_t tbase = tmem_base + ((sub * 32u) << 16);
-            const int row0 = tm * Cfg::BM + static_cast<int>(sub) * 32;
+            const int row = tm * Cfg::BM + static_cast<int>(sub) * 32 + static_cast<int>(lane);
             const int col0 = tn * Cfg::BN;
-            const int row = row0 + static_cast<int>(lane);
-            if (lane == 0) bulk_wait_group_read<0>();   // last tile's stores are done reading
-            __syncwarp();
+            uint16_t *crow = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * 2);
 #pragma unroll 1
             for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
                 uint32_t v0[32], v1[32], packed[32];
-                tmem_ld_32x32b_x32(tbase + c * 64, v0);
-                tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
+                tmem_ld_32x32b_x32(tbase + c * Cfg::EPI_COLS, v0);
+                tmem_ld_32x32b_x32(tbase + c * Cfg::EPI_COLS + 32, v1);
                 tmem_ld_wait();
+                if (c == Cfg::EPI_CHUNKS - 1) {
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_local(tempty_bar);
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
                     packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
                 }
                 const int cstart = col0 + c * Cfg::EPI_COLS;
-                if (cstart < N && cstart + Cfg::EPI_COLS > n_tma && row < M) {
-                    // the row's last partial 16-byte granule: plain stores
-                    uint16_t *crow = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(C) +
-                                                                  static_cast<int64_t>(row) * ldc * 2);
+                if (row >= M || cstart >= N) continue;
 #pragma unroll
-                    for (int w = 0; w < Cfg::EPI_COLS; ++w) {
-                        const int col = cstart + w;
-                        if (col >= n_tma && col < N)
-                            crow[col] = static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
+                for (int v = 0; v < 8; ++v) {                 // 8 bf16 = 16 bytes per store
+                    const int col = cstart + 8 * v;
+                    if (col + 8 <= N) {
+                        *reinterpret_cast<uint4 *>(crow + col) =
+                            make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            if (col + e < N)
+                                crow[col + e] = static_cast<uint16_t>(packed[4 * v + (e >> 1)] >> (16 * (e & 1)));
                     }
                 }
-                const uint32_t row_addr = sbuf + c * Cfg::EPI_BUF + lane * 128u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4),
-                                 packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                }
-            }
-            tc_fence_before_sync();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_local(tempty_bar);
-                for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
-                    const int cstart = col0 + c * Cfg::EPI_COLS;
-                    if (cstart < n_tma) tma_store_2d(&tmC, sbuf + c * Cfg::EPI_BUF, cstart, row0);
-                }
-                bulk_commit_group();
             }
         }
-        if (lane == 0) bulk_wait_group<0>();
-        __syncwarp();
     }
 
     tc_fence_before_sync();

@@ -120,3 +120,28 @@ def test_mxfp8_8192_cube():
     half_ulp = (2.0 ** -8) * np.abs(got)
     assert np.all(np.abs(got.sum(axis=1) - r) <= 1e-3 * r_mag + 1e-6 * N + half_ulp.sum(axis=1))
     assert np.all(np.abs(got.sum(axis=0) - cl) <= 1e-3 * cl_mag + 1e-6 * M + half_ulp.sum(axis=0))
+
+
+def test_unaligned_scale_pointers_take_the_byte_path():
+    """Scales may sit at any address: at K = 1024 (scale rows of 32 bytes) an
+    offset of one byte forces the repack's byte-load path."""
+    import torch
+    M, N, K = 200, 300, 1024
+    a, sfa, b, sfb = synth.mxfp8_operands(M, N, K, workload=47)
+
+    def dev_off(x):
+        buf = torch.zeros(x.size + 16, dtype=torch.uint8, device="cuda")
+        buf[1:1 + x.size] = torch.from_numpy(np.ascontiguousarray(x).reshape(-1)).cuda()
+        return buf, buf.data_ptr() + 1
+
+    A = torch.from_numpy(a).cuda()
+    B = torch.from_numpy(b).cuda()
+    SA, pa = dev_off(sfa)
+    SB, pb = dev_off(sfb)
+    ldc = 312                                  # 624-byte rows: a multiple of 16
+    C = torch.zeros((M, ldc), dtype=torch.bfloat16, device="cuda")
+    G.gemm_mxfp8(A, pa, B, pb, C, M, N, K, K, K, ldc)
+    G.gemm_check_device_status()
+    got = oracle.decode_bf16(C.cpu().view(torch.int16).numpy().view(np.uint16))[:, :N]
+    c_ref, s_abs = oracle.gemm_mxfp8_f64(a, sfa, b, sfb, with_abs=True)
+    assert_close(got, c_ref, s_abs, BF16, "unaligned scales")
