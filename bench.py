@@ -335,8 +335,12 @@ def main():
     dev = p.device_arrays(torch)
     C = p.empty_out(torch)
     G.gemm_force_config(args.config)
-    cfg_name = "mxfp8_128x256" if p.kind == "mxfp8" else \
-        {v: k for k, v in G.CONFIGS.items()}[G.gemm_select_config(p.M, p.N, p.K)]
+    if p.kind == "mxfp8":
+        pair_tiles = ((p.M + 255) // 256) * ((p.N + 255) // 256)
+        cfg_name = args.config if args.config.startswith("mxfp8") else \
+            ("mxfp8_2cta_256x256" if pair_tiles >= 74 else "mxfp8_1cta_128x256")
+    else:
+        cfg_name = {v: k for k, v in G.CONFIGS.items()}[G.gemm_select_config(p.M, p.N, p.K)]
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):

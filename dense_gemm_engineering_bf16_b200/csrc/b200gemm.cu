@@ -34,7 +34,8 @@ using Cfg2x256F32C = b200::GemmBf16Cfg<2, 256, 6, 0, true>;
 using Cfg2x256B16C = b200::GemmBf16Cfg<2, 256, 6, 1, true>;
 using Cfg1x256F32C = b200::GemmBf16Cfg<1, 256, 4, 0, true>;
 using Cfg1x256B16C = b200::GemmBf16Cfg<1, 256, 4, 1, true>;
-using CfgMxf8 = b200::GemmMxf8Cfg<4>;
+using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
+using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
 using CfgSk64B16 = b200::GemmSkinnyCfg<64, 8, 1>;
 using CfgSk128F32 = b200::GemmSkinnyCfg<128, 6, 0>;
@@ -52,8 +53,9 @@ struct DeviceState {
     // per (config, out type): smem attribute set, co-resident clusters
     bool attr_done[GEMM_CFG_COUNT_][2] = {};
     int max_clusters[GEMM_CFG_COUNT_][2] = {};
-    // block-scaled path: kernel attribute set, repacked-scale workspace
-    bool mx_attr_done = false;
+    // block-scaled path: kernel attributes (1-CTA, pair), repacked-scale workspace
+    bool mx_attr_done[2] = {};
+    int mx_max_clusters[2] = {};
     uint8_t *mx_ws = nullptr;
     size_t mx_ws_bytes = 0;
     // skinny path: kernel attributes (per template), split-tile workspace
@@ -188,13 +190,14 @@ gemm_status_t check_args(const void *A, const void *B, const void *C, int64_t M,
 // ------------------------------------------------------------ tensor maps --
 
 gemm_status_t encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, int64_t inner,
-                        int64_t outer, int64_t ld_bytes, uint32_t box_inner, uint32_t box_outer) {
+                        int64_t outer, int64_t ld_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_bytes)};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, dtype, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         g_last_cuda_error = static_cast<int>(r);
@@ -207,7 +210,7 @@ gemm_status_t encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void 
 
 gemm_config_t select_config(int64_t M, int64_t N, int64_t /*K*/) {
     const int forced = g_forced.load(std::memory_order_relaxed);
-    if (forced != GEMM_CFG_AUTO) return static_cast<gemm_config_t>(forced);
+    if (forced != GEMM_CFG_AUTO && forced < GEMM_CFG_MXFP8_1CTA_128x256) return static_cast<gemm_config_t>(forced);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int64_t wide_tiles = ((M + 127) / 128) * ((N + 255) / 256);
     // two or more waves of pair tiles: Cluster Launch Control evens out the
@@ -445,13 +448,30 @@ gemm_status_t noalloc_device(int &dev, DeviceState *&st) {
 
 // ------------------------------------------------------ block-scaled path --
 
-// Bytes of repacked scales for an M x N x K problem: 512 per (128-row block,
-// 128-wide K block) of A, and of B padded to whole 256-row tiles.
-size_t mx_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    const int64_t kb = (K + 127) / 128;
-    const int64_t a_blocks = (M + 127) / 128;
-    const int64_t b_blocks = 2 * ((N + 255) / 256);
-    return static_cast<size_t>((a_blocks + b_blocks) * kb * 512);
+// Block-scaled configuration: CTA pairs (256 x 256) once there is a full wave
+// of pair tiles, single CTAs (128 x 256) below that.
+gemm_config_t select_mx_config(int64_t M, int64_t N) {
+    const int forced = g_forced.load(std::memory_order_relaxed);
+    if (forced == GEMM_CFG_MXFP8_1CTA_128x256 || forced == GEMM_CFG_MXFP8_2CTA_256x256)
+        return static_cast<gemm_config_t>(forced);
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    return pair_tiles >= 74 ? GEMM_CFG_MXFP8_2CTA_256x256 : GEMM_CFG_MXFP8_1CTA_128x256;
+}
+
+// Repacked-scale layout: 512-byte chunks, row block major ([rb][kb]).  A has
+// a_blocks row blocks (padded to whole tiles), B has b_blocks (whole 256-row
+// tiles); B's chunks follow A's.
+struct MxLayout {
+    int64_t kb, a_blocks, b_blocks;
+    size_t bytes() const { return static_cast<size_t>((a_blocks + b_blocks) * kb * 512); }
+};
+
+MxLayout mx_layout(int64_t M, int64_t N, int64_t K, int cg) {
+    MxLayout l;
+    l.kb = (K + 127) / 128;
+    l.a_blocks = cg == 2 ? 2 * ((M + 255) / 256) : (M + 127) / 128;
+    l.b_blocks = 2 * ((N + 255) / 256);
+    return l;
 }
 
 // Grows the device's workspace on demand.  cudaFree waits for the device to
@@ -473,46 +493,66 @@ gemm_status_t mx_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
     return GEMM_OK;
 }
 
-gemm_status_t launch_mxf8(DeviceState *st, const void *A, const uint8_t *sfa, const void *B,
+template <class Cfg>
+gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const uint8_t *sfa, const void *B,
                           const uint8_t *sfb, void *C, int64_t M, int64_t N, int64_t K, int64_t lda,
                           int64_t ldb, int64_t ldc, cudaStream_t stream) {
-    using Cfg = CfgMxf8;
     auto kernel = b200::gemm_mxf8_sm100_kernel<Cfg>;
     cudaError_t e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Cfg::CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.blockDim = dim3(Cfg::THREADS, 1, 1);
+    lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    lc.stream = stream;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
     {
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (!st->mx_attr_done) {
+        if (!st->mx_attr_done[attr_slot]) {
             if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           Cfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
-            st->mx_attr_done = true;
+            int clusters = st->sm_count / Cfg::CG;
+            if (Cfg::CG > 1) {
+                lc.gridDim = dim3(Cfg::CG * clusters, 1, 1);
+                int n = 0;
+                if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
+                if (n > 0) clusters = n;
+            }
+            st->mx_max_clusters[attr_slot] = clusters;
+            st->mx_attr_done[attr_slot] = true;
         }
     }
+    const MxLayout l = mx_layout(M, N, K, Cfg::CG);
     uint8_t *ws = nullptr;
     gemm_status_t s;
-    if ((s = mx_workspace(st, mx_workspace_bytes(M, N, K), ws)) != GEMM_OK) return s;
-    const int64_t kb = (K + 127) / 128;
-    const int64_t a_blocks = (M + 127) / 128;
-    const int64_t b_blocks = 2 * ((N + 255) / 256);
+    if ((s = mx_workspace(st, l.bytes(), ws)) != GEMM_OK) return s;
 
     // 1. scales -> TMEM-ready 512-byte chunks
-    const int64_t blocks = (a_blocks + b_blocks) * ((kb + b200::kRepackKb - 1) / b200::kRepackKb);
+    const int64_t blocks = (l.a_blocks + l.b_blocks) * ((l.kb + b200::kRepackKb - 1) / b200::kRepackKb);
     b200::mxf8_repack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        sfa, M, a_blocks, sfb, N, b_blocks, K / 32, kb, reinterpret_cast<uint32_t *>(ws));
+        sfa, M, l.a_blocks, sfb, N, l.b_blocks, K / 32, l.kb, reinterpret_cast<uint32_t *>(ws));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
 
-    // 2. the block-scaled GEMM
-    alignas(64) CUtensorMap tmA, tmB;
-    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, lda, Cfg::BK, Cfg::BM)) != GEMM_OK) return s;
-    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, ldb, Cfg::BK, Cfg::BN)) != GEMM_OK) return s;
+    // 2. the block-scaled GEMM; the scale chunks are read through a map that
+    // sees the workspace as rows of 128 x 32-bit words (one chunk per row)
+    alignas(64) CUtensorMap tmA, tmB, tmSF;
+    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, lda, Cfg::BK, Cfg::BM_CTA)) != GEMM_OK) return s;
+    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, ldb, Cfg::BK, Cfg::B_ROWS)) != GEMM_OK) return s;
+    if ((s = encode_2d(&tmSF, CU_TENSOR_MAP_DATA_TYPE_UINT32, ws, 128, (l.a_blocks + l.b_blocks) * l.kb, 512, 128, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != GEMM_OK)
+        return s;
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
-    const int64_t grid = tiles < st->sm_count ? tiles : st->sm_count;
-    const uint8_t *sfa_chunks = ws;
-    const uint8_t *sfb_chunks = ws + a_blocks * kb * 512;
-    kernel<<<static_cast<unsigned>(grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
-        tmA, tmB, sfa_chunks, sfb_chunks, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), C, ldc,
-        raster_group_m(), st->status, watchdog_ns(K));
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    const int64_t clusters = tiles < st->mx_max_clusters[attr_slot] ? tiles : st->mx_max_clusters[attr_slot];
+    lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
+    e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmSF, static_cast<int64_t>(l.a_blocks * l.kb),
+                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), C, ldc, raster_group_m(),
+                           st->status, watchdog_ns(K));
+    if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
 
@@ -574,7 +614,9 @@ gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const
     DeviceState *st;
     if ((s = current_device(dev, st)) != GEMM_OK) return s;
     if (K == 0) return launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
-    return launch_mxf8(st, A, sfa, B, sfb, C, M, N, K, lda, ldb, ldc, stream);
+    if (select_mx_config(M, N) == GEMM_CFG_MXFP8_2CTA_256x256)
+        return launch_mxf8<CfgMxf8Pair>(st, 1, A, sfa, B, sfb, C, M, N, K, lda, ldb, ldc, stream);
+    return launch_mxf8<CfgMxf8>(st, 0, A, sfa, B, sfb, C, M, N, K, lda, ldb, ldc, stream);
 }
 
 gemm_status_t gemm_check_device_status(cudaStream_t stream) {

@@ -15,11 +15,15 @@
 //       r*16 + q*4 + j holds the scale of row 32q + r for the j-th 32-wide
 //       K step.  Padding rows and K steps get 127 (2^0), so zero-filled
 //       operand tails stay zero.
-//   gemm_mxf8_sm100_kernel  persistent, warp-specialised, one CTA per
-//       128 x 256 tile, BK = 128 (one 128-byte swizzle row of E4M3):
-//       warp 0 loads A and B by TMA and the scale chunks by 1-D bulk copy;
-//       warp 1 copies the stage's scales into TMEM (tcgen05.cp, two slots
-//       alternating) and issues 4 block-scaled MMAs (K = 32 each, the byte of
+//   gemm_mxf8_sm100_kernel  persistent, warp-specialised, one CTA (CG = 1,
+//       128 x 256 tile) or a CTA pair (CG = 2, 256 x 256 tile, cta_group::2)
+//       per tile, BK = 128 (one 128-byte swizzle row of E4M3):
+//       warp 0 loads A, B and the scale chunks by TMA (for a pair, every
+//       byte counts on the leader's barrier; each CTA holds its own 128 rows
+//       of A scales and the scales of all 256 rows of B);
+//       warp 1 of the (leader) CTA copies the stage's scales into TMEM
+//       (tcgen05.cp, cta_group::2 for a pair: each CTA's SMEM to its own
+//       TMEM; two slots alternating) and issues 4 block-scaled MMAs (K = 32 each, the byte of
 //       the scale column chosen in the instruction descriptor); warps 2-5
 //       drain the accumulator to registers, release TMEM once the last
 //       columns are read, and write bf16 C with 16-byte global stores.
@@ -35,21 +39,25 @@
 
 namespace b200 {
 
-template <int STAGES_>
+template <int CG_, int STAGES_>
 struct GemmMxf8Cfg {
+    static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
     static constexpr int STAGES = STAGES_;
-    static constexpr int BM = 128;
-    static constexpr int BN = 256;
+    static constexpr int BM_CTA = 128;             // accumulator rows per CTA
+    static constexpr int BM = 128 * CG;            // tile M == MMA M
+    static constexpr int BN = 256;                 // tile N == MMA N
+    static constexpr int B_ROWS = BN / CG;         // rows of B this CTA loads
     static constexpr int BK = 128;                 // E4M3 elements (bytes) per k-tile
     static constexpr int UMMA_K = 32;              // K per block-scaled MMA
     static constexpr int MMAS = BK / UMMA_K;       // 4, one scale byte each
-    static constexpr int A_BYTES = BM * BK;
-    static constexpr int B_BYTES = BN * BK;
+    static constexpr int A_BYTES = BM_CTA * BK;
+    static constexpr int B_BYTES = B_ROWS * BK;
     static constexpr int SF_CHUNK = 512;           // scales of 128 rows x 4 K steps
-    static constexpr int SFA_BYTES = SF_CHUNK;
-    static constexpr int SFB_BYTES = 2 * SF_CHUNK;
-    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int STAGE_BYTES = ((TX_BYTES + 1023) / 1024) * 1024;
+    static constexpr int SFA_BYTES = SF_CHUNK;     // this CTA's 128 rows of A
+    static constexpr int SFB_BYTES = 2 * SF_CHUNK; // all 256 rows of B (every CTA needs them)
+    static constexpr int CTA_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int TX_BYTES = CTA_BYTES * CG;  // bytes landing on the leader's full[s]
+    static constexpr int STAGE_BYTES = ((CTA_BYTES + 1023) / 1024) * 1024;
     static constexpr int EPI_COLS = 64;            // accumulator columns drained per step
     static constexpr int EPI_CHUNKS = BN / EPI_COLS;
     static constexpr int NUM_BARS = 2 * STAGES + 2;
@@ -58,6 +66,8 @@ struct GemmMxf8Cfg {
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL0 = 256;
     static constexpr int THREADS = 192;
+    static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
+    static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows");
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
 };
 
@@ -133,14 +143,19 @@ mxf8_repack_scales_kernel(const uint8_t *__restrict__ sfa, int64_t M, int64_t a_
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const uint8_t *sfa_chunks, const uint8_t *sfb_chunks, int M, int N, int K, void *C,
-                       int64_t ldc, int group_m, DeviceStatus *status, uint64_t timeout_ns) {
+                       const __grid_constant__ CUtensorMap tmSF, int64_t sfb_row0, int M, int N, int K,
+                       void *C, int64_t ldc, int group_m, DeviceStatus *status, uint64_t timeout_ns) {
+    // tmSF views the repacked scales as rows of 512 bytes (128 x 32-bit):
+    // row rb * num_kb + kb is the chunk of 128-row block rb at K block kb; the
+    // blocks of B start at row sfb_row0.
+    constexpr int CG = Cfg::CG;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     const uint32_t base = smem_addr(smem);
     const uint32_t warp = threadIdx.x / 32;
     const uint32_t lane = threadIdx.x % 32;
+    const uint32_t rank = (CG == 2) ? cluster_cta_rank() : 0u;
 
     const uint32_t bar0 = base + Cfg::BAR_OFF;
     auto full_bar = [&](uint32_t s) { return bar0 + 8u * s; };
@@ -158,20 +173,22 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
-        mbar_init(tempty_bar, 4);
+        mbar_init(tempty_bar, 4 * CG);
         *abort_flag = 0u;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmB);
+        tma_prefetch_map(&tmSF);
     }
     if (warp == 1) {
-        tmem_alloc<1>(tmem_slot, Cfg::TMEM_COLS);
-        tmem_relinquish<1>();
+        tmem_alloc<CG>(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish<CG>();
     }
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot_ptr;
 
@@ -179,21 +196,25 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + Cfg::BK - 1) / Cfg::BK;
+    const int cluster_id = static_cast<int>(blockIdx.x) / CG;
+    const int num_clusters = static_cast<int>(gridDim.x) / CG;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
                 int tm, tn;
                 raster_tile(tile, num_m, num_n, group_m, tm, tn);
-                const uint8_t *sfa_row = sfa_chunks + static_cast<int64_t>(tm) * num_kb * Cfg::SF_CHUNK;
-                const uint8_t *sfb_row0 = sfb_chunks + static_cast<int64_t>(2 * tn) * num_kb * Cfg::SF_CHUNK;
-                const uint8_t *sfb_row1 = sfb_row0 + static_cast<int64_t>(num_kb) * Cfg::SF_CHUNK;
+                const int a_rb = tm * CG + static_cast<int>(rank);         // this CTA's 128-row block of A
+                const int a_row = a_rb * Cfg::BM_CTA;
+                const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
+                const int sfa_y = a_rb * num_kb;
+                const int sfb_y = static_cast<int>(sfb_row0) + (2 * tn) * num_kb;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarEmpty);
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarEmpty);
                         ok = false;
                         break;
                     }
@@ -201,20 +222,30 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                     const uint32_t b_dst = a_dst + Cfg::A_BYTES;
                     const uint32_t sfa_dst = b_dst + Cfg::B_BYTES;
                     const uint32_t sfb_dst = sfa_dst + Cfg::SFA_BYTES;
-                    const uint32_t fb = full_bar(stage);
-                    mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
-                    tma_load_2d(a_dst, &tmA, fb, kb * Cfg::BK, tm * Cfg::BM);
-                    tma_load_2d(b_dst, &tmB, fb, kb * Cfg::BK, tn * Cfg::BN);
-                    const int64_t off = static_cast<int64_t>(kb) * Cfg::SF_CHUNK;
-                    bulk_load_1d(sfa_dst, sfa_row + off, Cfg::SF_CHUNK, fb);
-                    bulk_load_1d(sfb_dst, sfb_row0 + off, Cfg::SF_CHUNK, fb);
-                    bulk_load_1d(sfb_dst + Cfg::SF_CHUNK, sfb_row1 + off, Cfg::SF_CHUNK, fb);
+                    const int kx = kb * Cfg::BK;
+                    if constexpr (CG == 1) {
+                        const uint32_t fb = full_bar(stage);
+                        mbar_arrive_expect_tx(fb, Cfg::TX_BYTES);
+                        tma_load_2d(a_dst, &tmA, fb, kx, a_row);
+                        tma_load_2d(b_dst, &tmB, fb, kx, b_row);
+                        tma_load_2d(sfa_dst, &tmSF, fb, 0, sfa_y + kb);
+                        tma_load_2d(sfb_dst, &tmSF, fb, 0, sfb_y + kb);
+                        tma_load_2d(sfb_dst + Cfg::SF_CHUNK, &tmSF, fb, 0, sfb_y + num_kb + kb);
+                    } else {
+                        if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
+                        const uint32_t fb = map_to_cta(full_bar(stage), 0);
+                        tma_load_2d_pair(a_dst, &tmA, fb, kx, a_row);
+                        tma_load_2d_pair(b_dst, &tmB, fb, kx, b_row);
+                        tma_load_2d_pair(sfa_dst, &tmSF, fb, 0, sfa_y + kb);
+                        tma_load_2d_pair(sfb_dst, &tmSF, fb, 0, sfb_y + kb);
+                        tma_load_2d_pair(sfb_dst + Cfg::SF_CHUNK, &tmSF, fb, 0, sfb_y + num_kb + kb);
+                    }
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarTail);
+                    record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarTail);
                     ok = false;
                 }
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -222,21 +253,21 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------- scale copy + MMA issuer --
-        if (lane == 0) {
+        // -------------------------- scale copy + MMA issuer (pair leader) --
+        if (rank == 0 && lane == 0) {
             uint32_t stage = 0, phase = 0, sf_slot = 0;
             bool ok = true;
             int t = 0;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++t) {
+            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters, ++t) {
                 if (!mbar_wait(tempty_bar, (static_cast<uint32_t>(t) & 1u) ^ 1u, abort_flag, 3 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarTmemEmpty);
+                    record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarTmemEmpty);
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarFull);
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarFull);
                         ok = false;
                         break;
                     }
@@ -249,46 +280,56 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                     const uint32_t sfb_t = sfa_t + 16u;
                     // tcgen05.cp and tcgen05.mma issued by one thread execute in
                     // issue order, so the MMAs below see these scales.
-                    tmem_cp_32x128b_warpx4(sfa_t, rows16_desc(sfa_smem));
-                    tmem_cp_32x128b_warpx4(sfb_t, rows16_desc(sfb_smem));
-                    tmem_cp_32x128b_warpx4(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+                    if constexpr (CG == 1) {
+                        tmem_cp_32x128b_warpx4(sfa_t, rows16_desc(sfa_smem));
+                        tmem_cp_32x128b_warpx4(sfb_t, rows16_desc(sfb_smem));
+                        tmem_cp_32x128b_warpx4(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+                    } else {
+                        tmem_cp_32x128b_warpx4_pair(sfa_t, rows16_desc(sfa_smem));
+                        tmem_cp_32x128b_warpx4_pair(sfb_t, rows16_desc(sfb_smem));
+                        tmem_cp_32x128b_warpx4_pair(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+                    }
 #pragma unroll
                     for (int j = 0; j < Cfg::MMAS; ++j) {
-                        mma_mxf8_ss(tmem_base, sw128_kmajor_desc(a0 + j * 32), sw128_kmajor_desc(b0 + j * 32),
-                                    idesc_mxf8_e8m0(Cfg::BM, Cfg::BN, static_cast<uint32_t>(j),
-                                                    static_cast<uint32_t>(j)),
-                                    sfa_t, sfb_t, (kb | j) != 0 ? 1u : 0u);
+                        const uint32_t idesc = idesc_mxf8_e8m0(Cfg::BM, Cfg::BN, static_cast<uint32_t>(j),
+                                                               static_cast<uint32_t>(j));
+                        const uint64_t ad = sw128_kmajor_desc(a0 + j * 32);
+                        const uint64_t bd = sw128_kmajor_desc(b0 + j * 32);
+                        const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+                        if constexpr (CG == 1) mma_mxf8_ss(tmem_base, ad, bd, idesc, sfa_t, sfb_t, acc);
+                        else mma_mxf8_ss_pair(tmem_base, ad, bd, idesc, sfa_t, sfb_t, acc);
                     }
-                    mma_commit<1>(empty_bar(stage), 0);
+                    mma_commit<CG>(empty_bar(stage), 0x3);
                     sf_slot ^= 1u;
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                mma_commit<1>(tfull_bar, 0);
+                mma_commit<CG>(tfull_bar, 0x3);
             }
         }
         __syncwarp();
     } else {
         // ----------------------------------------------------- epilogue --
         // TMEM -> registers -> bf16 -> global, 16-byte stores: thread `lane`
-        // of warp `sub` owns row 32*sub + lane of the tile.  No shared-memory
-        // staging, so the whole SMEM budget goes to the operand ring; TMEM is
-        // handed back as soon as the last columns are in registers.
+        // of warp `sub` owns row 32*sub + lane of this CTA's 128 rows.  No
+        // shared-memory staging, so the whole SMEM budget goes to the operand
+        // ring; TMEM is handed back once the last columns are in registers.
         const uint32_t sub = warp & 3u;
         int t = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+        for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++t) {
             int tm, tn;
             raster_tile(tile, num_m, num_n, group_m, tm, tn);
             uint32_t ready = 1;
             if (lane == 0 && !mbar_wait(tfull_bar, static_cast<uint32_t>(t) & 1u, abort_flag, 3 * timeout_ns)) {
-                record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
+                record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarTmemFull);
                 ready = 0;
             }
             ready = __shfl_sync(0xffffffffu, ready, 0);
             if (!ready) break;
             tc_fence_after_sync();
             const uint32_t tbase = tmem_base + ((sub * 32u) << 16);
-            const int row = tm * Cfg::BM + static_cast<int>(sub) * 32 + static_cast<int>(lane);
+            const int row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32 +
+                            static_cast<int>(lane);
             const int col0 = tn * Cfg::BN;
             uint16_t *crow = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * 2);
 #pragma unroll 1
@@ -300,7 +341,10 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                 if (c == Cfg::EPI_CHUNKS - 1) {
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_local(tempty_bar);
+                    if (lane == 0) {
+                        if constexpr (CG == 1) mbar_arrive_local(tempty_bar);
+                        else mbar_arrive_cluster(map_to_cta(tempty_bar, 0));
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -328,14 +372,16 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();
     if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
     }
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc<1>(tmem_base, Cfg::TMEM_COLS);
+        tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
     }
 }
 

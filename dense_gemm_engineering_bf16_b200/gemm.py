@@ -31,6 +31,8 @@ CONFIGS = {
     "skinny": 4,
     "2cta_256x256_clc": 5,
     "1cta_128x256_clc": 6,
+    "mxfp8_1cta_128x256": 7,
+    "mxfp8_2cta_256x256": 8,
 }
 
 STATUS_NAMES = {

@@ -81,7 +81,9 @@ typedef enum {
     GEMM_CFG_2CTA_256x256_CLC = 5,  /* as 2CTA_256x256, tiles handed out by Cluster Launch Control:
                                        one cluster per tile, running pairs claim pending ones */
     GEMM_CFG_1CTA_128x256_CLC = 6,  /* as 1CTA_128x256 with Cluster Launch Control */
-    GEMM_CFG_COUNT_ = 7
+    GEMM_CFG_MXFP8_1CTA_128x256 = 7,/* gemm_mxfp8: one CTA per 128 x 256 tile */
+    GEMM_CFG_MXFP8_2CTA_256x256 = 8,/* gemm_mxfp8: CTA pair per 256 x 256 tile, cta_group::2 */
+    GEMM_CFG_COUNT_ = 9
 } gemm_config_t;
 
 /*
@@ -180,7 +182,9 @@ B200GEMM_API const char *gemm_status_string(gemm_status_t status);
 B200GEMM_API int gemm_last_cuda_error(void);
 
 /* Force a kernel configuration for subsequent calls in this process
- * (GEMM_CFG_AUTO restores shape-based selection).  Returns
+ * (GEMM_CFG_AUTO restores shape-based selection).  A gemm_bf16
+ * configuration applies to gemm_bf16 / gemm_bf16_noalloc, an MXFP8 one to
+ * gemm_mxfp8; the other entry points keep choosing by shape.  Returns
  * GEMM_ERR_INVALID_VALUE for an unknown configuration. */
 B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
 

@@ -132,7 +132,7 @@ def sample_indices(n: int, tile: int, extra: int, seed: int) -> np.ndarray:
 
 
 def run_mxfp8(a_codes: np.ndarray, sfa: np.ndarray, b_codes: np.ndarray, sfb: np.ndarray,
-              M: int, N: int, K: int, ldc: int | None = None):
+              M: int, N: int, K: int, ldc: int | None = None, config: str = "auto"):
     """Run the block-scaled GEMM through the C ABI; returns the GuardedC (bf16)."""
     lda = a_codes.shape[1] if a_codes.size else 16
     ldb = b_codes.shape[1] if b_codes.size else 16
@@ -145,7 +145,11 @@ def run_mxfp8(a_codes: np.ndarray, sfa: np.ndarray, b_codes: np.ndarray, sfb: np
 
     A, B, SA, SB = dev(a_codes), dev(b_codes), dev(sfa), dev(sfb)
     C = GuardedC(M, N, ldc, G.OUT_BF16)
-    G.gemm_mxfp8(A, SA, B, SB, C.ptr, M, N, K, lda, ldb, ldc)
+    G.gemm_force_config(config)
+    try:
+        G.gemm_mxfp8(A, SA, B, SB, C.ptr, M, N, K, lda, ldb, ldc)
+    finally:
+        G.gemm_force_config("auto")
     G.gemm_check_device_status()
     torch.cuda.synchronize()
     return C

@@ -18,6 +18,7 @@ from gpu_helpers import assert_close, assert_exact, run_mxfp8, sample_indices
 
 pytestmark = pytest.mark.gpu
 BF16 = G.OUT_BF16
+MX_CFGS = ["mxfp8_1cta_128x256", "mxfp8_2cta_256x256"]
 
 
 def _int_operands(M, N, K, seed, exp_lo=0, exp_hi=0):
@@ -28,8 +29,8 @@ def _int_operands(M, N, K, seed, exp_lo=0, exp_hi=0):
     return a, sfa, b, sfb
 
 
-def _check(a, sfa, b, sfb, M, N, K, exact=False, ldc=None):
-    C = run_mxfp8(a, sfa, b, sfb, M, N, K, ldc=ldc)
+def _check(a, sfa, b, sfb, M, N, K, exact=False, ldc=None, cfg="auto"):
+    C = run_mxfp8(a, sfa, b, sfb, M, N, K, ldc=ldc, config=cfg)
     got, guard_ok = C.download()
     assert guard_ok, "write outside C's M x N window"
     c_ref, s_abs = oracle.gemm_mxfp8_f64(a, sfa, b, sfb, K=K, with_abs=True)
@@ -39,29 +40,34 @@ def _check(a, sfa, b, sfb, M, N, K, exact=False, ldc=None):
         assert_close(got, c_ref, s_abs, BF16, f"mxfp8 {M}x{N}x{K}")
 
 
-def test_single_tile_unit_scales_bit_exact():
-    _check(*_int_operands(128, 256, 128, seed=1), 128, 256, 128, exact=True)
+@pytest.mark.parametrize("cfg", MX_CFGS)
+def test_single_tile_unit_scales_bit_exact(cfg):
+    _check(*_int_operands(128, 256, 128, seed=1), 128, 256, 128, exact=True, cfg=cfg)
 
 
-def test_scaled_integers_bit_exact():
+@pytest.mark.parametrize("cfg", MX_CFGS)
+def test_scaled_integers_bit_exact(cfg):
     # exponents in [-1, 1]: every partial sum is a multiple of 2^-2 below 2^22
     M, N, K = 256, 512, 1024
-    _check(*_int_operands(M, N, K, seed=5, exp_lo=-1, exp_hi=1), M, N, K, exact=True)
+    _check(*_int_operands(M, N, K, seed=5, exp_lo=-1, exp_hi=1), M, N, K, exact=True, cfg=cfg)
 
 
-def test_random_values_and_scales_multi_tile():
-    M, N, K = 384, 768, 1024
+@pytest.mark.parametrize("cfg", MX_CFGS)
+def test_random_values_and_scales_multi_tile(cfg):
+    M, N, K = 640, 768, 1024
     a, sfa, b, sfb = synth.mxfp8_operands(M, N, K, workload=40)
-    _check(a, sfa, b, sfb, M, N, K)
+    _check(a, sfa, b, sfb, M, N, K, cfg=cfg)
 
 
+@pytest.mark.parametrize("cfg", MX_CFGS)
 @pytest.mark.parametrize("shape", [(1, 8, 32), (3, 5, 32), (127, 129, 96), (200, 300, 160),
-                                   (129, 257, 64), (300, 40, 544), (1, 1000, 256)],
+                                   (129, 257, 64), (300, 40, 544), (1, 1000, 256), (257, 513, 4000)],
                          ids=lambda s: "x".join(map(str, s)))
-def test_ragged_tails(shape):
+def test_ragged_tails(shape, cfg):
     M, N, K = shape
+    K = K // 32 * 32
     a, sfa, b, sfb = synth.mxfp8_operands(M, N, K, workload=41 + M)
-    _check(a, sfa, b, sfb, M, N, K)
+    _check(a, sfa, b, sfb, M, N, K, cfg=cfg)
 
 
 def test_strided_operands():
@@ -87,11 +93,12 @@ def test_k_zero_writes_zeros():
     assert guard_ok and np.all(got == 0)
 
 
-def test_nan_scale_poisons_its_block_only():
+@pytest.mark.parametrize("cfg", MX_CFGS)
+def test_nan_scale_poisons_its_block_only(cfg):
     M, N, K = 130, 140, 128
     a, sfa, b, sfb = synth.mxfp8_operands(M, N, K, workload=46)
     sfa[7, 2] = 0xFF
-    C = run_mxfp8(a, sfa, b, sfb, M, N, K)
+    C = run_mxfp8(a, sfa, b, sfb, M, N, K, config=cfg)
     got, _ = C.download()
     c_ref, s_abs = oracle.gemm_mxfp8_f64(a, sfa, b, sfb, with_abs=True)
     assert np.isnan(got[7]).all() and not np.isnan(np.delete(got, 7, axis=0)).any()
@@ -103,11 +110,13 @@ def test_rejects_k_not_multiple_of_32():
                             0x7F0000400000, 64, 64, 48, 48, 48, 64, 0) == 1
 
 
-def test_mxfp8_8192_cube():
-    """8192^3 block-scaled: E4M3 U[-1,1], scale exponents U{-4..4}, bf16 out."""
+@pytest.mark.parametrize("cfg", ["auto", "mxfp8_1cta_128x256"])
+def test_mxfp8_8192_cube(cfg):
+    """8192^3 block-scaled: E4M3 U[-1,1], scale exponents U{-4..4}, bf16 out
+    (auto = the CTA-pair kernel the benchmark times)."""
     M = N = K = 8192
     a, sfa, b, sfb = synth.mxfp8_operands(M, N, K, workload=8)
-    C = run_mxfp8(a, sfa, b, sfb, M, N, K)
+    C = run_mxfp8(a, sfa, b, sfb, M, N, K, config=cfg)
     got, guard_ok = C.download()
     assert guard_ok and np.isfinite(got).all()
     rows = sample_indices(M, 128, 40, seed=81)
