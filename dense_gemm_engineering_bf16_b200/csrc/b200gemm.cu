@@ -208,7 +208,7 @@ gemm_status_t encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void 
 
 // --------------------------------------------------------------- launches --
 
-gemm_config_t select_config(int64_t M, int64_t N, int64_t /*K*/) {
+gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     const int forced = g_forced.load(std::memory_order_relaxed);
     if (forced != GEMM_CFG_AUTO && forced < GEMM_CFG_MXFP8_1CTA_128x256) return static_cast<gemm_config_t>(forced);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
@@ -217,7 +217,11 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t /*K*/) {
     // tail; a single wave: the static persistent schedule
     if (pair_tiles >= 148) return GEMM_CFG_2CTA_256x256_CLC;
     if (pair_tiles >= 74) return GEMM_CFG_2CTA_256x256;
-    if (M <= 256) return GEMM_CFG_SKINNY;          // too few tiles to fill the SMs: stream-K
+    // few rows, too few tiles to fill the SMs, and a long K to split: stream-K.
+    // (A short K gains nothing from splitting; the plain 128 x 128 kernel has
+    // the lower fixed cost there: 4.8 vs 9.6 us at 128^3 under graph replay.)
+    const int64_t small_tiles = ((M + 127) / 128) * ((N + 127) / 128);
+    if (M <= 256 && K >= 1024 && small_tiles < 148) return GEMM_CFG_SKINNY;
     if (wide_tiles >= 148) return GEMM_CFG_1CTA_128x256;
     return GEMM_CFG_1CTA_128x128;
 }

@@ -103,7 +103,8 @@ def test_status_strings_and_config_control():
     assert G.gemm_select_config(16, 16, 16) == G.CONFIGS["2cta_256x256"]
     G.gemm_force_config("auto")
     assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]
-    assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["skinny"]
+    assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
+    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(1000, 8192, 8192) == G.CONFIGS["2cta_256x256"]
     assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_clc"]
