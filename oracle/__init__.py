@@ -18,6 +18,9 @@ computes:
   sum to the output type.
 * ``gemm_tile_ledger``: the per-K-iteration tile ledger of "GPU 执行模型",
   section "Tile 小账本".
+* ``axpby`` / ``epilogue``: the epilogue variants C = act(alpha A.B + beta C
+  + bias) in fp64, and ``fusion_saving_bytes``, the HBM bytes a fused
+  epilogue saves ("GPU 执行模型", section "Fusion 的收益与上限").
 
 Layouts: A is row-major M x K with leading dimension lda; B is stored K-major,
 i.e. as an N x K array with leading dimension ldb (b(k,j) = B[j, k]); C is
@@ -273,3 +276,57 @@ def gemm_line_sums_f64(a64: np.ndarray, b64_nk: np.ndarray):
     cols = b64 @ a_row
     cols_mag = np.abs(b64) @ a_abs
     return rows, rows_mag, cols, cols_mag
+
+
+# ------------------------------------------------------- epilogue variants --
+
+def axpby(c_ab64: np.ndarray, c_old64: np.ndarray, alpha: float, beta: float) -> np.ndarray:
+    """C <- alpha (A.B) + beta C_old, in fp64, the BLAS-style reading of the
+    epilogue variants (alpha/beta) of a GEMM: the old C is used only when
+    beta != 0, so beta = 0 ignores whatever it holds (NaN included)."""
+    c = float(alpha) * np.asarray(c_ab64, dtype=np.float64)
+    if beta != 0.0:
+        c = c + float(beta) * np.asarray(c_old64, dtype=np.float64)
+    return c
+
+
+ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
+
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    """x Phi(x), Phi the standard normal CDF, written with erf (fp64)."""
+    from math import erf, sqrt
+    x = np.asarray(x, dtype=np.float64)
+    return x * 0.5 * (1.0 + np.vectorize(erf, otypes=[np.float64])(x / sqrt(2.0)))
+
+
+def relu(x: np.ndarray) -> np.ndarray:
+    """0 where x < 0, else x itself (NaN stays NaN)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(x < 0.0, 0.0, x)
+
+
+def epilogue(c_ab64: np.ndarray, c_old64: np.ndarray, alpha: float, beta: float,
+             bias64: np.ndarray | None, act: int) -> np.ndarray:
+    """A fused GEMM epilogue, in fp64: act(alpha (A.B) + beta C_old + bias),
+    the bias one value per column of C.  Its arithmetic is the pointwise
+    sequence that fusion folds into the GEMM's write-back ("GPU 执行模型",
+    section "Fusion 的收益与上限"); which pointwise ops to offer (bias, ReLU,
+    GELU) is this library's choice."""
+    c = axpby(c_ab64, c_old64, alpha, beta)
+    if bias64 is not None:
+        c = c + np.asarray(bias64, dtype=np.float64)[None, :]
+    if act == ACT_RELU:
+        return relu(c)
+    if act == ACT_GELU:
+        return gelu(c)
+    if act != ACT_NONE:
+        raise ValueError(f"unknown activation {act}")
+    return c
+
+
+def fusion_saving_bytes(intermediate_bytes: int) -> int:
+    """HBM bytes saved by fusing a pointwise step into the producer: the
+    intermediate tensor is neither written out nor read back, about
+    2 M_intermediate ("GPU 执行模型", section "Fusion 的收益与上限")."""
+    return 2 * int(intermediate_bytes)

@@ -341,3 +341,45 @@ def test_line_sums_match_full_product():
     rows, rows_mag, cols, cols_mag = oracle.gemm_line_sums_f64(a, b)
     assert np.array_equal(rows, c.sum(axis=1)) and np.array_equal(cols, c.sum(axis=0))
     assert np.array_equal(rows_mag, s.sum(axis=1)) and np.array_equal(cols_mag, s.sum(axis=0))
+
+
+def test_axpby_epilogue_closed_forms():
+    ab = np.array([[1.0, -2.0], [3.5, 0.25]])
+    old = np.array([[10.0, np.nan], [-4.0, 8.0]])
+    assert np.array_equal(oracle.axpby(ab, old, 1.0, 0.0), ab)            # beta = 0: old C ignored, NaN too
+    got = oracle.axpby(ab, np.nan_to_num(old), 2.0, -1.0)
+    assert np.array_equal(got, np.array([[2.0 - 10.0, -4.0], [7.0 + 4.0, 0.5 - 8.0]]))
+    assert np.array_equal(oracle.axpby(np.zeros((2, 2)), np.nan_to_num(old), 3.0, 0.5), 0.5 * np.nan_to_num(old))
+
+
+def test_gelu_relu_closed_forms():
+    # Phi(1) and Phi(-1) from the standard normal table; GELU(x) = x Phi(x)
+    assert oracle.gelu(np.array([1.0]))[0] == pytest.approx(0.8413447460685429, abs=1e-15)
+    assert oracle.gelu(np.array([-1.0]))[0] == pytest.approx(-0.15865525393145707, abs=1e-15)
+    assert oracle.gelu(np.array([0.0]))[0] == 0.0
+    x = np.linspace(-6.0, 6.0, 121)
+    # Phi(x) + Phi(-x) = 1, so GELU(x) - GELU(-x) = x
+    assert np.allclose(oracle.gelu(x) - oracle.gelu(-x), x, atol=1e-15, rtol=0)
+    assert np.allclose(oracle.gelu(np.array([40.0, -40.0])), [40.0, 0.0], atol=1e-300)
+    r = oracle.relu(np.array([-2.0, -0.0, 0.0, 3.5, np.nan]))
+    assert np.array_equal(r[:4], [0.0, 0.0, 0.0, 3.5]) and np.isnan(r[4])
+
+
+def test_epilogue_order_and_bias_broadcast():
+    ab = np.array([[1.0, -2.0, 0.5], [3.0, 0.0, -1.0]])
+    old = np.array([[1.0, 1.0, 1.0], [2.0, 2.0, 2.0]])
+    bias = np.array([0.0, 10.0, -1.0])
+    lin = oracle.epilogue(ab, old, 2.0, -1.0, bias, oracle.ACT_NONE)
+    assert np.array_equal(lin, np.array([[1.0, 5.0, -1.0], [4.0, 8.0, -5.0]]))
+    # the activation comes last: relu after bias, not before
+    assert np.array_equal(oracle.epilogue(ab, old, 2.0, -1.0, bias, oracle.ACT_RELU),
+                          np.array([[1.0, 5.0, 0.0], [4.0, 8.0, 0.0]]))
+    assert np.allclose(oracle.epilogue(ab, old, 2.0, -1.0, bias, oracle.ACT_GELU), oracle.gelu(lin))
+    assert np.array_equal(oracle.epilogue(ab, old, 1.0, 0.0, None, oracle.ACT_NONE), ab)
+    with pytest.raises(ValueError):
+        oracle.epilogue(ab, old, 1.0, 0.0, None, 7)
+
+
+def test_fusion_saving_is_one_write_and_one_read():
+    # an 8192 x 8192 fp32 intermediate: 268 MB out and 268 MB back in
+    assert oracle.fusion_saving_bytes(8192 * 8192 * 4) == 536870912
