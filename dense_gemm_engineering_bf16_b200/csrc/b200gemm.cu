@@ -165,21 +165,26 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int64_t kMaxDim = 0x7FFFFFFF;
 
-// Checks shared by every entry point.  elem sizes in bytes.
+// Checks shared by every entry point.  elem sizes in bytes; a_mn / b_mn:
+// A stored K x M, B stored K x N (else M x K and N x K).
 gemm_status_t check_args(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K,
-                         int64_t lda, int64_t ldb, int64_t ldc, int64_t ea, int64_t eb, int64_t ec) {
+                         int64_t lda, int64_t ldb, int64_t ldc, int64_t ea, int64_t eb, int64_t ec,
+                         bool a_mn = false, bool b_mn = false) {
     if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_VALUE;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return GEMM_ERR_TOO_LARGE;
     if (M == 0 || N == 0) return GEMM_OK;
     if (!C) return GEMM_ERR_INVALID_VALUE;
     if (ldc < N) return GEMM_ERR_INVALID_VALUE;
     if (K > 0) {
+        const int64_t a_rows = a_mn ? K : M, a_cols = a_mn ? M : K;
+        const int64_t b_rows = b_mn ? K : N, b_cols = b_mn ? N : K;
         if (!A || !B) return GEMM_ERR_INVALID_VALUE;
-        if (lda < K || ldb < K) return GEMM_ERR_INVALID_VALUE;
+        if (lda < a_cols || ldb < b_cols) return GEMM_ERR_INVALID_VALUE;
         if (!aligned16(A) || !aligned16(B)) return GEMM_ERR_MISALIGNED;
         if ((lda * ea) % 16 || (ldb * eb) % 16) return GEMM_ERR_MISALIGNED;
         if (lda * ea >= (int64_t(1) << 40) || ldb * eb >= (int64_t(1) << 40)) return GEMM_ERR_TOO_LARGE;
-        if (overlaps(C, M, N, ldc, ec, A, M, K, lda, ea) || overlaps(C, M, N, ldc, ec, B, N, K, ldb, eb))
+        if (overlaps(C, M, N, ldc, ec, A, a_rows, a_cols, lda, ea) ||
+            overlaps(C, M, N, ldc, ec, B, b_rows, b_cols, ldb, eb))
             return GEMM_ERR_ALIAS;
     }
     if (!aligned16(C) || (ldc * ec) % 16) return GEMM_ERR_MISALIGNED;
@@ -229,7 +234,7 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
 template <class Cfg>
 gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, const void *B, void *C,
                           int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, float alpha = 1.0f, float beta = 0.0f, uint32_t layout = 0) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
     cudaError_t e;
@@ -265,8 +270,18 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
     const int64_t ec = Cfg::OUT == 0 ? 4 : 2;
     alignas(64) CUtensorMap tmA, tmB, tmC;
     gemm_status_t s;
-    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK, Cfg::BM_CTA)) != GEMM_OK) return s;
-    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::B_ROWS)) != GEMM_OK) return s;
+    // K-major operands: boxes of 64 (K) x rows; MN-major (stored K x M / K x N):
+    // boxes of 64 (MN) x 64 (K)
+    if (layout & b200::kLayoutAMajorM)
+        s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, M, K, lda * 2, 64, Cfg::BK);
+    else
+        s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK, Cfg::BM_CTA);
+    if (s != GEMM_OK) return s;
+    if (layout & b200::kLayoutBMajorN)
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, K, ldb * 2, 64, Cfg::BK);
+    else
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::B_ROWS);
+    if (s != GEMM_OK) return s;
     // The store map covers the columns that end on a 16-byte granule; the
     // kernel writes the rest of each row ([n_tma, N)) with plain stores.  If
     // no whole granule exists the map is a placeholder the kernel never uses.
@@ -282,7 +297,7 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
                            static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
-                           watchdog_ns(K), inject_flags());
+                           watchdog_ns(K), inject_flags(), alpha, beta, layout);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -335,7 +350,8 @@ gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
 
 template <class Cfg>
 gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const void *B, void *C, int64_t M,
-                            int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream) {
+                            int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
+                            float alpha, float beta, uint32_t layout) {
     auto kernel = b200::gemm_bf16_skinny_sm100_kernel<Cfg>;
     cudaError_t e;
     uint32_t epoch;
@@ -356,8 +372,11 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
     if ((s = sk_workspace(st, static_cast<size_t>(l.partial_bytes + l.counter_bytes), ws)) != GEMM_OK) return s;
     const int64_t mpad = (M + 15) / 16 * 16;
     alignas(64) CUtensorMap tmB, tmA;
-    if ((s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N)) != GEMM_OK)
-        return s;
+    if (layout & b200::kLayoutBMajorN)
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, K, ldb * 2, 64, Cfg::BK);
+    else
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N);
+    if (s != GEMM_OK) return s;
     if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK,
                        static_cast<uint32_t>(mpad))) != GEMM_OK)
         return s;
@@ -365,22 +384,37 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
     unsigned long long *counters = reinterpret_cast<unsigned long long *>(ws + l.partial_bytes);
     kernel<<<static_cast<unsigned>(l.grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
         tmB, tmA, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(mpad), C, ldc,
-        partials, counters, static_cast<int>(l.slots), epoch, st->status, watchdog_ns(K));
+        partials, counters, static_cast<int>(l.slots), epoch, st->status, watchdog_ns(K), alpha, beta, layout);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
 
 gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const void *B, void *C, int64_t M,
-                                int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream) {
-    if (M > 256) return GEMM_ERR_INVALID_VALUE;
+                                int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
+                                float alpha = 1.0f, float beta = 0.0f, uint32_t layout = 0) {
+    // the skinny kernel reads A K-major only (A stored M x K)
+    if (M > 256 || (layout & b200::kLayoutAMajorM)) return GEMM_ERR_INVALID_VALUE;
     if (M <= 64)
-        return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                   : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                   : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
     if (M <= 128)
-        return f32 ? launch_skinny<CfgSk128F32>(st, 2, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                   : launch_skinny<CfgSk128B16>(st, 3, A, B, C, M, N, K, lda, ldb, ldc, stream);
-    return f32 ? launch_skinny<CfgSk256F32>(st, 4, A, B, C, M, N, K, lda, ldb, ldc, stream)
-               : launch_skinny<CfgSk256B16>(st, 5, A, B, C, M, N, K, lda, ldb, ldc, stream);
+        return f32 ? launch_skinny<CfgSk128F32>(st, 2, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                   : launch_skinny<CfgSk128B16>(st, 3, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
+    return f32 ? launch_skinny<CfgSk256F32>(st, 4, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+               : launch_skinny<CfgSk256B16>(st, 5, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
+}
+
+// C = beta * C (K == 0 with beta != 0): the empty sum plus the beta term.
+template <typename T>
+gemm_status_t launch_scale(void *C, int64_t M, int64_t N, int64_t ldc, float beta, int sm_count,
+                           cudaStream_t stream) {
+    const int64_t total = M * N;
+    int64_t blocks = (total + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    b200::scale_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<T *>(C), M, N, ldc, beta);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
 }
 
 template <typename T>
@@ -564,42 +598,59 @@ gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const u
 
 extern "C" {
 
-gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
-                        int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, cudaStream_t stream) {
+gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                           int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, gemm_layout_t a_layout,
+                           gemm_layout_t b_layout, float alpha, float beta, cudaStream_t stream) {
     if (c_type != GEMM_OUT_F32 && c_type != GEMM_OUT_BF16) return GEMM_ERR_INVALID_VALUE;
+    if ((a_layout != GEMM_LAYOUT_KMAJOR && a_layout != GEMM_LAYOUT_MNMAJOR) ||
+        (b_layout != GEMM_LAYOUT_KMAJOR && b_layout != GEMM_LAYOUT_MNMAJOR))
+        return GEMM_ERR_INVALID_VALUE;
+    const bool a_mn = a_layout == GEMM_LAYOUT_MNMAJOR, b_mn = b_layout == GEMM_LAYOUT_MNMAJOR;
     const int64_t ec = c_type == GEMM_OUT_F32 ? 4 : 2;
-    gemm_status_t s = check_args(A, B, C, M, N, K, lda, ldb, ldc, 2, 2, ec);
+    gemm_status_t s = check_args(A, B, C, M, N, K, lda, ldb, ldc, 2, 2, ec, a_mn, b_mn);
     if (s != GEMM_OK || M == 0 || N == 0) return s;
     int dev;
     DeviceState *st;
     if ((s = current_device(dev, st)) != GEMM_OK) return s;
-    if (K == 0) {
-        return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
-                                      : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
-    }
-    const gemm_config_t cfg = select_config(M, N, K);
     const bool f32 = c_type == GEMM_OUT_F32;
+    if (K == 0) {
+        // the empty sum: C = beta * C (zeros when beta == 0, C not read)
+        if (beta == 0.0f)
+            return f32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
+                       : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
+        return f32 ? launch_scale<float>(C, M, N, ldc, beta, st->sm_count, stream)
+                   : launch_scale<__nv_bfloat16>(C, M, N, ldc, beta, st->sm_count, stream);
+    }
+    const uint32_t layout = (a_mn ? b200::kLayoutAMajorM : 0u) | (b_mn ? b200::kLayoutBMajorN : 0u);
+    gemm_config_t cfg = select_config(M, N, K);
+    if (cfg == GEMM_CFG_SKINNY && a_mn) cfg = GEMM_CFG_1CTA_128x128;   // skinny reads A K-major only
     switch (cfg) {
         case GEMM_CFG_1CTA_128x256:
-            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
         case GEMM_CFG_1CTA_128x128:
-            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
         case GEMM_CFG_2CTA_256x256:
-            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
         case GEMM_CFG_SKINNY:
-            return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream);
+            return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
         case GEMM_CFG_2CTA_256x256_CLC:
-            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
         case GEMM_CFG_1CTA_128x256_CLC:
-            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
+            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
+                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
         default:
             return GEMM_ERR_INVALID_VALUE;
     }
+}
+
+gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                        int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, cudaStream_t stream) {
+    return gemm_bf16_ex(A, B, C, M, N, K, lda, ldb, ldc, c_type, GEMM_LAYOUT_KMAJOR, GEMM_LAYOUT_KMAJOR, 1.0f, 0.0f,
+                        stream);
 }
 
 gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const uint8_t *sfb, void *C,

@@ -83,12 +83,16 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         : "r"(taddr));
 }
 
+// C[m][n] = alpha * v + beta * C[m][n]  (C read only when beta != 0).
 template <int OUT>
-__device__ __forceinline__ void store_c(void *C, int64_t ldc, int m, int n, float v) {
+__device__ __forceinline__ void store_c(void *C, int64_t ldc, int m, int n, float v, float alpha, float beta) {
+    const int64_t i = static_cast<int64_t>(m) * ldc + n;
     if constexpr (OUT == 0) {
-        static_cast<float *>(C)[static_cast<int64_t>(m) * ldc + n] = v;
+        float *c = static_cast<float *>(C);
+        c[i] = beta != 0.0f ? fmaf(alpha, v, beta * c[i]) : alpha * v;
     } else {
-        static_cast<__nv_bfloat16 *>(C)[static_cast<int64_t>(m) * ldc + n] = __float2bfloat16_rn(v);
+        __nv_bfloat16 *c = static_cast<__nv_bfloat16 *>(C);
+        c[i] = __float2bfloat16_rn(beta != 0.0f ? fmaf(alpha, v, beta * __bfloat162float(c[i])) : alpha * v);
     }
 }
 
@@ -102,7 +106,7 @@ template <int OUT>
 __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_elems, int slots_per_cta,
                                            int64_t c_lo, int64_t c_hi, int64_t t, int64_t total, int64_t g,
                                            int64_t kb_per_tile, int M, int N, void *C, int64_t ldc,
-                                           uint32_t epi_tid) {
+                                           uint32_t epi_tid, float alpha, float beta) {
     constexpr int ROWS = 8;                      // rows per round for this thread
     const int n4 = static_cast<int>(epi_tid & 31u) * 4;
     const int msub = static_cast<int>(epi_tid >> 5);
@@ -142,7 +146,25 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
         for (int r = 0; r < ROWS; ++r) {
             const int m = m0 + 4 * r;
             if (m >= M || n >= N) continue;
-            const float vals[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
+            float vals[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
+            if (n + 4 <= N && (alpha != 1.0f || beta != 0.0f)) {
+                float old[4] = {0.f, 0.f, 0.f, 0.f};
+                if (beta != 0.0f) {
+                    if constexpr (OUT == 0) {
+                        const float4 x = *reinterpret_cast<const float4 *>(static_cast<const float *>(C) +
+                                                                           static_cast<int64_t>(m) * ldc + n);
+                        old[0] = x.x; old[1] = x.y; old[2] = x.z; old[3] = x.w;
+                    } else {
+                        const uint2 x = *reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(C) +
+                                                                         static_cast<int64_t>(m) * ldc + n);
+                        old[0] = __uint_as_float(x.x << 16); old[1] = __uint_as_float(x.x & 0xFFFF0000u);
+                        old[2] = __uint_as_float(x.y << 16); old[3] = __uint_as_float(x.y & 0xFFFF0000u);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vals[q] = beta != 0.0f ? fmaf(alpha, vals[q], beta * old[q]) : alpha * vals[q];
+                acc[r] = make_float4(vals[0], vals[1], vals[2], vals[3]);
+            }
             if (n + 4 <= N) {
                 if constexpr (OUT == 0) {
                     *reinterpret_cast<float4 *>(static_cast<float *>(C) + static_cast<int64_t>(m) * ldc + n) = acc[r];
@@ -155,7 +177,7 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
             } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    if (n + q < N) store_c<OUT>(C, ldc, m, n + q, vals[q]);
+                    if (n + q < N) store_c<OUT>(C, ldc, m, n + q, vals[q], alpha, beta);
             }
         }
     }
@@ -167,7 +189,10 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                               const __grid_constant__ CUtensorMap tmA,   // A as M x K, box 64 x mpad
                               int M, int N, int K, int mpad, void *C, int64_t ldc,
                               float *partials, unsigned long long *counters, int slots_per_cta,
-                              uint32_t epoch, DeviceStatus *status, uint64_t timeout_ns) {
+                              uint32_t epoch, DeviceStatus *status, uint64_t timeout_ns,
+                              float alpha, float beta, uint32_t layout) {
+    // B stored K x N arrives as MN-major tiles; A must be stored M x K here.
+    const bool b_mn = (layout & kLayoutBMajorN) != 0;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -238,7 +263,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 const uint32_t b_dst = base + stage * Cfg::STAGE_BYTES;
                 const uint32_t a_dst = b_dst + Cfg::B_BYTES;
                 mbar_arrive_expect_tx(full_bar(stage), tx);
-                tma_load_2d(b_dst, &tmB, full_bar(stage), kb * Cfg::BK, t * Cfg::TILE_N);
+                load_operand_tile<1>(b_dst, &tmB, full_bar(stage), kb * Cfg::BK, t * Cfg::TILE_N, Cfg::TILE_N, b_mn);
                 tma_load_2d(a_dst, &tmA, full_bar(stage), kb * Cfg::BK, 0);
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
             }
@@ -254,7 +279,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(Cfg::TILE_N, mpad);
+            const uint32_t idesc = idesc_bf16_f32(Cfg::TILE_N, mpad, b_mn ? 1u : 0u, 0u);
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             int seg = 0;
@@ -281,7 +306,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                     const uint32_t a0 = b0 + Cfg::B_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
-                        mma_bf16_ss<1>(d_tmem, sw128_kmajor_desc(b0 + kk * 32), sw128_kmajor_desc(a0 + kk * 32),
+                        mma_bf16_ss<1>(d_tmem, operand_desc(b0, kk, b_mn), sw128_kmajor_desc(a0 + kk * 32),
                                        idesc, (j != it || kk != 0) ? 1u : 0u);
                     }
                     mma_commit<1>(empty_bar(stage), 0);
@@ -335,7 +360,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                     if (m < M) {
                         const float x = __uint_as_float(v[i]);
                         if (shared_tile) my_partial[static_cast<int64_t>(m) * Cfg::TILE_N + n_local] = x;
-                        else if (n < N) store_c<Cfg::OUT>(C, ldc, m, n, x);
+                        else if (n < N) store_c<Cfg::OUT>(C, ldc, m, n, x, alpha, beta);
                     }
                 }
             }
@@ -367,7 +392,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 if (*last_flag) {
                     __threadfence();
                     fixup_tile<Cfg::OUT>(partials, slot_elems, slots_per_cta, c_lo, c_hi, t, total, g,
-                                         kb_per_tile, M, N, C, ldc, epi_tid);
+                                         kb_per_tile, M, N, C, ldc, epi_tid, alpha, beta);
                     // every contributor has arrived: leave the counter at zero
                     // arrivals so a replay of this launch (same epoch, e.g.
                     // from a CUDA graph) starts from a clean count

@@ -29,12 +29,19 @@
 //               of idling) and hands the tile id to every role of both CTAs
 //               through a 2-deep shared-memory ring.
 //
+// Operands may be K-major (A as M x K, B as N x K) or MN-major (A as K x M,
+// B as K x N): MN-major tiles arrive as 64-wide boxes and the MMA reads them
+// through MN-major descriptors.  The epilogue computes alpha * A.B + beta * C
+// (C read only when beta != 0).
+//
 // Tails: TMA loads zero-fill outside [0,K) x [0,M) / [0,N) element by
 // element.  TMA stores clip rows exactly but write whole 16-byte granules
 // along a row, so C's tensor map covers only the columns [0, n_tma) that end
 // on a granule boundary; the last < 16 bytes of each row ([n_tma, N)) are
 // written with plain predicated stores.  Every mbarrier wait is bounded.
 #pragma once
+#include <cuda_bf16.h>
+
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -134,14 +141,97 @@ __device__ __forceinline__ void record_timeout(DeviceStatus *status, volatile ui
     if (cg == 2) store_cluster_u32(map_to_cta(abort_smem, cluster_cta_rank() ^ 1u), 1u);
 }
 
+// Operand layouts in global memory (kernel `layout` word).
+constexpr uint32_t kLayoutAMajorM = 1u;   // A stored K x M: a(i,k) at A[k*lda + i]
+constexpr uint32_t kLayoutBMajorN = 2u;   // B stored K x N: b(k,j) at B[k*ldb + j]
+
+// One k-tile of an operand into shared memory.  K-major: one box of 64 (K)
+// x rows.  MN-major: rows / 64 boxes of 64 (MN) x 64 (K), 8 KB apart (the
+// layout sw128_mnmajor_desc describes).  Completion counts on `bar`.
+template <int CG>
+__device__ __forceinline__ void load_operand_tile(uint32_t dst, const CUtensorMap *map, uint32_t bar, int kx,
+                                                  int row, int rows, bool mn) {
+    if (!mn) {
+        if constexpr (CG == 1) tma_load_2d(dst, map, bar, kx, row);
+        else tma_load_2d_pair(dst, map, bar, kx, row);
+        return;
+    }
+    for (int h = 0; h < rows / 64; ++h) {
+        if constexpr (CG == 1) tma_load_2d(dst + 8192u * h, map, bar, row + 64 * h, kx);
+        else tma_load_2d_pair(dst + 8192u * h, map, bar, row + 64 * h, kx);
+    }
+}
+
+// Descriptor of K step kk (16 elements) of an operand tile at `base`.
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk, bool mn) {
+    return mn ? sw128_mnmajor_desc(base + 2048u * kk) : sw128_kmajor_desc(base + 32u * kk);
+}
+
+// v[j] <- alpha * v[j] + beta * C[row][col0 + j] for 32 fp32 values held as
+// bits (C fp32); C is read only when beta != 0 and only inside M x N.
+__device__ __forceinline__ void axpby_f32(uint32_t (&v)[32], const void *C, int64_t ldc, int row, int col0,
+                                          int M, int N, float alpha, float beta) {
+    const float *crow = static_cast<const float *>(C) + static_cast<int64_t>(row) * ldc;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float old[4] = {0.f, 0.f, 0.f, 0.f};
+        const int col = col0 + 4 * q;
+        if (beta != 0.0f && row < M) {
+            if (col + 4 <= N) {
+                const float4 x = *reinterpret_cast<const float4 *>(crow + col);
+                old[0] = x.x; old[1] = x.y; old[2] = x.z; old[3] = x.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (col + e < N) old[e] = crow[col + e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float acc = __uint_as_float(v[4 * q + e]);
+            v[4 * q + e] = __float_as_uint(beta != 0.0f ? fmaf(alpha, acc, beta * old[e]) : alpha * acc);
+        }
+    }
+}
+
+// The same for 32 fp32 accumulator values whose C elements are bf16.
+__device__ __forceinline__ void axpby_bf16src(uint32_t (&v)[32], const void *C, int64_t ldc, int row, int col0,
+                                              int M, int N, float alpha, float beta) {
+    const uint16_t *crow = static_cast<const uint16_t *>(C) + static_cast<int64_t>(row) * ldc;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        const int col = col0 + 8 * q;
+        if (beta != 0.0f && row < M) {
+            if (col + 8 <= N) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(crow + col);
+                w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (col + e < N) w[e >> 1] |= static_cast<uint32_t>(crow[col + e]) << (16 * (e & 1));
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float old = __uint_as_float((w[e >> 1] >> (16 * (e & 1))) << 16);   // bf16 -> f32
+            const float acc = __uint_as_float(v[8 * q + e]);
+            v[8 * q + e] = __float_as_uint(beta != 0.0f ? fmaf(alpha, acc, beta * old) : alpha * acc);
+        }
+    }
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC,
                        int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m,
-                       DeviceStatus *status, uint64_t timeout_ns, uint32_t inject) {
+                       DeviceStatus *status, uint64_t timeout_ns, uint32_t inject,
+                       float alpha, float beta, uint32_t layout) {
     constexpr int CG = Cfg::CG;
+    const bool a_mn = (layout & kLayoutAMajorM) != 0;   // A stored K x M
+    const bool b_mn = (layout & kLayoutBMajorN) != 0;   // B stored K x N
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-memory window offset (swizzle atoms).
     const uint32_t raw = smem_addr(smem_raw);
@@ -260,16 +350,16 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                         continue;
                     }
+                    uint32_t bar;
                     if constexpr (CG == 1) {
-                        mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
-                        tma_load_2d(a_dst, &tmA, full_bar(stage), kx, a_row);
-                        tma_load_2d(b_dst, &tmB, full_bar(stage), kx, b_row);
+                        bar = full_bar(stage);
+                        mbar_arrive_expect_tx(bar, Cfg::TX_BYTES);
                     } else {
                         if (rank == leader_rank) mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
-                        const uint32_t bar = map_to_cta(full_bar(stage), leader_rank);
-                        tma_load_2d_pair(a_dst, &tmA, bar, kx, a_row);
-                        tma_load_2d_pair(b_dst, &tmB, bar, kx, b_row);
+                        bar = map_to_cta(full_bar(stage), leader_rank);
                     }
+                    load_operand_tile<CG>(a_dst, &tmA, bar, kx, a_row, Cfg::BM_CTA, a_mn);
+                    load_operand_tile<CG>(b_dst, &tmB, bar, kx, b_row, Cfg::B_ROWS, b_mn);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -290,7 +380,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
         if (rank == 0 && lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN);
+            const uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN, a_mn ? 1u : 0u, b_mn ? 1u : 0u);
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             int t = 0;
@@ -315,8 +405,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t b0 = a0 + Cfg::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
-                        mma_bf16_ss<CG>(d_tmem, sw128_kmajor_desc(a0 + kk * 32),
-                                        sw128_kmajor_desc(b0 + kk * 32), idesc,
+                        mma_bf16_ss<CG>(d_tmem, operand_desc(a0, kk, a_mn), operand_desc(b0, kk, b_mn), idesc,
                                         (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit<CG>(empty_bar(stage), 0x3);
@@ -364,6 +453,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         // ----------------------------------------------------- epilogue --
         const uint32_t sub = warp & 3u;            // TMEM lanes [32*sub, 32*sub + 32)
         const uint32_t ew = warp - 2u;             // staging slot
+        const bool scaled = !(alpha == 1.0f && beta == 0.0f);
         const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
         uint32_t nstore = 0;
         int t = 0;
@@ -388,14 +478,20 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll 1
             for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
                 uint32_t packed[32];
+                const int erow = row0 + static_cast<int>(lane);   // this thread's row of C
                 if constexpr (Cfg::OUT == 0) {
                     tmem_ld_32x32b_x32(tbase + c * 32, packed);
                     tmem_ld_wait();
+                    if (scaled) axpby_f32(packed, C, ldc, erow, col0 + c * 32, M, N, alpha, beta);
                 } else {
                     uint32_t v0[32], v1[32];
                     tmem_ld_32x32b_x32(tbase + c * 64, v0);
                     tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
                     tmem_ld_wait();
+                    if (scaled) {
+                        axpby_bf16src(v0, C, ldc, erow, col0 + c * 64, M, N, alpha, beta);
+                        axpby_bf16src(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, alpha, beta);
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
@@ -494,6 +590,18 @@ __global__ void zero_fill_kernel(T *C, int64_t M, int64_t N, int64_t ldc) {
         const int64_t r = i / N;
         const int64_t c = i - r * N;
         C[r * ldc + c] = T(0);
+    }
+}
+
+// C = beta * C, one element per thread, grid-stride (K == 0 with beta != 0).
+template <typename T>
+__global__ void scale_kernel(T *C, int64_t M, int64_t N, int64_t ldc, float beta) {
+    const int64_t total = M * N;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / N;
+        const int64_t c = i - r * N;
+        C[r * ldc + c] = static_cast<T>(beta * static_cast<float>(C[r * ldc + c]));
     }
 }
 

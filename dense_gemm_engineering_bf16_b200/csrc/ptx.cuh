@@ -341,11 +341,30 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem) {
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by
+// TMA with the 128-byte swizzle in boxes of 64 (MN) x 64 (K) bf16: each box
+// is 64 K-rows of 128 bytes (64 MN elements), boxes for successive 64-wide
+// MN groups 8 KB apart.  Fields: start >> 4, leading byte offset = distance
+// between 64-element MN groups (8192 B), stride byte offset = distance
+// between 8-row K groups (1024 B), version 1, 128-byte swizzle.  A K step
+// of 16 moves the start address by 16 rows = 2048 bytes.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(8192 >> 4) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B, f32 accumulator,
-// both operands K-major, dense: D format (bits 4-5) = 1 (f32), A format
-// (7-9) = 1 (bf16), B format (10-12) = 1 (bf16), N >> 3 (17-22), M >> 4 (24-28).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) |
+// dense: D format (bits 4-5) = 1 (f32), A format (7-9) = 1 (bf16), B format
+// (10-12) = 1 (bf16), A / B MN-major (15 / 16), N >> 3 (17-22), M >> 4 (24-28).
+// a_mn / b_mn set the "transpose" (MN-major) bits 15 / 16 for an operand
+// stored MN-major in shared memory.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, uint32_t a_mn = 0, uint32_t b_mn = 0) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) |
            (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 

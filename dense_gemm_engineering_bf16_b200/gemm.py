@@ -22,6 +22,8 @@ lib = ctypes.CDLL(library_path)
 
 OUT_F32 = 0
 OUT_BF16 = 1
+KMAJOR = 0      # A as M x K, B as N x K
+MNMAJOR = 1     # A as K x M, B as K x N (row-major K x N)
 
 CONFIGS = {
     "auto": 0,
@@ -49,6 +51,9 @@ lib.gemm_bf16.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _in
 lib.gemm_bf16.restype = _int
 lib.gemm_bf16_noalloc.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp]
 lib.gemm_bf16_noalloc.restype = _int
+lib.gemm_bf16_ex.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int,
+                             ctypes.c_float, ctypes.c_float, _vp]
+lib.gemm_bf16_ex.restype = _int
 lib.gemm_mxfp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]
 lib.gemm_mxfp8.restype = _int
 lib.gemm_check_device_status.argtypes = [_vp]
@@ -112,6 +117,16 @@ def gemm_bf16(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
     """
     st = lib.gemm_bf16(_ptr(A), _ptr(B), _ptr(C), M, N, K, lda, ldb, ldc, int(c_type), _stream(stream))
     return _check(st, "gemm_bf16", check)
+
+
+def gemm_bf16_ex(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
+                 c_type: int = OUT_F32, a_layout: int = KMAJOR, b_layout: int = KMAJOR,
+                 alpha: float = 1.0, beta: float = 0.0, stream=None, check: bool = True) -> int:
+    """C = alpha * A.B + beta * C with K-major or MN-major operands
+    (see include/b200gemm.h, gemm_bf16_ex)."""
+    st = lib.gemm_bf16_ex(_ptr(A), _ptr(B), _ptr(C), M, N, K, lda, ldb, ldc, int(c_type), int(a_layout),
+                          int(b_layout), float(alpha), float(beta), _stream(stream))
+    return _check(st, "gemm_bf16_ex", check)
 
 
 def gemm_mxfp8(A, sfa, B, sfb, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,

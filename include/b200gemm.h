@@ -68,6 +68,16 @@ typedef enum {
     GEMM_OUT_BF16 = 1               /* C is bfloat16, rounded to nearest even */
 } gemm_out_t;
 
+/* How an operand is stored (gemm_bf16_ex).  K-major is the layout of
+ * gemm_bf16: A as M rows of K (a(i,k) at A[i*lda + k]), B as N rows of K
+ * (b(k,j) at B[j*ldb + k]).  MN-major stores the other way round: A as K rows
+ * of M (a(i,k) at A[k*lda + i]), B as K rows of N (b(k,j) at B[k*ldb + j],
+ * the row-major K x N matrix of C = A.B as most frameworks hold it). */
+typedef enum {
+    GEMM_LAYOUT_KMAJOR = 0,
+    GEMM_LAYOUT_MNMAJOR = 1
+} gemm_layout_t;
+
 /* Kernel configurations.  GEMM_CFG_AUTO picks by shape; the others force a
  * configuration (for tests and benchmarks) through gemm_force_config(). */
 typedef enum {
@@ -104,6 +114,26 @@ B200GEMM_API gemm_status_t gemm_bf16(const void *A, const void *B, void *C,
                         int64_t M, int64_t N, int64_t K,
                         int64_t lda, int64_t ldb, int64_t ldc,
                         gemm_out_t c_type, cudaStream_t stream);
+
+/*
+ * gemm_bf16_ex: C = alpha * A . B + beta * C, with each operand stored
+ * K-major or MN-major (gemm_layout_t).  bf16 A and B, fp32 accumulation,
+ * C as c_type; alpha and beta are applied in fp32 to the fp32 accumulator
+ * and the (widened) old C before the single rounding to c_type.  C is read
+ * only when beta != 0 (beta == 0: C's old contents, NaN included, are
+ * ignored).  K == 0 gives C = beta * C.  These are the epilogue and operand
+ * variants of a GEMM's correctness contract ("GPU 执行模型", section
+ * "正确性契约": layout, stride, which buffers are read and written).
+ *   a_layout K-major: lda >= K; MN-major: lda >= M.
+ *   b_layout K-major: ldb >= K; MN-major: ldb >= N.
+ * Other rules as gemm_bf16, which is gemm_bf16_ex with both operands
+ * K-major, alpha = 1, beta = 0.
+ */
+B200GEMM_API gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C,
+                                        int64_t M, int64_t N, int64_t K,
+                                        int64_t lda, int64_t ldb, int64_t ldc,
+                                        gemm_out_t c_type, gemm_layout_t a_layout, gemm_layout_t b_layout,
+                                        float alpha, float beta, cudaStream_t stream);
 
 /*
  * gemm_mxfp8: block-scaled C = (sa . A) . (sb . B) with FP8 E4M3 A and B and

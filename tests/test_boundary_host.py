@@ -67,6 +67,28 @@ def test_rejects_bad_arguments_before_any_launch():
     assert _call(C_=B) == 3                         # C overlaps B
 
 
+def _call_ex(A_=A, B_=B, C_=C, M=128, N=96, K=64, lda=None, ldb=None, ldc=None, ct=G.OUT_F32,
+             al=G.KMAJOR, bl=G.KMAJOR, alpha=1.0, beta=0.0):
+    lda = (M if al == G.MNMAJOR else K) if lda is None else lda
+    ldb = (N if bl == G.MNMAJOR else K) if ldb is None else ldb
+    ldc = N if ldc is None else ldc
+    return G.lib.gemm_bf16_ex(A_, B_, C_, M, N, K, lda, ldb, ldc, ct, al, bl, alpha, beta, 0)
+
+
+def test_ex_rejects_bad_layouts_and_pitches_before_any_launch():
+    assert _call_ex(al=2) == 1 and _call_ex(bl=-1) == 1 and _call_ex(ct=3) == 1
+    # A stored K x M: the pitch covers M, not K
+    assert _call_ex(al=G.MNMAJOR, lda=64) == 1              # lda < M = 128
+    assert _call_ex(al=G.MNMAJOR, M=100, lda=100) == 2       # 200-byte pitch
+    assert _call_ex(bl=G.MNMAJOR, ldb=64) == 1               # ldb < N = 96
+    assert _call_ex(bl=G.MNMAJOR, N=90, ldb=90, ldc=92) == 2  # 180-byte pitch
+    # a K x M A of 64 rows with pitch 128 spans 16 KiB; C placed inside it aliases
+    assert _call_ex(al=G.MNMAJOR, C_=A + 8192) == 3
+    # K = 0 reads no operand: null A and B are fine, and C alone is validated
+    assert _call_ex(K=0, A_=0, B_=0, C_=0) == 1
+    assert _call_ex(K=0, A_=0, B_=0, C_=C + 4) == 2
+
+
 def test_mxfp8_rejects_bad_arguments_before_any_launch():
     f = G.lib.gemm_mxfp8
     sa, sb = 0x7F0000300000, 0x7F0000400000
