@@ -1,7 +1,7 @@
 """Benchmark: bf16 GEMM TFLOP/s at 8192^3 on B200 (C = A.B, bf16 in, fp32 accumulate and out).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload square8192|square4096|ragged|skinny1000|skinny16|mxfp8_8192]
+                    [--workload square8192|square4096|ragged|skinny1000|skinny16|mxfp8_8192|fused8192]
                     [--shape M N K] [--config auto|1cta_128x128|1cta_128x256|2cta_256x256]
 
 One step = one library call over the whole M x N x K problem with the inputs
@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "bf16 GEMM TFLOP/s at 8192³ on 1 B200 (fraction of dense BF16 tensor peak)"
 METRIC_MXFP8 = "MXFP8 block-scaled GEMM TFLOP/s at 8192³ on 1 B200"
+METRIC_FUSED = "bf16 GEMM + bias + GELU (fused epilogue, bf16 out) TFLOP/s at 8192³ on 1 B200"
 UNIT = "TFLOP/s"
 
 # name: (M, N, K, kind, distribution, workload id, description)
@@ -47,6 +48,8 @@ WORKLOADS = {
     "skinny16": (16, 8192, 8192, "bf16", "normal", 6, "gemm 16x8192x8192, bf16 N(0,1) in, fp32 out"),
     "mxfp8_8192": (8192, 8192, 8192, "mxfp8", "uniform", 8,
                    "block-scaled gemm 8192^3, E4M3 U[-1,1], E8M0 per 32 (exp U{-4..4}), bf16 out"),
+    "fused8192": (8192, 8192, 8192, "fused", "uniform", 3,
+                  "gelu(A.B + bias) 8192^3, bf16 U[-1,1] in, bias N(0,1) fp32, fp32 accumulate, bf16 out"),
 }
 
 L2_BYTES = 126 * 1024 * 1024
@@ -57,9 +60,9 @@ FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # The device sources each kernel is compiled from; an ncu traffic figure is
 # valid only while these files are unchanged.
 KERNEL_SOURCES = {
-    "bf16": ["ptx.cuh", "gemm_bf16_sm100.cuh"],
-    "skinny": ["ptx.cuh", "gemm_bf16_sm100.cuh", "gemm_bf16_skinny_sm100.cuh"],
-    "mxfp8": ["ptx.cuh", "gemm_bf16_sm100.cuh", "gemm_mxfp8_sm100.cuh"],
+    "bf16": ["ptx.cuh", "epilogue.cuh", "gemm_bf16_sm100.cuh"],
+    "skinny": ["ptx.cuh", "epilogue.cuh", "gemm_bf16_sm100.cuh", "gemm_bf16_skinny_sm100.cuh"],
+    "mxfp8": ["ptx.cuh", "epilogue.cuh", "gemm_bf16_sm100.cuh", "gemm_mxfp8_sm100.cuh"],
 }
 
 
@@ -195,8 +198,9 @@ class Problem:
         if shape:
             M, N, K = shape
             dist, wid = "uniform", 90
-            desc = (f"gemm {M}x{N}x{K}, bf16 U[-1,1] in, fp32 out" if kind == "bf16" else
-                    f"block-scaled gemm {M}x{N}x{K}, E4M3 U[-1,1], E8M0 per 32, bf16 out")
+            desc = {"bf16": f"gemm {M}x{N}x{K}, bf16 U[-1,1] in, fp32 out",
+                    "fused": f"gelu(A.B + bias) {M}x{N}x{K}, bf16 U[-1,1] in, bf16 out",
+                    "mxfp8": f"block-scaled gemm {M}x{N}x{K}, E4M3 U[-1,1], E8M0 per 32, bf16 out"}[kind]
         self.name, self.M, self.N, self.K, self.kind, self.desc = name, M, N, K, kind, desc
         self.flops = 2.0 * M * N * K
         if kind == "bf16":
@@ -204,6 +208,12 @@ class Problem:
             self.host = [self.a, self.b]
             self.in_bytes = 2 * (M * K + N * K)
             self.out_bytes = 4 * M * N
+        elif kind == "fused":
+            self.a, self.b = synth.bf16_operands(M, N, K, dist, workload=wid, base=rank)
+            self.bias = synth.normal(synth.derive_seed(wid, 4, rank), (N,)).astype(np.float32)
+            self.host = [self.a, self.b, self.bias]
+            self.in_bytes = 2 * (M * K + N * K) + 4 * N
+            self.out_bytes = 2 * M * N
         else:
             self.a, self.sfa, self.b, self.sfb = synth.mxfp8_operands(M, N, K, workload=wid, base=rank)
             self.host = [self.a, self.sfa, self.b, self.sfb]
@@ -213,6 +223,9 @@ class Problem:
     def device_arrays(self, torch):
         if self.kind == "bf16":
             return [torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) for x in self.host]
+        if self.kind == "fused":
+            return [torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) for x in self.host[:2]] + \
+                [torch.from_numpy(self.bias).cuda()]
         return [torch.from_numpy(np.ascontiguousarray(x)).cuda() for x in self.host]
 
     def empty_out(self, torch, pinned=False):
@@ -226,6 +239,10 @@ class Problem:
         if self.kind == "bf16":
             A, B = dev
             G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_F32, stream=stream)
+        elif self.kind == "fused":
+            A, B, bias = dev
+            G.gemm_bf16_fused(A, B, C, M, N, K, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias,
+                              G.ACT_GELU, stream=stream)
         else:
             A, SA, B, SB = dev
             G.gemm_mxfp8(A, SA, B, SB, C, M, N, K, K, K, N, stream=stream)
@@ -237,7 +254,58 @@ class Problem:
         import oracle
         if self.kind == "bf16":
             return oracle.gemm_bf16_f64(self.a[:rows], self.b, K=self.K)
+        if self.kind == "fused":
+            c = oracle.gemm_bf16_f64(self.a[:rows], self.b, K=self.K)
+            return oracle.epilogue(c, None, 1.0, 0.0, self.bias.astype(np.float64), oracle.ACT_GELU)
         return oracle.gemm_mxfp8_f64(self.a[:rows], self.sfa[:rows], self.b, self.sfb, K=self.K)
+
+
+def fusion_comparison(p, G, dev, torch, stream, steps):
+    """The unfused form of the fused workload, timed beside it: a plain GEMM
+    writing the bf16 intermediate, then a separate pass C = gelu(C + bias)
+    that reads it back and writes it again.  Fusion saves that pass's two
+    intermediate-sized transfers ("GPU 执行模型", section "Fusion 的收益与
+    上限": about 2 x the intermediate's bytes).  The fused call, the plain
+    GEMM and the pass are interleaved step by step, so all three see the
+    same clocks; medians are reported."""
+    A, B, bias = dev
+    M, N, K = p.M, p.N, p.K
+    C1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    C2 = torch.empty_like(C1)
+
+    def fused():
+        G.gemm_bf16_fused(A, B, C1, M, N, K, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias,
+                          G.ACT_GELU, stream=stream)
+
+    def gemm():
+        G.gemm_bf16(A, B, C2, M, N, K, K, K, N, G.OUT_BF16, stream=stream)
+
+    def pointwise():
+        G.gemm_bf16_fused(A, B, C2, M, N, 0, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 1.0, bias,
+                          G.ACT_GELU, stream=stream)
+
+    for _ in range(3):
+        fused(), gemm(), pointwise()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for e in ev:
+        e[0].record(stream)
+        fused()
+        e[1].record(stream)
+        gemm()
+        e[2].record(stream)
+        pointwise()
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    G.gemm_check_device_status(stream)
+    med = lambda i: statistics.median(e[i].elapsed_time(e[i + 1]) for e in ev)  # noqa: E731
+    fused_ms, gemm_ms, pass_ms = med(0), med(1), med(2)
+    inter = 2 * M * N                       # the bf16 intermediate, bytes
+    return {"fused_ms": fused_ms, "unfused_gemm_ms": gemm_ms, "unfused_pass_ms": pass_ms,
+            "unfused_ms": gemm_ms + pass_ms, "saved_ms": gemm_ms + pass_ms - fused_ms,
+            "fused_over_plain_gemm_ms": fused_ms - gemm_ms,
+            "ledger_saved_bytes": 2 * inter,
+            "unfused_pass_gbs": (2 * inter + 4 * N) / (pass_ms * 1e-3) / 1e9, "steps": steps}
 
 
 def oracle_sample(problem: Problem, budget_s: float):
@@ -259,6 +327,10 @@ def oracle_sample(problem: Problem, budget_s: float):
     return 2.0 * R * problem.N * problem.K, dt, R
 
 
+def metric_of(kind: str) -> str:
+    return {"bf16": METRIC, "mxfp8": METRIC_MXFP8, "fused": METRIC_FUSED}[kind]
+
+
 def run_reference(args, rank):
     """Reference arm: the CPU oracle, as it stands, on the host cores."""
     if rank != 0:
@@ -278,7 +350,7 @@ def run_reference(args, rank):
     total = sum(times)
     value = 2.0 * R * p.N * p.K * len(times) / total / 1e12
     line = {
-        "impl": "reference", "metric": METRIC if p.kind == "bf16" else METRIC_MXFP8, "value": value,
+        "impl": "reference", "metric": metric_of(p.kind), "value": value,
         "unit": UNIT, "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -353,21 +425,43 @@ def main():
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
         pass
+    # Working sets under twice the L2 would be served partly from L2 across
+    # back-to-back steps: flush it between steps (write a buffer larger than
+    # L2 outside the events) and time each step on its own.
+    traffic_bytes = p.in_bytes + p.out_bytes
+    flush = traffic_bytes < 2 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
     sampler = ClockSampler(gpu_id)
     sampler.start()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     barrier()
     torch.cuda.synchronize()
-    ev[0].record(stream)
-    for i in range(args.steps):
-        p.call(G, dev, C, stream)
-        ev[i + 1].record(stream)
+    if flush:
+        ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            scratch.zero_()
+            ev_s[i].record(stream)
+            p.call(G, dev, C, stream)
+            ev_e[i].record(stream)
+    else:
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(stream)
+        for i in range(args.steps):
+            p.call(G, dev, C, stream)
+            ev[i + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
     sampler.stop()
     G.gemm_check_device_status(stream)
-    per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    t_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, "cuda")
+    if flush:
+        per_step_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+        local_ms = sum(per_step_ms)
+    else:
+        per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+        local_ms = ev[0].elapsed_time(ev[-1])
+    t_ms = max_over_ranks(local_ms, world, "cuda")
+
+    fusion = fusion_comparison(p, G, dev, torch, stream, min(args.steps, 50)) if p.kind == "fused" else None
 
     # ------------------------------------------- end to end, host buffers --
     e2e = None
@@ -413,9 +507,9 @@ def main():
     achieved = p.flops / (mean_step_ms * 1e-3) / 1e12
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    ratio = 1.0 if p.kind == "bf16" else FP8_OVER_BF16
+    ratio = FP8_OVER_BF16 if p.kind == "mxfp8" else 1.0
     peak = bf16_peak * ratio
-    peak_note = (f"{peak_src} bf16_tflops (burst, cuBLAS 8192^3)" if p.kind == "bf16" else
+    peak_note = (f"{peak_src} bf16_tflops (burst, cuBLAS 8192^3)" if p.kind != "mxfp8" else
                  f"{peak_src} bf16_tflops x {FP8_OVER_BF16:g} (nominal fp8/bf16 dense ratio)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": profile_traffic(p.name, cfg_name),
@@ -432,17 +526,17 @@ def main():
                "sample": f"rows 0..{R - 1} of A against all of B ({R}x{p.N}x{p.K}), fp64 triple loop, "
                          f"{dt:.1f} s"}
 
-    traffic_bytes = p.in_bytes + p.out_bytes
     line = {
-        "metric": METRIC if p.kind == "bf16" else METRIC_MXFP8, "value": value, "unit": UNIT,
+        "metric": metric_of(p.kind), "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if p.kind == "bf16" else "e4m3",
+        "dtype": "e4m3" if p.kind == "mxfp8" else "bf16",
         "data": "synthetic",
         "config": {"workload": p.desc, "M": p.M, "N": p.N, "K": p.K, "kernel_config": cfg_name,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": (f"no flush: inputs+output {traffic_bytes / 2**20:.0f} MiB > 126 MiB L2"
-                          if traffic_bytes > L2_BYTES else "inputs fit in L2 (not flushed)"),
+                   "l2": (f"flushed between steps ({2 * L2_BYTES // 2**20} MiB written outside the events): "
+                          f"inputs+output {traffic_bytes / 2**20:.0f} MiB < 2 x 126 MiB L2" if flush else
+                          f"no flush: inputs+output {traffic_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2"),
                    "step_ms_median": statistics.median(per_step_ms),
                    "step_ms_p90": float(np.percentile(per_step_ms, 90))},
         "e2e": e2e,
@@ -451,6 +545,11 @@ def main():
         "clocks": sampler.summary(),
         "gpu_launches": args.steps * p.launches(G) * world,
     }
+    if fusion:
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        fusion["ledger_saved_ms_at_hbm_peak"] = fusion["ledger_saved_bytes"] / (hbm * 1e9) * 1e3
+        fusion["unfused_pass_frac_of_hbm_peak"] = fusion["unfused_pass_gbs"] / hbm
+        line["fusion"] = fusion
     print(json.dumps(line), flush=True)
 
 

@@ -10,9 +10,10 @@ fallback path.
 from importlib import import_module
 
 _BINDING_NAMES = {
-    "gemm_bf16", "gemm_bf16_ex", "gemm_bf16_noalloc", "gemm_mxfp8", "gemm_check_device_status", "gemm_status_string",
+    "gemm_bf16", "gemm_bf16_ex", "gemm_bf16_fused", "gemm_bf16_noalloc", "gemm_mxfp8", "gemm_check_device_status", "gemm_status_string",
     "gemm_force_config", "gemm_select_config", "gemm_launches_per_call",
-    "gemm_last_timeout_detail", "GemmError", "OUT_F32", "OUT_BF16", "KMAJOR", "MNMAJOR", "CONFIGS",
+    "gemm_last_timeout_detail", "GemmError", "OUT_F32", "OUT_BF16", "KMAJOR", "MNMAJOR", "ACT_NONE", "ACT_RELU",
+    "ACT_GELU", "CONFIGS",
     "STATUS_NAMES", "lib", "library_path",
 }
 

@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "b200gemm.h"
 #include "gemm_bf16_sm100.cuh"
@@ -34,6 +35,9 @@ using Cfg2x256F32C = b200::GemmBf16Cfg<2, 256, 6, 0, true>;
 using Cfg2x256B16C = b200::GemmBf16Cfg<2, 256, 6, 1, true>;
 using Cfg1x256F32C = b200::GemmBf16Cfg<1, 256, 4, 0, true>;
 using Cfg1x256B16C = b200::GemmBf16Cfg<1, 256, 4, 1, true>;
+// two MMA consumers sharing B: 512 x 256 pair tiles, single-buffered TMEM
+using Cfg2x512F32C = b200::GemmBf16Cfg<2, 256, 4, 0, true, 2>;
+using Cfg2x512B16C = b200::GemmBf16Cfg<2, 256, 4, 1, true, 2>;
 using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
@@ -63,6 +67,9 @@ struct DeviceState {
     uint8_t *sk_ws = nullptr;
     size_t sk_ws_bytes = 0;
     uint32_t sk_epoch = 0;
+    // Workspaces replaced by larger ones.  They are kept, not freed: a CUDA
+    // graph captured earlier still holds their addresses.
+    std::vector<void *> retired;
 };
 
 std::mutex g_mutex;
@@ -113,9 +120,21 @@ uint32_t inject_flags() {
     return (s && s[0] == '1') ? b200::kInjectDropFirstStage : 0u;
 }
 
+// True while `stream` is being captured into a CUDA graph (or when that
+// cannot be told, so that no one-time set-up runs inside a capture).
+bool capturing(cudaStream_t stream) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return true;
+    }
+    return cs != cudaStreamCaptureStatusNone;
+}
+
 // Device of the current thread, checked to be compute capability 10.0, with
-// its status block allocated.
-gemm_status_t current_device(int &dev, DeviceState *&st) {
+// its status block allocated.  The one-time set-up (cudaMalloc, a blocking
+// cudaMemset) may not run inside a stream capture: GEMM_ERR_CAPTURE then.
+gemm_status_t current_device(int &dev, DeviceState *&st, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         g_last_cuda_error = static_cast<int>(e);
@@ -124,6 +143,7 @@ gemm_status_t current_device(int &dev, DeviceState *&st) {
     std::lock_guard<std::mutex> lock(g_mutex);
     st = &g_devices[dev];
     if (!st->ready) {
+        if (capturing(stream)) return GEMM_ERR_CAPTURE;
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
@@ -215,7 +235,8 @@ gemm_status_t encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void 
 
 gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     const int forced = g_forced.load(std::memory_order_relaxed);
-    if (forced != GEMM_CFG_AUTO && forced < GEMM_CFG_MXFP8_1CTA_128x256) return static_cast<gemm_config_t>(forced);
+    if (forced != GEMM_CFG_AUTO && forced != GEMM_CFG_MXFP8_1CTA_128x256 && forced != GEMM_CFG_MXFP8_2CTA_256x256)
+        return static_cast<gemm_config_t>(forced);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int64_t wide_tiles = ((M + 127) / 128) * ((N + 255) / 256);
     // two or more waves of pair tiles: Cluster Launch Control evens out the
@@ -234,7 +255,8 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
 template <class Cfg>
 gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, const void *B, void *C,
                           int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                          cudaStream_t stream, float alpha = 1.0f, float beta = 0.0f, uint32_t layout = 0) {
+                          cudaStream_t stream, const b200::Epilogue &epi = b200::plain_epilogue(),
+                          uint32_t layout = 0) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
     cudaError_t e;
@@ -252,6 +274,7 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!st->attr_done[cfg_id][oi]) {
+            if (capturing(stream)) return GEMM_ERR_CAPTURE;
             if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           Cfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
@@ -297,7 +320,7 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
                            static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
-                           watchdog_ns(K), inject_flags(), alpha, beta, layout);
+                           watchdog_ns(K), inject_flags(), epi, layout);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -328,14 +351,15 @@ SkinnyLayout skinny_layout(int64_t N, int64_t K, int sm_count) {
     return l;
 }
 
-// Grows the skinny workspace on demand (counters start at zero; cudaFree
-// waits for the device to go idle before the old buffer goes).
-gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
+// Grows the skinny workspace on demand (counters start at zero).  Growing
+// is refused inside a stream capture; the old buffer is retired, not freed.
+gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (st->sk_ws_bytes < bytes) {
+        if (capturing(stream)) return GEMM_ERR_CAPTURE;
         cudaError_t e;
         if (st->sk_ws) {
-            if ((e = cudaFree(st->sk_ws)) != cudaSuccess) return cuda_fail(e);
+            st->retired.push_back(st->sk_ws);
             st->sk_ws = nullptr;
             st->sk_ws_bytes = 0;
         }
@@ -351,13 +375,14 @@ gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
 template <class Cfg>
 gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const void *B, void *C, int64_t M,
                             int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
-                            float alpha, float beta, uint32_t layout) {
+                            const b200::Epilogue &epi, uint32_t layout) {
     auto kernel = b200::gemm_bf16_skinny_sm100_kernel<Cfg>;
     cudaError_t e;
     uint32_t epoch;
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!st->sk_attr_done[attr_slot]) {
+            if (capturing(stream)) return GEMM_ERR_CAPTURE;
             if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           Cfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
@@ -369,7 +394,8 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
     const SkinnyLayout l = skinny_layout<Cfg>(N, K, st->sm_count);
     uint8_t *ws = nullptr;
     gemm_status_t s;
-    if ((s = sk_workspace(st, static_cast<size_t>(l.partial_bytes + l.counter_bytes), ws)) != GEMM_OK) return s;
+    if ((s = sk_workspace(st, static_cast<size_t>(l.partial_bytes + l.counter_bytes), ws, stream)) != GEMM_OK)
+        return s;
     const int64_t mpad = (M + 15) / 16 * 16;
     alignas(64) CUtensorMap tmB, tmA;
     if (layout & b200::kLayoutBMajorN)
@@ -384,35 +410,34 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
     unsigned long long *counters = reinterpret_cast<unsigned long long *>(ws + l.partial_bytes);
     kernel<<<static_cast<unsigned>(l.grid), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
         tmB, tmA, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(mpad), C, ldc,
-        partials, counters, static_cast<int>(l.slots), epoch, st->status, watchdog_ns(K), alpha, beta, layout);
+        partials, counters, static_cast<int>(l.slots), epoch, st->status, watchdog_ns(K), epi, layout);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
 
 gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const void *B, void *C, int64_t M,
                                 int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
-                                float alpha = 1.0f, float beta = 0.0f, uint32_t layout = 0) {
+                                const b200::Epilogue &epi = b200::plain_epilogue(), uint32_t layout = 0) {
     // the skinny kernel reads A K-major only (A stored M x K)
     if (M > 256 || (layout & b200::kLayoutAMajorM)) return GEMM_ERR_INVALID_VALUE;
     if (M <= 64)
-        return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                   : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
+        return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                   : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
     if (M <= 128)
-        return f32 ? launch_skinny<CfgSk128F32>(st, 2, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                   : launch_skinny<CfgSk128B16>(st, 3, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-    return f32 ? launch_skinny<CfgSk256F32>(st, 4, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-               : launch_skinny<CfgSk256B16>(st, 5, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
+        return f32 ? launch_skinny<CfgSk128F32>(st, 2, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                   : launch_skinny<CfgSk128B16>(st, 3, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+    return f32 ? launch_skinny<CfgSk256F32>(st, 4, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+               : launch_skinny<CfgSk256B16>(st, 5, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
 }
 
-// C = beta * C (K == 0 with beta != 0): the empty sum plus the beta term.
+// C = act(beta * C + bias) for K == 0 (the empty product, then the epilogue).
 template <typename T>
-gemm_status_t launch_scale(void *C, int64_t M, int64_t N, int64_t ldc, float beta, int sm_count,
-                           cudaStream_t stream) {
-    const int64_t total = M * N;
-    int64_t blocks = (total + 255) / 256;
+gemm_status_t launch_epilogue_only(void *C, int64_t M, int64_t N, int64_t ldc, const b200::Epilogue &epi,
+                                   int sm_count, cudaStream_t stream) {
     const int64_t cap = static_cast<int64_t>(sm_count) * 8;
-    if (blocks > cap) blocks = cap;
-    b200::scale_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<T *>(C), M, N, ldc, beta);
+    const int64_t blocks = M < cap ? M : cap;
+    b200::epilogue_only_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<T *>(C), M, N,
+                                                                                      ldc, epi);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
 }
@@ -426,6 +451,36 @@ gemm_status_t launch_zero(void *C, int64_t M, int64_t N, int64_t ldc, int sm_cou
     b200::zero_fill_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<T *>(C), M, N, ldc);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
+// The dense bf16 kernels, by configuration.
+gemm_status_t launch_dense(DeviceState *st, gemm_config_t cfg, bool f32, const void *A, const void *B, void *C,
+                           int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                           cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout) {
+    switch (cfg) {
+        case GEMM_CFG_1CTA_128x256:
+            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_1CTA_128x128:
+            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_2CTA_256x256:
+            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_SKINNY:
+            return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_2CTA_256x256_CLC:
+            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_2CTA_512x256_CLC:
+            return f32 ? launch_bf16<Cfg2x512F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x512B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_1CTA_128x256_CLC:
+            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        default:
+            return GEMM_ERR_INVALID_VALUE;
+    }
 }
 
 // ------------------------------------------------ allocation-free variant --
@@ -447,7 +502,7 @@ DeviceState g_noalloc_devices[kMaxDevices];
 // Per-device set-up, once, with the device current: check the device, take
 // the address of the scratch array with cudaGetSymbolAddress (host code may
 // not use the array's name as a device address), and zero it.
-gemm_status_t noalloc_device(int &dev, DeviceState *&st) {
+gemm_status_t noalloc_device(int &dev, DeviceState *&st, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         g_last_cuda_error = static_cast<int>(e);
@@ -456,6 +511,7 @@ gemm_status_t noalloc_device(int &dev, DeviceState *&st) {
     std::lock_guard<std::mutex> lock(g_mutex);
     st = &g_noalloc_devices[dev];
     if (!st->ready) {
+        if (capturing(stream)) return GEMM_ERR_CAPTURE;
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
@@ -512,14 +568,16 @@ MxLayout mx_layout(int64_t M, int64_t N, int64_t K, int cg) {
     return l;
 }
 
-// Grows the device's workspace on demand.  cudaFree waits for the device to
-// go idle, so work still using the old buffer has finished before it goes.
-gemm_status_t mx_workspace(DeviceState *st, size_t bytes, uint8_t *&ws) {
+// Grows the device's workspace on demand.  Growing is refused inside a
+// stream capture; the old buffer is retired, not freed (work queued on it,
+// or a graph captured with its address, may still use it).
+gemm_status_t mx_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (st->mx_ws_bytes < bytes) {
+        if (capturing(stream)) return GEMM_ERR_CAPTURE;
         cudaError_t e;
         if (st->mx_ws) {
-            if ((e = cudaFree(st->mx_ws)) != cudaSuccess) return cuda_fail(e);
+            st->retired.push_back(st->mx_ws);
             st->mx_ws = nullptr;
             st->mx_ws_bytes = 0;
         }
@@ -551,6 +609,7 @@ gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const u
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!st->mx_attr_done[attr_slot]) {
+            if (capturing(stream)) return GEMM_ERR_CAPTURE;
             if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           Cfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
@@ -568,7 +627,7 @@ gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const u
     const MxLayout l = mx_layout(M, N, K, Cfg::CG);
     uint8_t *ws = nullptr;
     gemm_status_t s;
-    if ((s = mx_workspace(st, l.bytes(), ws)) != GEMM_OK) return s;
+    if ((s = mx_workspace(st, l.bytes(), ws, stream)) != GEMM_OK) return s;
 
     // 1. scales -> TMEM-ready 512-byte chunks
     const int64_t blocks = (l.a_blocks + l.b_blocks) * ((l.kb + b200::kRepackKb - 1) / b200::kRepackKb);
@@ -598,10 +657,12 @@ gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const u
 
 extern "C" {
 
-gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
-                           int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, gemm_layout_t a_layout,
-                           gemm_layout_t b_layout, float alpha, float beta, cudaStream_t stream) {
+gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                              int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, gemm_layout_t a_layout,
+                              gemm_layout_t b_layout, float alpha, float beta, const float *bias, gemm_act_t act,
+                              cudaStream_t stream) {
     if (c_type != GEMM_OUT_F32 && c_type != GEMM_OUT_BF16) return GEMM_ERR_INVALID_VALUE;
+    if (act != GEMM_ACT_NONE && act != GEMM_ACT_RELU && act != GEMM_ACT_GELU) return GEMM_ERR_INVALID_VALUE;
     if ((a_layout != GEMM_LAYOUT_KMAJOR && a_layout != GEMM_LAYOUT_MNMAJOR) ||
         (b_layout != GEMM_LAYOUT_KMAJOR && b_layout != GEMM_LAYOUT_MNMAJOR))
         return GEMM_ERR_INVALID_VALUE;
@@ -609,42 +670,35 @@ gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C, int64_t M, int
     const int64_t ec = c_type == GEMM_OUT_F32 ? 4 : 2;
     gemm_status_t s = check_args(A, B, C, M, N, K, lda, ldb, ldc, 2, 2, ec, a_mn, b_mn);
     if (s != GEMM_OK || M == 0 || N == 0) return s;
+    if (bias) {
+        if (!aligned16(bias)) return GEMM_ERR_MISALIGNED;
+        if (overlaps(C, M, N, ldc, ec, bias, 1, N, N, 4)) return GEMM_ERR_ALIAS;
+    }
+    const b200::Epilogue epi{alpha, beta, bias, static_cast<uint32_t>(act)};
     int dev;
     DeviceState *st;
-    if ((s = current_device(dev, st)) != GEMM_OK) return s;
+    if ((s = current_device(dev, st, stream)) != GEMM_OK) return s;
     const bool f32 = c_type == GEMM_OUT_F32;
     if (K == 0) {
-        // the empty sum: C = beta * C (zeros when beta == 0, C not read)
-        if (beta == 0.0f)
+        // the empty sum: C = act(beta * C + bias); plain zeros (C not read)
+        // when there is neither a beta term, a bias nor an activation
+        if (beta == 0.0f && !bias && act == GEMM_ACT_NONE)
             return f32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
                        : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
-        return f32 ? launch_scale<float>(C, M, N, ldc, beta, st->sm_count, stream)
-                   : launch_scale<__nv_bfloat16>(C, M, N, ldc, beta, st->sm_count, stream);
+        return f32 ? launch_epilogue_only<float>(C, M, N, ldc, epi, st->sm_count, stream)
+                   : launch_epilogue_only<__nv_bfloat16>(C, M, N, ldc, epi, st->sm_count, stream);
     }
     const uint32_t layout = (a_mn ? b200::kLayoutAMajorM : 0u) | (b_mn ? b200::kLayoutBMajorN : 0u);
     gemm_config_t cfg = select_config(M, N, K);
     if (cfg == GEMM_CFG_SKINNY && a_mn) cfg = GEMM_CFG_1CTA_128x128;   // skinny reads A K-major only
-    switch (cfg) {
-        case GEMM_CFG_1CTA_128x256:
-            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-        case GEMM_CFG_1CTA_128x128:
-            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-        case GEMM_CFG_2CTA_256x256:
-            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-        case GEMM_CFG_SKINNY:
-            return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-        case GEMM_CFG_2CTA_256x256_CLC:
-            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-        case GEMM_CFG_1CTA_128x256_CLC:
-            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout)
-                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, alpha, beta, layout);
-        default:
-            return GEMM_ERR_INVALID_VALUE;
-    }
+    return launch_dense(st, cfg, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+}
+
+gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                           int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, gemm_layout_t a_layout,
+                           gemm_layout_t b_layout, float alpha, float beta, cudaStream_t stream) {
+    return gemm_bf16_fused(A, B, C, M, N, K, lda, ldb, ldc, c_type, a_layout, b_layout, alpha, beta, nullptr,
+                           GEMM_ACT_NONE, stream);
 }
 
 gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
@@ -667,7 +721,7 @@ gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const
     }
     int dev;
     DeviceState *st;
-    if ((s = current_device(dev, st)) != GEMM_OK) return s;
+    if ((s = current_device(dev, st, stream)) != GEMM_OK) return s;
     if (K == 0) return launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
     if (select_mx_config(M, N) == GEMM_CFG_MXFP8_2CTA_256x256)
         return launch_mxf8<CfgMxf8Pair>(st, 1, A, sfa, B, sfb, C, M, N, K, lda, ldb, ldc, stream);
@@ -709,6 +763,7 @@ const char *gemm_status_string(gemm_status_t s) {
         case GEMM_ERR_LAUNCH: return "GEMM_ERR_LAUNCH: a CUDA runtime or driver call failed";
         case GEMM_ERR_TIMEOUT: return "GEMM_ERR_TIMEOUT: a bounded wait inside a kernel expired (device watchdog)";
         case GEMM_ERR_TOO_LARGE: return "GEMM_ERR_TOO_LARGE: a dimension or stride exceeds the TMA limits";
+        case GEMM_ERR_CAPTURE: return "GEMM_ERR_CAPTURE: one-time set-up (device state, kernel attributes or workspace growth) cannot run inside a stream capture; make one call with the same shapes outside the capture first";
         default: return "unknown gemm_status_t";
     }
 }
@@ -738,7 +793,7 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
     if (noalloc_scratch_bytes() > kNoAllocScratchBytes) return GEMM_ERR_TOO_LARGE;
     int dev;
     DeviceState *st;
-    if ((s = noalloc_device(dev, st)) != GEMM_OK) return s;
+    if ((s = noalloc_device(dev, st, stream)) != GEMM_OK) return s;
     if (K == 0) {
         return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
                                       : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
@@ -750,20 +805,8 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
     // the one-CTA 128 x 128 kernel instead.
     gemm_config_t cfg = select_config(M, N, K);
     if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128;
-    const bool f32 = c_type == GEMM_OUT_F32;
-    switch (cfg) {
-        case GEMM_CFG_1CTA_128x256:
-            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
-        case GEMM_CFG_1CTA_128x128:
-            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
-        case GEMM_CFG_2CTA_256x256:
-            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream)
-                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream);
-        default:
-            return GEMM_ERR_INVALID_VALUE;
-    }
+    return launch_dense(st, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc, stream,
+                        b200::plain_epilogue(), 0u);
 }
 
 }  // extern "C"

@@ -83,16 +83,18 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         : "r"(taddr));
 }
 
-// C[m][n] = alpha * v + beta * C[m][n]  (C read only when beta != 0).
+// C[m][n] = finish(v, C[m][n], bias[n]): the fused epilogue of one element
+// (C read only when beta != 0).
 template <int OUT>
-__device__ __forceinline__ void store_c(void *C, int64_t ldc, int m, int n, float v, float alpha, float beta) {
+__device__ __forceinline__ void store_c(void *C, int64_t ldc, int m, int n, float v, const Epilogue &e) {
     const int64_t i = static_cast<int64_t>(m) * ldc + n;
+    const float b = e.bias ? __ldg(e.bias + n) : 0.0f;
     if constexpr (OUT == 0) {
         float *c = static_cast<float *>(C);
-        c[i] = beta != 0.0f ? fmaf(alpha, v, beta * c[i]) : alpha * v;
+        c[i] = finish(v, e.beta != 0.0f ? c[i] : 0.0f, b, e);
     } else {
         __nv_bfloat16 *c = static_cast<__nv_bfloat16 *>(C);
-        c[i] = __float2bfloat16_rn(beta != 0.0f ? fmaf(alpha, v, beta * __bfloat162float(c[i])) : alpha * v);
+        c[i] = __float2bfloat16_rn(finish(v, e.beta != 0.0f ? __bfloat162float(c[i]) : 0.0f, b, e));
     }
 }
 
@@ -106,7 +108,7 @@ template <int OUT>
 __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_elems, int slots_per_cta,
                                            int64_t c_lo, int64_t c_hi, int64_t t, int64_t total, int64_t g,
                                            int64_t kb_per_tile, int M, int N, void *C, int64_t ldc,
-                                           uint32_t epi_tid, float alpha, float beta) {
+                                           uint32_t epi_tid, const Epilogue &epi) {
     constexpr int ROWS = 8;                      // rows per round for this thread
     const int n4 = static_cast<int>(epi_tid & 31u) * 4;
     const int msub = static_cast<int>(epi_tid >> 5);
@@ -147,9 +149,9 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
             const int m = m0 + 4 * r;
             if (m >= M || n >= N) continue;
             float vals[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
-            if (n + 4 <= N && (alpha != 1.0f || beta != 0.0f)) {
+            if (n + 4 <= N && !epi.identity()) {
                 float old[4] = {0.f, 0.f, 0.f, 0.f};
-                if (beta != 0.0f) {
+                if (epi.beta != 0.0f) {
                     if constexpr (OUT == 0) {
                         const float4 x = *reinterpret_cast<const float4 *>(static_cast<const float *>(C) +
                                                                            static_cast<int64_t>(m) * ldc + n);
@@ -161,8 +163,11 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
                         old[2] = __uint_as_float(x.y << 16); old[3] = __uint_as_float(x.y & 0xFFFF0000u);
                     }
                 }
+                float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (epi.bias) b = __ldg(reinterpret_cast<const float4 *>(epi.bias + n));
+                const float bb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) vals[q] = beta != 0.0f ? fmaf(alpha, vals[q], beta * old[q]) : alpha * vals[q];
+                for (int q = 0; q < 4; ++q) vals[q] = finish(vals[q], old[q], bb[q], epi);
                 acc[r] = make_float4(vals[0], vals[1], vals[2], vals[3]);
             }
             if (n + 4 <= N) {
@@ -177,7 +182,7 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
             } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    if (n + q < N) store_c<OUT>(C, ldc, m, n + q, vals[q], alpha, beta);
+                    if (n + q < N) store_c<OUT>(C, ldc, m, n + q, vals[q], epi);
             }
         }
     }
@@ -190,7 +195,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                               int M, int N, int K, int mpad, void *C, int64_t ldc,
                               float *partials, unsigned long long *counters, int slots_per_cta,
                               uint32_t epoch, DeviceStatus *status, uint64_t timeout_ns,
-                              float alpha, float beta, uint32_t layout) {
+                              Epilogue epi, uint32_t layout) {
     // B stored K x N arrives as MN-major tiles; A must be stored M x K here.
     const bool b_mn = (layout & kLayoutBMajorN) != 0;
     extern __shared__ uint8_t smem_raw[];
@@ -360,7 +365,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                     if (m < M) {
                         const float x = __uint_as_float(v[i]);
                         if (shared_tile) my_partial[static_cast<int64_t>(m) * Cfg::TILE_N + n_local] = x;
-                        else if (n < N) store_c<Cfg::OUT>(C, ldc, m, n, x, alpha, beta);
+                        else if (n < N) store_c<Cfg::OUT>(C, ldc, m, n, x, epi);
                     }
                 }
             }
@@ -392,7 +397,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 if (*last_flag) {
                     __threadfence();
                     fixup_tile<Cfg::OUT>(partials, slot_elems, slots_per_cta, c_lo, c_hi, t, total, g,
-                                         kb_per_tile, M, N, C, ldc, epi_tid, alpha, beta);
+                                         kb_per_tile, M, N, C, ldc, epi_tid, epi);
                     // every contributor has arrived: leave the counter at zero
                     // arrivals so a replay of this launch (same epoch, e.g.
                     // from a CUDA graph) starts from a clean count

@@ -31,8 +31,9 @@
 //
 // Operands may be K-major (A as M x K, B as N x K) or MN-major (A as K x M,
 // B as K x N): MN-major tiles arrive as 64-wide boxes and the MMA reads them
-// through MN-major descriptors.  The epilogue computes alpha * A.B + beta * C
-// (C read only when beta != 0).
+// through MN-major descriptors.  The epilogue computes
+// act(alpha * A.B + beta * C + bias) in fp32 before the output rounding
+// (epilogue.cuh; C read only when beta != 0).
 //
 // Tails: TMA loads zero-fill outside [0,K) x [0,M) / [0,N) element by
 // element.  TMA stores clip rows exactly but write whole 16-byte granules
@@ -44,6 +45,7 @@
 
 #include <cstdint>
 
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace b200 {
@@ -74,27 +76,34 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     return p;
 }
 
-template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false>
+template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1>
 struct GemmBf16Cfg {
     static constexpr bool CLC = CLC_;              // tiles from Cluster Launch Control, not a fixed stride
     static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
     static constexpr int BN = BN_;                 // tile N == MMA N
     static constexpr int STAGES = STAGES_;         // shared-memory ring depth
     static constexpr int OUT = OUT_;               // 0: f32 C, 1: bf16 C
-    static constexpr int BM_CTA = 128;             // accumulator rows per CTA (TMEM lanes)
-    static constexpr int BM = 128 * CG;            // tile M == MMA M
+    // MMA consumers per tile: 2 stacks two MMA-M row blocks in one tile that
+    // share every B k-tile (a 512 x 256 pair tile), each with its own TMEM
+    // accumulator; TMEM then holds no second tile, so it is single-buffered.
+    static constexpr int CONSUMERS = CONSUMERS_;
+    static constexpr int BM_CTA = 128;             // accumulator rows per CTA and consumer (TMEM lanes)
+    static constexpr int BM_MMA = 128 * CG;        // MMA M
+    static constexpr int BM = BM_MMA * CONSUMERS;  // tile M
     static constexpr int BK = 64;                  // 64 bf16 = one 128-byte swizzle row
     static constexpr int UMMA_K = 16;              // K per tcgen05.mma (kind::f16)
     static constexpr int B_ROWS = BN / CG;         // B rows this CTA loads per k-tile
-    static constexpr int A_BYTES = BM_CTA * BK * 2;
+    static constexpr int A_PART_BYTES = BM_CTA * BK * 2;     // one consumer's A rows of this CTA
+    static constexpr int A_BYTES = CONSUMERS * A_PART_BYTES;
     static constexpr int B_BYTES = B_ROWS * BK * 2;
+    static constexpr int ACC_BUFS = CONSUMERS == 1 ? 2 : 1;  // tiles held in TMEM at once
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TX_BYTES = STAGE_BYTES * CG;   // bytes landing on the leader's full[s]
     static constexpr int EPI_COLS = OUT == 0 ? 32 : 64; // columns in one 128-byte staged row
     static constexpr int EPI_CHUNKS = BN / EPI_COLS;
     static constexpr int EPI_BUF = 32 * 128;       // one warp's 32 rows x 128 bytes
     static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
-    static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
+    static constexpr int TMEM_COLS = pow2_at_least(ACC_BUFS * CONSUMERS * BN, 32);
     // full[S], empty[S], tmem_full[2], tmem_empty[2] (+ clc[2], sched_full[2], sched_empty[2])
     static constexpr int NUM_BARS = 2 * STAGES + 4 + (CLC ? 6 : 0);
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
@@ -104,12 +113,14 @@ struct GemmBf16Cfg {
     static constexpr int SCHED_CONSUMERS = CG == 1 ? 6 : 11;  // arrivals that free a tile slot
 
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
+    static_assert(CONSUMERS == 1 || CONSUMERS == 2, "one or two MMA consumers");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
     static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows <= 256, whole 8-row swizzle atoms");
     static_assert(BN % EPI_COLS == 0, "epilogue chunks cover the tile");
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
+    static_assert(SMEM_BYTES < (1 << 18), "descriptor start addresses (18 bits) cannot carry");
 };
 
 // Tile index -> (tile row, tile column), grouped along M so that CTAs
@@ -167,60 +178,6 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk, bool mn)
     return mn ? sw128_mnmajor_desc(base + 2048u * kk) : sw128_kmajor_desc(base + 32u * kk);
 }
 
-// v[j] <- alpha * v[j] + beta * C[row][col0 + j] for 32 fp32 values held as
-// bits (C fp32); C is read only when beta != 0 and only inside M x N.
-__device__ __forceinline__ void axpby_f32(uint32_t (&v)[32], const void *C, int64_t ldc, int row, int col0,
-                                          int M, int N, float alpha, float beta) {
-    const float *crow = static_cast<const float *>(C) + static_cast<int64_t>(row) * ldc;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        float old[4] = {0.f, 0.f, 0.f, 0.f};
-        const int col = col0 + 4 * q;
-        if (beta != 0.0f && row < M) {
-            if (col + 4 <= N) {
-                const float4 x = *reinterpret_cast<const float4 *>(crow + col);
-                old[0] = x.x; old[1] = x.y; old[2] = x.z; old[3] = x.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (col + e < N) old[e] = crow[col + e];
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float acc = __uint_as_float(v[4 * q + e]);
-            v[4 * q + e] = __float_as_uint(beta != 0.0f ? fmaf(alpha, acc, beta * old[e]) : alpha * acc);
-        }
-    }
-}
-
-// The same for 32 fp32 accumulator values whose C elements are bf16.
-__device__ __forceinline__ void axpby_bf16src(uint32_t (&v)[32], const void *C, int64_t ldc, int row, int col0,
-                                              int M, int N, float alpha, float beta) {
-    const uint16_t *crow = static_cast<const uint16_t *>(C) + static_cast<int64_t>(row) * ldc;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        const int col = col0 + 8 * q;
-        if (beta != 0.0f && row < M) {
-            if (col + 8 <= N) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(crow + col);
-                w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (col + e < N) w[e >> 1] |= static_cast<uint32_t>(crow[col + e]) << (16 * (e & 1));
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float old = __uint_as_float((w[e >> 1] >> (16 * (e & 1))) << 16);   // bf16 -> f32
-            const float acc = __uint_as_float(v[8 * q + e]);
-            v[8 * q + e] = __float_as_uint(beta != 0.0f ? fmaf(alpha, acc, beta * old) : alpha * acc);
-        }
-    }
-}
-
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -228,7 +185,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmC,
                        int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m,
                        DeviceStatus *status, uint64_t timeout_ns, uint32_t inject,
-                       float alpha, float beta, uint32_t layout) {
+                       Epilogue epi, uint32_t layout) {
     constexpr int CG = Cfg::CG;
     const bool a_mn = (layout & kLayoutAMajorM) != 0;   // A stored K x M
     const bool b_mn = (layout & kLayoutBMajorN) != 0;   // B stored K x N
@@ -333,7 +290,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int tile = cluster_id; ok && tile >= 0;) {
                 int tm, tn;
                 raster_tile(tile, num_m, num_n, group_m, tm, tn);
-                const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;
+                const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;   // + c * BM_MMA
                 const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
@@ -358,7 +315,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         if (rank == leader_rank) mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
                         bar = map_to_cta(full_bar(stage), leader_rank);
                     }
-                    load_operand_tile<CG>(a_dst, &tmA, bar, kx, a_row, Cfg::BM_CTA, a_mn);
+#pragma unroll
+                    for (int c = 0; c < Cfg::CONSUMERS; ++c)
+                        load_operand_tile<CG>(a_dst + c * Cfg::A_PART_BYTES, &tmA, bar, kx, a_row + c * Cfg::BM_MMA,
+                                              Cfg::BM_CTA, a_mn);
                     load_operand_tile<CG>(b_dst, &tmB, bar, kx, b_row, Cfg::B_ROWS, b_mn);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -380,20 +340,29 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
         if (rank == 0 && lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN, a_mn ? 1u : 0u, b_mn ? 1u : 0u);
+            const uint32_t idesc = idesc_bf16_f32(Cfg::BM_MMA, Cfg::BN, a_mn ? 1u : 0u, b_mn ? 1u : 0u);
+            // Descriptors of stage 0, K step 0.  A stage, a consumer's A part
+            // and a K step add their byte offset >> 4 to the start-address
+            // field (bits 0-13), which cannot carry out: shared addresses
+            // stay below 2^18.  One add per operand per MMA keeps the issue
+            // loop as short as with compile-time layouts.
+            const uint64_t a_desc0 = operand_desc(base, 0, a_mn);
+            const uint64_t b_desc0 = operand_desc(base + Cfg::A_BYTES, 0, b_mn);
+            const uint32_t a_kstep = (a_mn ? 2048u : 32u) >> 4;
+            const uint32_t b_kstep = (b_mn ? 2048u : 32u) >> 4;
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             int t = 0;
             for (int tile = cluster_id; ok && tile >= 0; ++t) {
-                const uint32_t buf = static_cast<uint32_t>(t) & 1u;
-                const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
+                const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
+                const uint32_t acc_phase = (static_cast<uint32_t>(t) / Cfg::ACC_BUFS) & 1u;
                 if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, 3 * timeout_ns)) {
                     record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarTmemEmpty);
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + buf * Cfg::BN;
+                const uint32_t d_tmem = tmem_base + buf * Cfg::CONSUMERS * Cfg::BN;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarFull);
@@ -401,12 +370,15 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a0 = base + stage * Cfg::STAGE_BYTES;
-                    const uint32_t b0 = a0 + Cfg::A_BYTES;
+                    const uint64_t soff = (stage * Cfg::STAGE_BYTES) >> 4;
 #pragma unroll
                     for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
-                        mma_bf16_ss<CG>(d_tmem, operand_desc(a0, kk, a_mn), operand_desc(b0, kk, b_mn), idesc,
-                                        (kb | kk) != 0 ? 1u : 0u);
+                        const uint64_t bd = b_desc0 + soff + kk * b_kstep;
+#pragma unroll
+                        for (int c = 0; c < Cfg::CONSUMERS; ++c)   // both consumers read this B k-step
+                            mma_bf16_ss<CG>(d_tmem + c * Cfg::BN,
+                                            a_desc0 + soff + (c * Cfg::A_PART_BYTES >> 4) + kk * a_kstep, bd, idesc,
+                                            (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit<CG>(empty_bar(stage), 0x3);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -453,15 +425,15 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         // ----------------------------------------------------- epilogue --
         const uint32_t sub = warp & 3u;            // TMEM lanes [32*sub, 32*sub + 32)
         const uint32_t ew = warp - 2u;             // staging slot
-        const bool scaled = !(alpha == 1.0f && beta == 0.0f);
+        const bool fused = !epi.identity();
         const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
         uint32_t nstore = 0;
         int t = 0;
         for (int tile = cluster_id; tile >= 0; ++t) {
             int tm, tn;
             raster_tile(tile, num_m, num_n, group_m, tm, tn);
-            const uint32_t buf = static_cast<uint32_t>(t) & 1u;
-            const uint32_t acc_phase = (static_cast<uint32_t>(t) >> 1) & 1u;
+            const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
+            const uint32_t acc_phase = (static_cast<uint32_t>(t) / Cfg::ACC_BUFS) & 1u;
             // One lane waits; the verdict is broadcast so the warp stays
             // converged for the .sync.aligned TMEM loads below.
             uint32_t ready = 1;
@@ -472,25 +444,30 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             ready = __shfl_sync(0xffffffffu, ready, 0);
             if (!ready) break;
             tc_fence_after_sync();
-            const int row0 = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
+            const int row_base = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
             const int col0 = tn * Cfg::BN;
-            const uint32_t tbase = tmem_base + ((sub * 32u) << 16) + buf * Cfg::BN;
+            const uint32_t tbase0 = tmem_base + ((sub * 32u) << 16) + buf * Cfg::CONSUMERS * Cfg::BN;
+            // chunk q: consumer q / EPI_CHUNKS (its own rows and accumulator),
+            // columns (q % EPI_CHUNKS) * EPI_COLS of the tile
 #pragma unroll 1
-            for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
+            for (int q = 0; q < Cfg::CONSUMERS * Cfg::EPI_CHUNKS; ++q) {
+                const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
+                const int row0 = row_base + cons * Cfg::BM_MMA;
+                const uint32_t tbase = tbase0 + static_cast<uint32_t>(cons) * Cfg::BN;
                 uint32_t packed[32];
                 const int erow = row0 + static_cast<int>(lane);   // this thread's row of C
                 if constexpr (Cfg::OUT == 0) {
                     tmem_ld_32x32b_x32(tbase + c * 32, packed);
                     tmem_ld_wait();
-                    if (scaled) axpby_f32(packed, C, ldc, erow, col0 + c * 32, M, N, alpha, beta);
+                    if (fused) epilogue32_f32c(packed, C, ldc, erow, col0 + c * 32, M, N, epi);
                 } else {
                     uint32_t v0[32], v1[32];
                     tmem_ld_32x32b_x32(tbase + c * 64, v0);
                     tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
                     tmem_ld_wait();
-                    if (scaled) {
-                        axpby_bf16src(v0, C, ldc, erow, col0 + c * 64, M, N, alpha, beta);
-                        axpby_bf16src(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, alpha, beta);
+                    if (fused) {
+                        epilogue32_bf16c(v0, C, ldc, erow, col0 + c * 64, M, N, epi);
+                        epilogue32_bf16c(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, epi);
                     }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -498,7 +475,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
                     }
                 }
-                if (c == Cfg::EPI_CHUNKS - 1) {
+                if (q == Cfg::CONSUMERS * Cfg::EPI_CHUNKS - 1) {
                     // This warp has read its whole slice of accumulator `buf`.
                     tc_fence_before_sync();
                     __syncwarp();
@@ -590,18 +567,6 @@ __global__ void zero_fill_kernel(T *C, int64_t M, int64_t N, int64_t ldc) {
         const int64_t r = i / N;
         const int64_t c = i - r * N;
         C[r * ldc + c] = T(0);
-    }
-}
-
-// C = beta * C, one element per thread, grid-stride (K == 0 with beta != 0).
-template <typename T>
-__global__ void scale_kernel(T *C, int64_t M, int64_t N, int64_t ldc, float beta) {
-    const int64_t total = M * N;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = i / N;
-        const int64_t c = i - r * N;
-        C[r * ldc + c] = static_cast<T>(beta * static_cast<float>(C[r * ldc + c]));
     }
 }
 

@@ -24,6 +24,9 @@ OUT_F32 = 0
 OUT_BF16 = 1
 KMAJOR = 0      # A as M x K, B as N x K
 MNMAJOR = 1     # A as K x M, B as K x N (row-major K x N)
+ACT_NONE = 0
+ACT_RELU = 1
+ACT_GELU = 2
 
 CONFIGS = {
     "auto": 0,
@@ -35,12 +38,13 @@ CONFIGS = {
     "1cta_128x256_clc": 6,
     "mxfp8_1cta_128x256": 7,
     "mxfp8_2cta_256x256": 8,
+    "2cta_512x256_clc": 9,
 }
 
 STATUS_NAMES = {
     0: "GEMM_OK", 1: "GEMM_ERR_INVALID_VALUE", 2: "GEMM_ERR_MISALIGNED", 3: "GEMM_ERR_ALIAS",
     4: "GEMM_ERR_UNSUPPORTED_DEVICE", 5: "GEMM_ERR_LAUNCH", 6: "GEMM_ERR_TIMEOUT",
-    7: "GEMM_ERR_TOO_LARGE",
+    7: "GEMM_ERR_TOO_LARGE", 8: "GEMM_ERR_CAPTURE",
 }
 
 _i64 = ctypes.c_int64
@@ -54,6 +58,9 @@ lib.gemm_bf16_noalloc.restype = _int
 lib.gemm_bf16_ex.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int,
                              ctypes.c_float, ctypes.c_float, _vp]
 lib.gemm_bf16_ex.restype = _int
+lib.gemm_bf16_fused.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int,
+                                ctypes.c_float, ctypes.c_float, _vp, _int, _vp]
+lib.gemm_bf16_fused.restype = _int
 lib.gemm_mxfp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]
 lib.gemm_mxfp8.restype = _int
 lib.gemm_check_device_status.argtypes = [_vp]
@@ -127,6 +134,19 @@ def gemm_bf16_ex(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
     st = lib.gemm_bf16_ex(_ptr(A), _ptr(B), _ptr(C), M, N, K, lda, ldb, ldc, int(c_type), int(a_layout),
                           int(b_layout), float(alpha), float(beta), _stream(stream))
     return _check(st, "gemm_bf16_ex", check)
+
+
+def gemm_bf16_fused(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
+                    c_type: int = OUT_F32, a_layout: int = KMAJOR, b_layout: int = KMAJOR,
+                    alpha: float = 1.0, beta: float = 0.0, bias=None, act: int = ACT_NONE,
+                    stream=None, check: bool = True) -> int:
+    """C = act(alpha * A.B + beta * C + bias) with bias one fp32 value per
+    column of C, fused into the GEMM's write-back (see include/b200gemm.h,
+    gemm_bf16_fused)."""
+    st = lib.gemm_bf16_fused(_ptr(A), _ptr(B), _ptr(C), M, N, K, lda, ldb, ldc, int(c_type), int(a_layout),
+                             int(b_layout), float(alpha), float(beta), _ptr(bias) if bias is not None else None,
+                             int(act), _stream(stream))
+    return _check(st, "gemm_bf16_fused", check)
 
 
 def gemm_mxfp8(A, sfa, B, sfb, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,

@@ -21,14 +21,28 @@
  *   32 consecutive K elements (kb = k/32), rows packed (leading dim K/32).
  *
  * Ownership: every pointer is a DEVICE pointer owned by the caller, valid
- * until the work queued on `stream` has finished.  The library keeps one
- * small per-device status block (allocated on the first call on a device)
- * and caches per-device launch attributes; nothing else is retained.
+ * until the work queued on `stream` has finished.  The library keeps, per
+ * device, a small status block (allocated on the first call on a device),
+ * cached launch attributes and, for the skinny and block-scaled paths, a
+ * workspace that grows on demand.  A workspace that a larger one replaces
+ * is kept, never freed, while the library is loaded.
  *
  * Execution: calls are asynchronous on `stream` (0 = the legacy default
  * stream) and never synchronise, except gemm_check_device_status().
- * C is overwritten (no alpha/beta).  Results are deterministic for a given
- * shape and configuration (fixed per-element accumulation order).
+ * gemm_bf16 and gemm_mxfp8 overwrite C; gemm_bf16_ex and gemm_bf16_fused
+ * add alpha/beta, a bias and an activation.  Results are deterministic for
+ * a given shape and configuration (fixed per-element accumulation order).
+ *
+ * CUDA graphs: every call may be captured into a graph, whose replays then
+ * reuse the captured addresses ("GPU 执行模型", section "Launch、CUDA Graph
+ * 与动态 shape": fixed shapes and reusable input, output and workspace
+ * addresses).  One-time set-up cannot run inside a capture: the first call
+ * on a device, the first call of each kernel configuration and output
+ * type, and any workspace growth return GEMM_ERR_CAPTURE there, with
+ * nothing queued.  So make one call of the same shapes and types outside
+ * the capture first.  Because replaced workspaces are never freed, a graph
+ * captured before a workspace grew still replays on valid memory.
+ * gemm_check_device_status() synchronises and may not be captured.
  *
  * Errors: every function returns a status and never aborts or throws.
  * Argument checks run on the host before anything is queued.  A device-side
@@ -60,7 +74,8 @@ typedef enum {
     GEMM_ERR_UNSUPPORTED_DEVICE = 4,/* no device, or not compute capability 10.0 */
     GEMM_ERR_LAUNCH = 5,            /* a CUDA runtime call failed (see gemm_last_cuda_error) */
     GEMM_ERR_TIMEOUT = 6,           /* a kernel's bounded wait expired (device watchdog) */
-    GEMM_ERR_TOO_LARGE = 7          /* a dimension exceeds 2^31-1 (TMA coordinates are int32) */
+    GEMM_ERR_TOO_LARGE = 7,         /* a dimension exceeds 2^31-1 (TMA coordinates are int32) */
+    GEMM_ERR_CAPTURE = 8            /* one-time set-up requested inside a stream capture (below) */
 } gemm_status_t;
 
 typedef enum {
@@ -78,6 +93,13 @@ typedef enum {
     GEMM_LAYOUT_MNMAJOR = 1
 } gemm_layout_t;
 
+/* Pointwise activation of the fused epilogue (gemm_bf16_fused). */
+typedef enum {
+    GEMM_ACT_NONE = 0,
+    GEMM_ACT_RELU = 1,              /* x < 0 ? 0 : x  (NaN stays NaN) */
+    GEMM_ACT_GELU = 2               /* x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), erff in fp32 */
+} gemm_act_t;
+
 /* Kernel configurations.  GEMM_CFG_AUTO picks by shape; the others force a
  * configuration (for tests and benchmarks) through gemm_force_config(). */
 typedef enum {
@@ -93,7 +115,10 @@ typedef enum {
     GEMM_CFG_1CTA_128x256_CLC = 6,  /* as 1CTA_128x256 with Cluster Launch Control */
     GEMM_CFG_MXFP8_1CTA_128x256 = 7,/* gemm_mxfp8: one CTA per 128 x 256 tile */
     GEMM_CFG_MXFP8_2CTA_256x256 = 8,/* gemm_mxfp8: CTA pair per 256 x 256 tile, cta_group::2 */
-    GEMM_CFG_COUNT_ = 9
+    GEMM_CFG_2CTA_512x256_CLC = 9,  /* CTA pair per 512 x 256 tile, two MMA consumers sharing each
+                                       B k-tile, one TMEM accumulator each (TMEM single-buffered);
+                                       Cluster Launch Control; forced only */
+    GEMM_CFG_COUNT_ = 10
 } gemm_config_t;
 
 /*
@@ -136,6 +161,29 @@ B200GEMM_API gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C,
                                         float alpha, float beta, cudaStream_t stream);
 
 /*
+ * gemm_bf16_fused: C = act(alpha * A . B + beta * C + bias), the bias one
+ * fp32 value per column of C (bias[j] for every row), act a gemm_act_t.
+ * The pointwise steps run on the fp32 accumulator in registers inside the
+ * GEMM's write-back, in that order, before the single rounding to c_type:
+ * the unfused sequence would write the M x N intermediate to memory and
+ * read it back, two intermediate-sized transfers that fusion saves ("GPU
+ * 执行模型", section "Fusion 的收益与上限").
+ *   bias  device pointer to N floats, 16-byte aligned, or NULL (no bias);
+ *         it must not overlap C.  Read only, owned by the caller.
+ *   act   GEMM_ACT_NONE, GEMM_ACT_RELU or GEMM_ACT_GELU; anything else is
+ *         GEMM_ERR_INVALID_VALUE.
+ * K == 0 gives C = act(beta * C + bias).  Every other argument, rule and
+ * layout is gemm_bf16_ex's, which is gemm_bf16_fused with bias == NULL and
+ * act == GEMM_ACT_NONE.
+ */
+B200GEMM_API gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C,
+                                           int64_t M, int64_t N, int64_t K,
+                                           int64_t lda, int64_t ldb, int64_t ldc,
+                                           gemm_out_t c_type, gemm_layout_t a_layout, gemm_layout_t b_layout,
+                                           float alpha, float beta, const float *bias, gemm_act_t act,
+                                           cudaStream_t stream);
+
+/*
  * gemm_mxfp8: block-scaled C = (sa . A) . (sb . B) with FP8 E4M3 A and B and
  * one E8M0 scale per 32 consecutive K elements of every row of A and of the
  * K-major B -- the block-scaled MMA with its scale factors in tensor memory
@@ -156,9 +204,8 @@ B200GEMM_API gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C,
  * Each call queues two kernels: a repack of the scales into a per-device
  * workspace of 512 bytes per (128 rows x 128 K) block of A and of B, which
  * the library allocates on first use and grows when a larger problem needs
- * it (cudaMalloc; growing waits for the device to go idle), then the GEMM.
- * Calls on streams that are not ordered with each other share that
- * workspace and must not overlap.
+ * it (cudaMalloc), then the GEMM.  Calls on streams that are not ordered
+ * with each other share that workspace and must not overlap.
  */
 B200GEMM_API gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const uint8_t *sfb,
                                       void *C, int64_t M, int64_t N, int64_t K,

@@ -89,6 +89,19 @@ def test_ex_rejects_bad_layouts_and_pitches_before_any_launch():
     assert _call_ex(K=0, A_=0, B_=0, C_=C + 4) == 2
 
 
+def test_fused_rejects_bad_bias_and_activation_before_any_launch():
+    f = G.lib.gemm_bf16_fused
+    bias = 0x7F0000500000
+
+    def call(bias_=bias, act=G.ACT_GELU, C_=C, K=64):
+        return f(A, B, C_, 128, 96, K, 64, 64, 96, G.OUT_F32, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias_, act, 0)
+    assert call(act=3) == 1 and call(act=-1) == 1
+    assert call(bias_=bias + 4) == 2                 # bias not 16-byte aligned
+    assert call(bias_=C + 128 * 4) == 3              # bias inside C's first rows
+    assert call(K=0, bias_=bias + 8) == 2            # checked for K = 0 as well
+    assert f(A, B, C, 0, 96, 64, 64, 64, 96, 0, 0, 0, 1.0, 0.0, bias + 4, 1, 0) == 0   # empty: nothing checked
+
+
 def test_mxfp8_rejects_bad_arguments_before_any_launch():
     f = G.lib.gemm_mxfp8
     sa, sb = 0x7F0000300000, 0x7F0000400000
@@ -123,6 +136,10 @@ def test_status_strings_and_config_control():
     assert G.lib.gemm_force_config(99) == 1
     G.gemm_force_config("2cta_256x256")
     assert G.gemm_select_config(16, 16, 16) == G.CONFIGS["2cta_256x256"]
+    G.gemm_force_config("2cta_512x256_clc")
+    assert G.gemm_select_config(16, 16, 16) == G.CONFIGS["2cta_512x256_clc"]
+    G.gemm_force_config("mxfp8_2cta_256x256")          # a block-scaled choice leaves bf16 on auto
+    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]
     G.gemm_force_config("auto")
     assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]
     assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]

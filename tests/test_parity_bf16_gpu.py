@@ -21,7 +21,7 @@ from gpu_helpers import (assert_close, assert_exact, run_gemm, sample_indices)
 
 pytestmark = pytest.mark.gpu
 
-CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "1cta_128x256_clc", "2cta_256x256_clc"]
+CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "1cta_128x256_clc", "2cta_256x256_clc", "2cta_512x256_clc"]
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 
 
@@ -154,7 +154,7 @@ def test_square_8192_headline_launch():
     _big_check(8192, 8192, 8192, "uniform", workload=3)
 
 
-@pytest.mark.parametrize("cfg", ["2cta_256x256_clc", "1cta_128x256_clc"])
+@pytest.mark.parametrize("cfg", ["2cta_256x256_clc", "1cta_128x256_clc", "2cta_512x256_clc"])
 def test_square_8192_cluster_launch_control(cfg):
     """8192^3 with tiles handed out by Cluster Launch Control: 1024 (pair) or
     2048 (single) clusters launched, ~74 / 148 running at a time."""
