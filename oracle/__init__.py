@@ -290,7 +290,7 @@ def axpby(c_ab64: np.ndarray, c_old64: np.ndarray, alpha: float, beta: float) ->
     return c
 
 
-ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
+ACT_NONE, ACT_RELU, ACT_GELU, ACT_GELU_TANH = 0, 1, 2, 3
 
 
 def gelu(x: np.ndarray) -> np.ndarray:
@@ -298,6 +298,14 @@ def gelu(x: np.ndarray) -> np.ndarray:
     from math import erf, sqrt
     x = np.asarray(x, dtype=np.float64)
     return x * 0.5 * (1.0 + np.vectorize(erf, otypes=[np.float64])(x / sqrt(2.0)))
+
+
+def gelu_tanh(x: np.ndarray) -> np.ndarray:
+    """The tanh form of GELU, 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))),
+    in fp64 (Hendrycks and Gimpel, "Gaussian Error Linear Units", 2016)."""
+    from math import pi, sqrt
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(sqrt(2.0 / pi) * (x + 0.044715 * x ** 3)))
 
 
 def relu(x: np.ndarray) -> np.ndarray:
@@ -312,7 +320,7 @@ def epilogue(c_ab64: np.ndarray, c_old64: np.ndarray, alpha: float, beta: float,
     the bias one value per column of C.  Its arithmetic is the pointwise
     sequence that fusion folds into the GEMM's write-back ("GPU 执行模型",
     section "Fusion 的收益与上限"); which pointwise ops to offer (bias, ReLU,
-    GELU) is this library's choice."""
+    GELU and its tanh form) is this library's choice."""
     c = axpby(c_ab64, c_old64, alpha, beta)
     if bias64 is not None:
         c = c + np.asarray(bias64, dtype=np.float64)[None, :]
@@ -320,6 +328,8 @@ def epilogue(c_ab64: np.ndarray, c_old64: np.ndarray, alpha: float, beta: float,
         return relu(c)
     if act == ACT_GELU:
         return gelu(c)
+    if act == ACT_GELU_TANH:
+        return gelu_tanh(c)
     if act != ACT_NONE:
         raise ValueError(f"unknown activation {act}")
     return c

@@ -383,3 +383,19 @@ def test_epilogue_order_and_bias_broadcast():
 def test_fusion_saving_is_one_write_and_one_read():
     # an 8192 x 8192 fp32 intermediate: 268 MB out and 268 MB back in
     assert oracle.fusion_saving_bytes(8192 * 8192 * 4) == 536870912
+
+
+def test_gelu_tanh_form_closed_forms():
+    # tanh is odd, so the tanh form keeps GELU(x) - GELU(-x) = x
+    x = np.linspace(-6.0, 6.0, 121)
+    assert np.allclose(oracle.gelu_tanh(x) - oracle.gelu_tanh(-x), x, atol=1e-15, rtol=0)
+    # at x = 1: 0.5 (1 + tanh(sqrt(2/pi) * 1.044715))
+    assert oracle.gelu_tanh(np.array([1.0]))[0] == pytest.approx(0.8411919906082768, abs=1e-15)
+    # it tracks the erf form to within 4.8e-4, the largest gap (about 4.73e-4)
+    # lying near x = 2.7; a wrong cubic coefficient moves both
+    xs = np.linspace(-10.0, 10.0, 200001)
+    gap = np.abs(oracle.gelu_tanh(xs) - oracle.gelu(xs))
+    assert 4.6e-4 < gap.max() < 4.8e-4
+    assert 2.5 < abs(xs[gap.argmax()]) < 2.9
+    assert np.array_equal(oracle.epilogue(np.array([[1.0]]), None, 1.0, 0.0, None, oracle.ACT_GELU_TANH),
+                          oracle.gelu_tanh(np.array([[1.0]])))
