@@ -1,7 +1,8 @@
 """Benchmark: bf16 GEMM TFLOP/s at 8192^3 on B200 (C = A.B, bf16 in, fp32 accumulate and out).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload square8192|square4096|ragged|skinny1000|skinny16|mxfp8_8192|fused8192]
+                    [--workload square8192|square4096|ragged|skinny1000|skinny16|mxfp8_8192|fused8192
+                                |fused8192_tanh]
                     [--shape M N K] [--config auto|1cta_128x128|1cta_128x256|2cta_256x256]
 
 One step = one library call over the whole M x N x K problem with the inputs
@@ -50,7 +51,12 @@ WORKLOADS = {
                    "block-scaled gemm 8192^3, E4M3 U[-1,1], E8M0 per 32 (exp U{-4..4}), bf16 out"),
     "fused8192": (8192, 8192, 8192, "fused", "uniform", 3,
                   "gelu(A.B + bias) 8192^3, bf16 U[-1,1] in, bias N(0,1) fp32, fp32 accumulate, bf16 out"),
+    "fused8192_tanh": (8192, 8192, 8192, "fused", "uniform", 3,
+                       "gelu_tanh(A.B + bias) 8192^3 (tanh form of GELU), bf16 U[-1,1] in, bias N(0,1) fp32, "
+                       "fp32 accumulate, bf16 out"),
 }
+# activation of the fused workloads (gemm_bf16_fused's act)
+FUSED_ACT = {"fused8192": "gelu", "fused8192_tanh": "gelu_tanh"}
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -202,6 +208,7 @@ class Problem:
                     "fused": f"gelu(A.B + bias) {M}x{N}x{K}, bf16 U[-1,1] in, bf16 out",
                     "mxfp8": f"block-scaled gemm {M}x{N}x{K}, E4M3 U[-1,1], E8M0 per 32, bf16 out"}[kind]
         self.name, self.M, self.N, self.K, self.kind, self.desc = name, M, N, K, kind, desc
+        self.act = FUSED_ACT.get(name, "gelu")
         self.flops = 2.0 * M * N * K
         if kind == "bf16":
             self.a, self.b = synth.bf16_operands(M, N, K, dist, workload=wid, base=rank)
@@ -242,7 +249,7 @@ class Problem:
         elif self.kind == "fused":
             A, B, bias = dev
             G.gemm_bf16_fused(A, B, C, M, N, K, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias,
-                              G.ACT_GELU, stream=stream)
+                              act_code(G, self.act), stream=stream)
         else:
             A, SA, B, SB = dev
             G.gemm_mxfp8(A, SA, B, SB, C, M, N, K, K, K, N, stream=stream)
@@ -256,13 +263,18 @@ class Problem:
             return oracle.gemm_bf16_f64(self.a[:rows], self.b, K=self.K)
         if self.kind == "fused":
             c = oracle.gemm_bf16_f64(self.a[:rows], self.b, K=self.K)
-            return oracle.epilogue(c, None, 1.0, 0.0, self.bias.astype(np.float64), oracle.ACT_GELU)
+            return oracle.epilogue(c, None, 1.0, 0.0, self.bias.astype(np.float64),
+                                   {"gelu": oracle.ACT_GELU, "gelu_tanh": oracle.ACT_GELU_TANH}[self.act])
         return oracle.gemm_mxfp8_f64(self.a[:rows], self.sfa[:rows], self.b, self.sfb, K=self.K)
+
+
+def act_code(G, name: str) -> int:
+    return {"gelu": G.ACT_GELU, "gelu_tanh": G.ACT_GELU_TANH}[name]
 
 
 def fusion_comparison(p, G, dev, torch, stream, steps):
     """The unfused form of the fused workload, timed beside it: a plain GEMM
-    writing the bf16 intermediate, then a separate pass C = gelu(C + bias)
+    writing the bf16 intermediate, then a separate pass C = act(C + bias)
     that reads it back and writes it again.  Fusion saves that pass's two
     intermediate-sized transfers ("GPU 执行模型", section "Fusion 的收益与
     上限": about 2 x the intermediate's bytes).  The fused call, the plain
@@ -273,16 +285,18 @@ def fusion_comparison(p, G, dev, torch, stream, steps):
     C1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     C2 = torch.empty_like(C1)
 
+    act = act_code(G, p.act)
+
     def fused():
         G.gemm_bf16_fused(A, B, C1, M, N, K, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias,
-                          G.ACT_GELU, stream=stream)
+                          act, stream=stream)
 
     def gemm():
         G.gemm_bf16(A, B, C2, M, N, K, K, K, N, G.OUT_BF16, stream=stream)
 
     def pointwise():
         G.gemm_bf16_fused(A, B, C2, M, N, 0, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 1.0, bias,
-                          G.ACT_GELU, stream=stream)
+                          act, stream=stream)
 
     for _ in range(3):
         fused(), gemm(), pointwise()
@@ -413,6 +427,8 @@ def main():
             ("mxfp8_2cta_256x256" if pair_tiles >= 74 else "mxfp8_1cta_128x256")
     else:
         cfg_name = {v: k for k, v in G.CONFIGS.items()}[G.gemm_select_config(p.M, p.N, p.K)]
+        if p.kind == "fused" and args.config == "auto" and cfg_name == "2cta_512x256_clc":
+            cfg_name = "2cta_256x256_clc"   # the library's choice for a non-plain epilogue
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):

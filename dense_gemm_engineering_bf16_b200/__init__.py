@@ -13,7 +13,7 @@ _BINDING_NAMES = {
     "gemm_bf16", "gemm_bf16_ex", "gemm_bf16_fused", "gemm_bf16_noalloc", "gemm_mxfp8", "gemm_check_device_status", "gemm_status_string",
     "gemm_force_config", "gemm_select_config", "gemm_launches_per_call",
     "gemm_last_timeout_detail", "GemmError", "OUT_F32", "OUT_BF16", "KMAJOR", "MNMAJOR", "ACT_NONE", "ACT_RELU",
-    "ACT_GELU", "CONFIGS",
+    "ACT_GELU", "ACT_GELU_TANH", "CONFIGS",
     "STATUS_NAMES", "lib", "library_path",
 }
 

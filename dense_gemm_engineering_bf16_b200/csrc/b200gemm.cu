@@ -40,6 +40,12 @@ using Cfg2x512F32C = b200::GemmBf16Cfg<2, 256, 4, 0, true, 2>;
 using Cfg2x512B16C = b200::GemmBf16Cfg<2, 256, 4, 1, true, 2>;
 using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
+// A few rows of A leave most of a stage to B: narrower A parts buy more
+// stages (bytes in flight per SM) for the HBM-bound small-M shapes.
+using CfgSk16F32 = b200::GemmSkinnyCfg<16, 12, 0>;
+using CfgSk16B16 = b200::GemmSkinnyCfg<16, 12, 1>;
+using CfgSk32F32 = b200::GemmSkinnyCfg<32, 11, 0>;
+using CfgSk32B16 = b200::GemmSkinnyCfg<32, 11, 1>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
 using CfgSk64B16 = b200::GemmSkinnyCfg<64, 8, 1>;
 using CfgSk128F32 = b200::GemmSkinnyCfg<128, 6, 0>;
@@ -63,7 +69,7 @@ struct DeviceState {
     uint8_t *mx_ws = nullptr;
     size_t mx_ws_bytes = 0;
     // skinny path: kernel attributes (per template), split-tile workspace
-    bool sk_attr_done[6] = {};
+    bool sk_attr_done[10] = {};
     uint8_t *sk_ws = nullptr;
     size_t sk_ws_bytes = 0;
     uint32_t sk_epoch = 0;
@@ -241,6 +247,11 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     const int64_t wide_tiles = ((M + 127) / 128) * ((N + 255) / 256);
     // two or more waves of pair tiles: Cluster Launch Control evens out the
     // tail; a single wave: the static persistent schedule
+    // two or more waves of 512 x 256 tiles: two MMA consumers share each B
+    // k-tile (25% fewer operand bytes into shared memory per FLOP, which
+    // under the power cap buys clock); fewer: the double-buffered 256 x 256
+    const int64_t tall_tiles = ((M + 511) / 512) * ((N + 255) / 256);
+    if (tall_tiles >= 148) return GEMM_CFG_2CTA_512x256_CLC;
     if (pair_tiles >= 148) return GEMM_CFG_2CTA_256x256_CLC;
     if (pair_tiles >= 74) return GEMM_CFG_2CTA_256x256;
     // few rows, too few tiles to fill the SMs, and a long K to split: stream-K.
@@ -420,6 +431,12 @@ gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const 
                                 const b200::Epilogue &epi = b200::plain_epilogue(), uint32_t layout = 0) {
     // the skinny kernel reads A K-major only (A stored M x K)
     if (M > 256 || (layout & b200::kLayoutAMajorM)) return GEMM_ERR_INVALID_VALUE;
+    if (M <= 16)
+        return f32 ? launch_skinny<CfgSk16F32>(st, 6, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                   : launch_skinny<CfgSk16B16>(st, 7, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+    if (M <= 32)
+        return f32 ? launch_skinny<CfgSk32F32>(st, 8, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                   : launch_skinny<CfgSk32B16>(st, 9, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
     if (M <= 64)
         return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                    : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
@@ -662,7 +679,8 @@ gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C, int64_t M, 
                               gemm_layout_t b_layout, float alpha, float beta, const float *bias, gemm_act_t act,
                               cudaStream_t stream) {
     if (c_type != GEMM_OUT_F32 && c_type != GEMM_OUT_BF16) return GEMM_ERR_INVALID_VALUE;
-    if (act != GEMM_ACT_NONE && act != GEMM_ACT_RELU && act != GEMM_ACT_GELU) return GEMM_ERR_INVALID_VALUE;
+    if (act != GEMM_ACT_NONE && act != GEMM_ACT_RELU && act != GEMM_ACT_GELU && act != GEMM_ACT_GELU_TANH)
+        return GEMM_ERR_INVALID_VALUE;
     if ((a_layout != GEMM_LAYOUT_KMAJOR && a_layout != GEMM_LAYOUT_MNMAJOR) ||
         (b_layout != GEMM_LAYOUT_KMAJOR && b_layout != GEMM_LAYOUT_MNMAJOR))
         return GEMM_ERR_INVALID_VALUE;
@@ -691,6 +709,11 @@ gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C, int64_t M, 
     const uint32_t layout = (a_mn ? b200::kLayoutAMajorM : 0u) | (b_mn ? b200::kLayoutBMajorN : 0u);
     gemm_config_t cfg = select_config(M, N, K);
     if (cfg == GEMM_CFG_SKINNY && a_mn) cfg = GEMM_CFG_1CTA_128x128;   // skinny reads A K-major only
+    // The two-consumer tile holds one tile in TMEM, so its epilogue stalls
+    // the MMA; with epilogue work beyond the plain store (beta, bias, an
+    // activation) the double-buffered 256 x 256 tile hides it instead.
+    if (cfg == GEMM_CFG_2CTA_512x256_CLC && !epi.identity() && g_forced.load() == GEMM_CFG_AUTO)
+        cfg = GEMM_CFG_2CTA_256x256_CLC;
     return launch_dense(st, cfg, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
 }
 

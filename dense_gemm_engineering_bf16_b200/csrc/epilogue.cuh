@@ -9,7 +9,7 @@
 
 namespace b200 {
 
-enum : uint32_t { kActNone = 0, kActRelu = 1, kActGelu = 2, kActCount = 3 };
+enum : uint32_t { kActNone = 0, kActRelu = 1, kActGelu = 2, kActGeluTanh = 3, kActCount = 4 };
 
 struct Epilogue {
     float alpha;
@@ -24,9 +24,21 @@ struct Epilogue {
 
 __host__ __device__ inline Epilogue plain_epilogue() { return Epilogue{1.0f, 0.0f, nullptr, kActNone}; }
 
+// The hardware tanh approximation (PTX tanh.approx.f32, one MUFU op).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float activate(float x, uint32_t act) {
     if (act == kActRelu) return x < 0.0f ? 0.0f : x;                       // NaN passes through
     if (act == kActGelu) return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));   // x Phi(x)
+    if (act == kActGeluTanh) {
+        // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh form of GELU
+        const float u = 0.79788456080286536f * fmaf(0.044715f * x, x * x, x);
+        return 0.5f * x * (1.0f + tanh_approx(u));
+    }
     return x;
 }
 

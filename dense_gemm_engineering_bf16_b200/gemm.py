@@ -27,6 +27,7 @@ MNMAJOR = 1     # A as K x M, B as K x N (row-major K x N)
 ACT_NONE = 0
 ACT_RELU = 1
 ACT_GELU = 2
+ACT_GELU_TANH = 3
 
 CONFIGS = {
     "auto": 0,

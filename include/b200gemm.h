@@ -97,7 +97,10 @@ typedef enum {
 typedef enum {
     GEMM_ACT_NONE = 0,
     GEMM_ACT_RELU = 1,              /* x < 0 ? 0 : x  (NaN stays NaN) */
-    GEMM_ACT_GELU = 2               /* x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), erff in fp32 */
+    GEMM_ACT_GELU = 2,              /* x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), erff in fp32 */
+    GEMM_ACT_GELU_TANH = 3          /* 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh
+                                       form of GELU (within 4.8e-4 of GELU), with the hardware
+                                       tanh approximation (PTX tanh.approx.f32) */
 } gemm_act_t;
 
 /* Kernel configurations.  GEMM_CFG_AUTO picks by shape; the others force a
@@ -117,7 +120,8 @@ typedef enum {
     GEMM_CFG_MXFP8_2CTA_256x256 = 8,/* gemm_mxfp8: CTA pair per 256 x 256 tile, cta_group::2 */
     GEMM_CFG_2CTA_512x256_CLC = 9,  /* CTA pair per 512 x 256 tile, two MMA consumers sharing each
                                        B k-tile, one TMEM accumulator each (TMEM single-buffered);
-                                       Cluster Launch Control; forced only */
+                                       Cluster Launch Control; chosen when there are >= 148
+                                       such tiles (two waves), e.g. 8192 x 8192 */
     GEMM_CFG_COUNT_ = 10
 } gemm_config_t;
 
@@ -170,8 +174,8 @@ B200GEMM_API gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C,
  * 执行模型", section "Fusion 的收益与上限").
  *   bias  device pointer to N floats, 16-byte aligned, or NULL (no bias);
  *         it must not overlap C.  Read only, owned by the caller.
- *   act   GEMM_ACT_NONE, GEMM_ACT_RELU or GEMM_ACT_GELU; anything else is
- *         GEMM_ERR_INVALID_VALUE.
+ *   act   GEMM_ACT_NONE, GEMM_ACT_RELU, GEMM_ACT_GELU or GEMM_ACT_GELU_TANH;
+ *         anything else is GEMM_ERR_INVALID_VALUE.
  * K == 0 gives C = act(beta * C + bias).  Every other argument, rule and
  * layout is gemm_bf16_ex's, which is gemm_bf16_fused with bias == NULL and
  * act == GEMM_ACT_NONE.

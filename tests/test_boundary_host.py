@@ -95,7 +95,7 @@ def test_fused_rejects_bad_bias_and_activation_before_any_launch():
 
     def call(bias_=bias, act=G.ACT_GELU, C_=C, K=64):
         return f(A, B, C_, 128, 96, K, 64, 64, 96, G.OUT_F32, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias_, act, 0)
-    assert call(act=3) == 1 and call(act=-1) == 1
+    assert call(act=4) == 1 and call(act=-1) == 1
     assert call(bias_=bias + 4) == 2                 # bias not 16-byte aligned
     assert call(bias_=C + 128 * 4) == 3              # bias inside C's first rows
     assert call(K=0, bias_=bias + 8) == 2            # checked for K = 0 as well
@@ -139,9 +139,11 @@ def test_status_strings_and_config_control():
     G.gemm_force_config("2cta_512x256_clc")
     assert G.gemm_select_config(16, 16, 16) == G.CONFIGS["2cta_512x256_clc"]
     G.gemm_force_config("mxfp8_2cta_256x256")          # a block-scaled choice leaves bf16 on auto
-    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]
+    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]
     G.gemm_force_config("auto")
-    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]
+    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 512 tiles of 512 x 256
+    assert G.gemm_select_config(6144, 6144, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 288
+    assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_clc"]   # 8 x 16 = 128 < 148
     assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
     assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]

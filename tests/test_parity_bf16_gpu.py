@@ -149,8 +149,9 @@ def test_square_4096(c_type):
 
 
 def test_square_8192_headline_launch():
-    """8192^3, U[-1,1], fp32 out, the shape-selected (benchmark) configuration."""
-    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]
+    """8192^3, U[-1,1], fp32 out, the shape-selected (benchmark) configuration:
+    512 x 256 pair tiles, two MMA consumers, Cluster Launch Control."""
+    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]
     _big_check(8192, 8192, 8192, "uniform", workload=3)
 
 

@@ -14,7 +14,7 @@ from gpu_helpers import assert_exact, to_device_bf16
 pytestmark = pytest.mark.gpu
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc", "skinny"]
-ACTS = {"none": G.ACT_NONE, "relu": G.ACT_RELU, "gelu": G.ACT_GELU}
+ACTS = {"none": G.ACT_NONE, "relu": G.ACT_RELU, "gelu": G.ACT_GELU, "gelu_tanh": G.ACT_GELU_TANH}
 
 
 def _run(M, N, K, dist, workload, cfg, act, alpha=1.0, beta=0.0, c_type=F32, c_old=None, bias=None,
@@ -51,13 +51,17 @@ def _tolerance(want, s_abs, old, lin, alpha, beta, c_type, act):
     if act == G.ACT_GELU:
         # |GELU'| <= 1.13; fp32 erff and the products add a few ulp of |x|
         t = 1.13 * t + 1e-6 * np.abs(lin) + 1e-6
+    if act == G.ACT_GELU_TANH:
+        # the same slope bound; the hardware tanh is within 2^-10 of tanh,
+        # which 0.5 x scales to 2^-11 |x|
+        t = 1.13 * t + 2.0 ** -11 * np.abs(lin) + 1e-6
     if c_type == BF16:
         t = t + 2.0 ** -8 * np.abs(want)
     return t
 
 
 @pytest.mark.parametrize("cfg", CFGS)
-@pytest.mark.parametrize("act", ["relu", "gelu"])
+@pytest.mark.parametrize("act", ["relu", "gelu", "gelu_tanh"])
 @pytest.mark.parametrize("c_type", [F32, BF16])
 def test_bias_activation_random(cfg, act, c_type):
     M, N, K = (250 if cfg == "skinny" else 257), 300, 1000
@@ -92,7 +96,7 @@ def test_integer_bias_relu_bit_exact(cfg, c_type):
     assert_exact(got, want, c_type, f"{cfg} ints bias relu")
 
 
-@pytest.mark.parametrize("act", ["none", "relu", "gelu"])
+@pytest.mark.parametrize("act", ["none", "relu", "gelu", "gelu_tanh"])
 def test_k_zero_is_epilogue_of_zero(act):
     M, N = 40, 72
     c_old = synth.normal(36, (M, N)).astype(np.float32)
@@ -104,7 +108,9 @@ def test_k_zero_is_epilogue_of_zero(act):
     G.gemm_check_device_status()
     got = C.cpu().numpy().astype(np.float64)
     want = oracle.epilogue(np.zeros((M, N)), c_old.astype(np.float64), 2.0, 0.5, bias.astype(np.float64), ACTS[act])
-    assert np.all(np.abs(got - want) <= 1e-6 * np.abs(want) + 1e-6)
+    lin = 0.5 * c_old.astype(np.float64) + bias.astype(np.float64)[None, :]
+    tol = 1e-6 * np.abs(want) + 1e-6 + (2.0 ** -11 * np.abs(lin) if act == "gelu_tanh" else 0.0)
+    assert np.all(np.abs(got - want) <= tol)
 
 
 def test_activation_without_bias_and_identity_matches_plain():
