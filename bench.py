@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -72,11 +73,20 @@ KERNEL_SOURCES = {
 }
 
 
+def code_only(text: str) -> str:
+    """C++ source without comments and blank lines: an edit to a comment
+    leaves the compiled kernel, and so its ncu counters, as they were.
+    (The kernel sources hold no '//' or '/*' inside string literals.)"""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(kernel: str = "bf16") -> str:
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "dense_gemm_engineering_bf16_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "dense_gemm_engineering_bf16_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -331,12 +341,17 @@ def oracle_sample(problem: Problem, budget_s: float):
         problem.oracle_rows(rows)
         return time.perf_counter() - t0
 
-    # each call decodes all of B once, then spends a fixed time per row of A:
-    # two calibration points give both parts
-    t4, t16 = timed(4), timed(16)
-    per_row = max((t16 - t4) / 12.0, 1e-6)
-    fixed = max(t4 - 4 * per_row, 0.0)
-    R = int(max(4, min(problem.M, (budget_s - fixed) / per_row)))
+    # each call decodes all of B once, then its threads share the rows of A:
+    # time(r) ~ fixed + r * per_row once every thread has rows, so the two
+    # calibration points are one and three rows per thread
+    import oracle
+    t = max(1, oracle.num_threads())
+    t1, t3 = timed(min(problem.M, t)), timed(min(problem.M, 3 * t))
+    per_row = max((t3 - t1) / (2.0 * t), 1e-6)
+    fixed = max(t1 - t * per_row, 0.0)
+    R = int(max(1, min(problem.M, (budget_s - fixed) / per_row)))
+    if R > t:
+        R -= R % t                          # whole rounds of rows per thread
     dt = timed(R)
     return 2.0 * R * problem.N * problem.K, dt, R
 

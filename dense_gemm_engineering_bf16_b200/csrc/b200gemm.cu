@@ -40,12 +40,6 @@ using Cfg2x512F32C = b200::GemmBf16Cfg<2, 256, 4, 0, true, 2>;
 using Cfg2x512B16C = b200::GemmBf16Cfg<2, 256, 4, 1, true, 2>;
 using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
-// A few rows of A leave most of a stage to B: narrower A parts buy more
-// stages (bytes in flight per SM) for the HBM-bound small-M shapes.
-using CfgSk16F32 = b200::GemmSkinnyCfg<16, 12, 0>;
-using CfgSk16B16 = b200::GemmSkinnyCfg<16, 12, 1>;
-using CfgSk32F32 = b200::GemmSkinnyCfg<32, 11, 0>;
-using CfgSk32B16 = b200::GemmSkinnyCfg<32, 11, 1>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
 using CfgSk64B16 = b200::GemmSkinnyCfg<64, 8, 1>;
 using CfgSk128F32 = b200::GemmSkinnyCfg<128, 6, 0>;
@@ -69,7 +63,7 @@ struct DeviceState {
     uint8_t *mx_ws = nullptr;
     size_t mx_ws_bytes = 0;
     // skinny path: kernel attributes (per template), split-tile workspace
-    bool sk_attr_done[10] = {};
+    bool sk_attr_done[6] = {};
     uint8_t *sk_ws = nullptr;
     size_t sk_ws_bytes = 0;
     uint32_t sk_epoch = 0;
@@ -431,12 +425,6 @@ gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const 
                                 const b200::Epilogue &epi = b200::plain_epilogue(), uint32_t layout = 0) {
     // the skinny kernel reads A K-major only (A stored M x K)
     if (M > 256 || (layout & b200::kLayoutAMajorM)) return GEMM_ERR_INVALID_VALUE;
-    if (M <= 16)
-        return f32 ? launch_skinny<CfgSk16F32>(st, 6, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                   : launch_skinny<CfgSk16B16>(st, 7, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
-    if (M <= 32)
-        return f32 ? launch_skinny<CfgSk32F32>(st, 8, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                   : launch_skinny<CfgSk32B16>(st, 9, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
     if (M <= 64)
         return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                    : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);

@@ -7,20 +7,25 @@
 // tile schedule (step 6), warp specialisation into TMA producer / MMA issuer
 // / write-back (step 7) and, for CG == 2, a CTA pair running one
 // cta_group::2 MMA over both CTAs' shared memory with a 256-row tile (step 8).
+// With CONSUMERS == 2 a second MMA consumer stacks another 256 rows on the
+// same B k-tiles, a 512 x 256 pair tile (step 9): both accumulators fill
+// TMEM, so it holds one tile at a time instead of two.
 //
 // Per CTA (192 threads):
 //   warp 0      TMA producer: waits empty[s], loads the A and B k-tiles of
 //               stage s (128-byte swizzle), completion counted in bytes on
 //               the pair leader's full[s].
 //   warp 1      TMEM owner (alloc / dealloc) and, in the pair leader only, the
-//               MMA issuer: waits full[s], issues BK/16 tcgen05.mma into the
-//               TMEM accumulator, commits to empty[s] (both CTAs); after the
-//               last k-tile of a tile commits to tmem_full[b].
+//               MMA issuer: waits full[s], issues BK/16 tcgen05.mma per
+//               consumer into its TMEM accumulator, commits to empty[s] (both
+//               CTAs); after the last k-tile of a tile commits to
+//               tmem_full[b].
 //   warps 2-5   epilogue: waits tmem_full[b], tcgen05.ld 32 rows x 32 columns
 //               per warp, converts, writes a swizzled staging buffer, and TMA-
 //               stores it; releases tmem_empty[b] (pair leader's barrier)
-//               once the accumulator is read, so tile i+1's main loop runs
-//               while tile i drains (TMEM double buffer, 2 x BN columns).
+//               once the accumulators are read.  With one consumer TMEM holds
+//               two tiles (2 x BN columns), so tile i+1's main loop runs while
+//               tile i drains; with two, the drain is the MMA's only stall.
 //
 //   warp 6      (CLC builds only) scheduler, in the pair leader: claims tiles
 //               of clusters that have not started with

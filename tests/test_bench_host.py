@@ -102,3 +102,14 @@ def test_reference_arm_prints_one_line_on_rank0():
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_kernel_hash_ignores_comments_only():
+    import bench
+    a = "int f() { return 1; }  // one\n/* block\n comment */\nint g;\n"
+    b = "// header\nint f() { return 1; }\n\n\nint g;   /* trailing */\n"
+    c = "int f() { return 2; }\nint g;\n"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(c)
+    for kernel in bench.KERNEL_SOURCES:
+        assert len(bench.kernel_source_hash(kernel)) == 16
