@@ -39,6 +39,10 @@
 
 namespace b200 {
 
+// Watchdog codes of the scale copier (role) and the scale-slot barriers.
+constexpr int kRoleSfCopy = 5;
+constexpr int kBarSfFull = 8, kBarSfEmpty = 9;
+
 template <int CG_, int STAGES_>
 struct GemmMxf8Cfg {
     static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
@@ -58,14 +62,22 @@ struct GemmMxf8Cfg {
     static constexpr int CTA_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int TX_BYTES = CTA_BYTES * CG;  // bytes landing on the leader's full[s]
     static constexpr int STAGE_BYTES = ((CTA_BYTES + 1023) / 1024) * 1024;
-    static constexpr int EPI_COLS = 64;            // accumulator columns drained per step
-    static constexpr int EPI_CHUNKS = BN / EPI_COLS;
-    static constexpr int NUM_BARS = 2 * STAGES + 2;
+    static constexpr int EPI_COLS = BN / 2;        // accumulator columns one epilogue warp drains
+    // Scale slots in TMEM (32 columns each, beside the accumulator): a
+    // separate warp copies stage s's scales into slot s % SF_SLOTS ahead of
+    // the MMAs that read them.
+    static constexpr int SF_SLOTS = 4;
+    // full[S], empty[S], tmem_full, tmem_empty, sf_full[SF_SLOTS], sf_empty[SF_SLOTS]
+    static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 * SF_SLOTS;
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL0 = 256;
-    static constexpr int THREADS = 192;
+    // warp 0 producer, warp 1 MMA, warps 2-9 epilogue (two per TMEM lane
+    // quarter, each draining half of the columns), warp 10 scale copier
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int THREADS = 32 * (3 + EPI_WARPS);
+    static_assert(SF_COL0 + 32 * SF_SLOTS <= TMEM_COLS, "scale slots fit beside the accumulator");
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
     static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows");
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
@@ -162,6 +174,8 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     auto empty_bar = [&](uint32_t s) { return bar0 + 8u * (Cfg::STAGES + s); };
     const uint32_t tfull_bar = bar0 + 8u * (2 * Cfg::STAGES);
     const uint32_t tempty_bar = tfull_bar + 8u;
+    auto sf_full = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + i); };
+    auto sf_empty = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + Cfg::SF_SLOTS + i); };
     const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
     const uint32_t abort_slot = tmem_slot + 4u;
     volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
@@ -173,7 +187,11 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
-        mbar_init(tempty_bar, 4 * CG);
+        mbar_init(tempty_bar, Cfg::EPI_WARPS * CG);
+        for (int i = 0; i < Cfg::SF_SLOTS; ++i) {
+            mbar_init(sf_full(i), 1);
+            mbar_init(sf_empty(i), 1);
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -253,9 +271,9 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         }
         __syncwarp();
     } else if (warp == 1) {
-        // -------------------------- scale copy + MMA issuer (pair leader) --
+        // ------------------------------------------ MMA issuer (pair leader) --
         if (rank == 0 && lane == 0) {
-            uint32_t stage = 0, phase = 0, sf_slot = 0;
+            uint32_t stage = 0, phase = 0, n = 0;
             bool ok = true;
             int t = 0;
             for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters, ++t) {
@@ -274,21 +292,15 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                     tc_fence_after_sync();
                     const uint32_t a0 = base + stage * Cfg::STAGE_BYTES;
                     const uint32_t b0 = a0 + Cfg::A_BYTES;
-                    const uint32_t sfa_smem = b0 + Cfg::B_BYTES;
-                    const uint32_t sfb_smem = sfa_smem + Cfg::SFA_BYTES;
-                    const uint32_t sfa_t = tmem_base + Cfg::SF_COL0 + 32u * sf_slot;
-                    const uint32_t sfb_t = sfa_t + 16u;
-                    // tcgen05.cp and tcgen05.mma issued by one thread execute in
-                    // issue order, so the MMAs below see these scales.
-                    if constexpr (CG == 1) {
-                        tmem_cp_32x128b_warpx4(sfa_t, rows16_desc(sfa_smem));
-                        tmem_cp_32x128b_warpx4(sfb_t, rows16_desc(sfb_smem));
-                        tmem_cp_32x128b_warpx4(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
-                    } else {
-                        tmem_cp_32x128b_warpx4_pair(sfa_t, rows16_desc(sfa_smem));
-                        tmem_cp_32x128b_warpx4_pair(sfb_t, rows16_desc(sfb_smem));
-                        tmem_cp_32x128b_warpx4_pair(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+                    const uint32_t slot = n % Cfg::SF_SLOTS;
+                    if (!mbar_wait(sf_full(slot), (n / Cfg::SF_SLOTS) & 1u, abort_flag, timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarSfFull);
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after_sync();
+                    const uint32_t sfa_t = tmem_base + Cfg::SF_COL0 + 32u * slot;
+                    const uint32_t sfb_t = sfa_t + 16u;
 #pragma unroll
                     for (int j = 0; j < Cfg::MMAS; ++j) {
                         const uint32_t idesc = idesc_mxf8_e8m0(Cfg::BM, Cfg::BN, static_cast<uint32_t>(j),
@@ -300,7 +312,8 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                         else mma_mxf8_ss_pair(tmem_base, ad, bd, idesc, sfa_t, sfb_t, acc);
                     }
                     mma_commit<CG>(empty_bar(stage), 0x3);
-                    sf_slot ^= 1u;
+                    mma_commit<CG>(sf_empty(slot), 0x1);      // the slot's scales are read
+                    ++n;
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -308,13 +321,66 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             }
         }
         __syncwarp();
+    } else if (warp == 2 + Cfg::EPI_WARPS) {
+        // ---------------------------------- scale copier (pair leader) --
+        // tcgen05.cp issued by the MMA thread would run in its issue order,
+        // between the MMAs; from this warp the copy of stage s + 1 (or later)
+        // is ordered only by the sf_full / sf_empty barriers, so it can run
+        // while stage s's MMAs execute.
+        if (rank == 0 && lane == 0) {
+            uint32_t stage = 0, phase = 0, n = 0;
+            bool ok = true;
+            for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
+                for (int kb = 0; kb < num_kb; ++kb, ++n) {
+                    const uint32_t slot = n % Cfg::SF_SLOTS;
+                    if (!mbar_wait(sf_empty(slot), ((n / Cfg::SF_SLOTS) & 1u) ^ 1u, abort_flag, 2 * timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleSfCopy * 16 + kBarSfEmpty);
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, 2 * timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, CG, kRoleSfCopy * 16 + kBarFull);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t sfa_smem = base + stage * Cfg::STAGE_BYTES + Cfg::A_BYTES + Cfg::B_BYTES;
+                    const uint32_t sfb_smem = sfa_smem + Cfg::SFA_BYTES;
+                    const uint32_t sfa_t = tmem_base + Cfg::SF_COL0 + 32u * slot;
+                    const uint32_t sfb_t = sfa_t + 16u;
+                    if constexpr (CG == 1) {
+                        tmem_cp_32x128b_warpx4(sfa_t, rows16_desc(sfa_smem));
+                        tmem_cp_32x128b_warpx4(sfb_t, rows16_desc(sfb_smem));
+                        tmem_cp_32x128b_warpx4(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+                    } else {
+                        tmem_cp_32x128b_warpx4_pair(sfa_t, rows16_desc(sfa_smem));
+                        tmem_cp_32x128b_warpx4_pair(sfb_t, rows16_desc(sfb_smem));
+                        tmem_cp_32x128b_warpx4_pair(sfb_t + 4u, rows16_desc(sfb_smem + Cfg::SF_CHUNK));
+                    }
+                    mma_commit<CG>(sf_full(slot), 0x1);
+                    if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // Tail: the MMA's last releases must land before this CTA exits.
+            for (int i = 0; ok && i < Cfg::SF_SLOTS; ++i, ++n) {
+                if (!mbar_wait(sf_empty(n % Cfg::SF_SLOTS), ((n / Cfg::SF_SLOTS) & 1u) ^ 1u, abort_flag,
+                               2 * timeout_ns)) {
+                    record_timeout(status, abort_flag, abort_slot, CG, kRoleSfCopy * 16 + kBarTail);
+                    ok = false;
+                }
+            }
+        }
+        __syncwarp();
     } else {
         // ----------------------------------------------------- epilogue --
         // TMEM -> registers -> bf16 -> global, 16-byte stores: thread `lane`
-        // of warp `sub` owns row 32*sub + lane of this CTA's 128 rows.  No
-        // shared-memory staging, so the whole SMEM budget goes to the operand
-        // ring; TMEM is handed back once the last columns are in registers.
+        // of warp `sub` owns row 32*sub + lane of this CTA's 128 rows, and
+        // each of the two warps on a lane quarter owns half of the columns.
+        // The accumulator is single-buffered, so the next tile's MMAs wait for
+        // this drain: a warp reads its whole share into registers (as packed
+        // bf16, 64 words a thread), hands TMEM back, and only then stores.
         const uint32_t sub = warp & 3u;
+        const int half = static_cast<int>(warp - 2) >> 2;
         int t = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++t) {
             int tm, tn;
@@ -327,44 +393,39 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             ready = __shfl_sync(0xffffffffu, ready, 0);
             if (!ready) break;
             tc_fence_after_sync();
-            const uint32_t tbase = tmem_base + ((sub * 32u) << 16);
+            const uint32_t tbase = tmem_base + ((sub * 32u) << 16) + static_cast<uint32_t>(half * Cfg::EPI_COLS);
             const int row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32 +
                             static_cast<int>(lane);
-            const int col0 = tn * Cfg::BN;
+            const int col0 = tn * Cfg::BN + half * Cfg::EPI_COLS;
             uint16_t *crow = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * 2);
-#pragma unroll 1
-            for (int c = 0; c < Cfg::EPI_CHUNKS; ++c) {
-                uint32_t v0[32], v1[32], packed[32];
-                tmem_ld_32x32b_x32(tbase + c * Cfg::EPI_COLS, v0);
-                tmem_ld_32x32b_x32(tbase + c * Cfg::EPI_COLS + 32, v1);
+            uint32_t packed[Cfg::EPI_COLS / 2];
+#pragma unroll
+            for (int g = 0; g < Cfg::EPI_COLS / 32; ++g) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tbase + g * 32, v);
                 tmem_ld_wait();
-                if (c == Cfg::EPI_CHUNKS - 1) {
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (CG == 1) mbar_arrive_local(tempty_bar);
-                        else mbar_arrive_cluster(map_to_cta(tempty_bar, 0));
-                    }
-                }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
-                    packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
-                }
-                const int cstart = col0 + c * Cfg::EPI_COLS;
-                if (row >= M || cstart >= N) continue;
+                for (int i = 0; i < 16; ++i)
+                    packed[16 * g + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 1) mbar_arrive_local(tempty_bar);
+                else mbar_arrive_cluster(map_to_cta(tempty_bar, 0));
+            }
+            if (row >= M) continue;
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {                 // 8 bf16 = 16 bytes per store
-                    const int col = cstart + 8 * v;
-                    if (col + 8 <= N) {
-                        *reinterpret_cast<uint4 *>(crow + col) =
-                            make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                    } else {
+            for (int v = 0; v < Cfg::EPI_COLS / 8; ++v) {    // 8 bf16 = 16 bytes per store
+                const int col = col0 + 8 * v;
+                if (col >= N) break;
+                if (col + 8 <= N) {
+                    *reinterpret_cast<uint4 *>(crow + col) =
+                        make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            if (col + e < N)
-                                crow[col + e] = static_cast<uint16_t>(packed[4 * v + (e >> 1)] >> (16 * (e & 1)));
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        if (col + e < N) crow[col + e] = static_cast<uint16_t>(packed[4 * v + (e >> 1)] >> (16 * (e & 1)));
                 }
             }
         }

@@ -152,3 +152,17 @@ def test_status_strings_and_config_control():
     assert G.gemm_select_config(300, 1000, 64) == G.CONFIGS["1cta_128x128"]
     with pytest.raises(G.GemmError):
         G.gemm_bf16(A, B, C, -1, 1, 1, 1, 1, 1, stream=0)
+
+
+def test_binding_constants_match_the_header():
+    text = "".join(open(h).read() for h in HEADERS)
+    enum = {name.upper(): int(v) for name, v in re.findall(r"\b(GEMM_[A-Z0-9_x]+)\s*=\s*(\d+)", text)}
+    for name, v in G.CONFIGS.items():
+        assert enum["GEMM_CFG_" + name.upper()] == v, name
+    assert enum["GEMM_CFG_COUNT_"] == max(G.CONFIGS.values()) + 1
+    for name in ("NONE", "RELU", "GELU", "GELU_TANH"):
+        assert enum["GEMM_ACT_" + name] == getattr(G, "ACT_" + name)
+    assert (enum["GEMM_LAYOUT_KMAJOR"], enum["GEMM_LAYOUT_MNMAJOR"]) == (G.KMAJOR, G.MNMAJOR)
+    assert (enum["GEMM_OUT_F32"], enum["GEMM_OUT_BF16"]) == (G.OUT_F32, G.OUT_BF16)
+    for code, name in G.STATUS_NAMES.items():
+        assert enum[name] == code

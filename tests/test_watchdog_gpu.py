@@ -30,7 +30,7 @@ CHILD = textwrap.dedent(r"""
     A, B = to_device_bf16(a), to_device_bf16(b)
     C = torch.zeros((M, N), dtype=torch.float32, device="cuda")
     ref, s = oracle.gemm_bf16_f64(a, b, with_abs=True)
-    for cfg in ("1cta_128x128", "2cta_256x256", "2cta_256x256_clc"):
+    for cfg in ("1cta_128x128", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc"):
         G.gemm_force_config(cfg)
         os.environ["B200GEMM_INJECT_TIMEOUT"] = "1"
         t0 = time.time()
