@@ -164,18 +164,28 @@ constexpr uint32_t kLayoutBMajorN = 2u;   // B stored K x N: b(k,j) at B[k*ldb +
 // One k-tile of an operand into shared memory.  K-major: one box of 64 (K)
 // x rows.  MN-major: rows / 64 boxes of 64 (MN) x 64 (K), 8 KB apart (the
 // layout sw128_mnmajor_desc describes).  Completion counts on `bar`.
-template <int CG>
+// HINT: the loads carry the L2 policy `policy` (else the default policy).
+template <int CG, bool HINT = false>
+__device__ __forceinline__ void load_one_box(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y,
+                                             uint64_t policy) {
+    if constexpr (HINT) {
+        if constexpr (CG == 1) tma_load_2d_hint(dst, map, bar, x, y, policy);
+        else tma_load_2d_pair_hint(dst, map, bar, x, y, policy);
+    } else {
+        (void)policy;
+        if constexpr (CG == 1) tma_load_2d(dst, map, bar, x, y);
+        else tma_load_2d_pair(dst, map, bar, x, y);
+    }
+}
+
+template <int CG, bool HINT = false>
 __device__ __forceinline__ void load_operand_tile(uint32_t dst, const CUtensorMap *map, uint32_t bar, int kx,
-                                                  int row, int rows, bool mn) {
+                                                  int row, int rows, bool mn, uint64_t policy = 0) {
     if (!mn) {
-        if constexpr (CG == 1) tma_load_2d(dst, map, bar, kx, row);
-        else tma_load_2d_pair(dst, map, bar, kx, row);
+        load_one_box<CG, HINT>(dst, map, bar, kx, row, policy);
         return;
     }
-    for (int h = 0; h < rows / 64; ++h) {
-        if constexpr (CG == 1) tma_load_2d(dst + 8192u * h, map, bar, row + 64 * h, kx);
-        else tma_load_2d_pair(dst + 8192u * h, map, bar, row + 64 * h, kx);
-    }
+    for (int h = 0; h < rows / 64; ++h) load_one_box<CG, HINT>(dst + 8192u * h, map, bar, row + 64 * h, kx, policy);
 }
 
 // Descriptor of K step kk (16 elements) of an operand tile at `base`.
@@ -292,6 +302,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             const uint32_t leader_rank = 0;
             uint32_t fetched = 0;
+
             for (int tile = cluster_id; ok && tile >= 0;) {
                 int tm, tn;
                 raster_tile(tile, num_m, num_n, group_m, tm, tn);
