@@ -67,10 +67,6 @@ struct DeviceState {
     uint8_t *sk_ws = nullptr;
     size_t sk_ws_bytes = 0;
     uint32_t sk_epoch = 0;
-    // split-tail parts of the square kernels: partial tiles and counters
-    uint8_t *st_ws = nullptr;
-    size_t st_ws_bytes = 0;
-    uint32_t st_epoch = 0;
     // Workspaces replaced by larger ones.  They are kept, not freed: a CUDA
     // graph captured earlier still holds their addresses.
     std::vector<void *> retired;
@@ -261,74 +257,11 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     return GEMM_CFG_1CTA_128x128;
 }
 
-// The split tail is off by default: measured on one B200 it made 4096^3,
-// 4000 x 3000 x 2000 and 1000 x 8192 x 8192 slower (153 / 275 / 311 us
-// against 118 / 53 / 117 us), because the last part's fix-up reads the other
-// parts' fp32 tiles back with little memory-level parallelism.  B200GEMM_SPLIT
-// turns it on: "auto" lets split_factor choose, 2..8 forces that factor.
-// Returns 1 (off), 0 (auto) or the forced factor.
-int split_override() {
-    static const int v = [] {
-        const char *s = std::getenv("B200GEMM_SPLIT");
-        if (!s) return 1;
-        if (std::strcmp(s, "auto") == 0) return 0;
-        const int x = std::atoi(s);
-        return (x >= 1 && x <= 8) ? x : 1;
-    }();
-    return v;
-}
-
-// Tail split for `tiles` tiles on `P` resident clusters: num_full = P *
-// floor(tiles / P) run whole, the rest in s parts each.  s minimises the
-// last wave's length in tile units, ceil(tail * s / P) / s, plus an
-// allowance of 0.05 + 0.02 s for writing and summing the parts; 1 (no split)
-// when nothing is gained.  Every part keeps at least one K block.
-int split_factor(int64_t tiles, int64_t P, int64_t num_kb, int64_t &num_full) {
-    num_full = P > 0 ? (tiles / P) * P : tiles;
-    const int64_t tail = tiles - num_full;
-    if (tail <= 0) return 1;
-    const int force = split_override();
-    if (force == 1) return 1;
-    if (force > 1) return static_cast<int>(force <= num_kb ? force : 1);
-    int best = 1;
-    double best_cost = 1.0;
-    for (int sf = 2; sf <= 8 && sf <= num_kb; ++sf) {
-        const double cost = static_cast<double>((tail * sf + P - 1) / P) / sf + 0.05 + 0.02 * sf;
-        if (cost < best_cost - 1e-9) {
-            best = sf;
-            best_cost = cost;
-        }
-    }
-    return best;
-}
-
-// Grows the split-tail workspace on demand (counters start at zero).  Like
-// the other workspaces it is refused inside a stream capture and retired,
-// not freed, when a larger one replaces it.
-gemm_status_t split_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStream_t stream) {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (st->st_ws_bytes < bytes) {
-        if (capturing(stream)) return GEMM_ERR_CAPTURE;
-        cudaError_t e;
-        if (st->st_ws) {
-            st->retired.push_back(st->st_ws);
-            st->st_ws = nullptr;
-            st->st_ws_bytes = 0;
-        }
-        const size_t want = bytes < (size_t(8) << 20) ? (size_t(8) << 20) : bytes;
-        if ((e = cudaMalloc(&st->st_ws, want)) != cudaSuccess) return cuda_fail(e);
-        if ((e = cudaMemset(st->st_ws, 0, want)) != cudaSuccess) return cuda_fail(e);
-        st->st_ws_bytes = want;
-    }
-    ws = st->st_ws;
-    return GEMM_OK;
-}
-
 template <class Cfg>
 gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, const void *B, void *C,
                           int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                           cudaStream_t stream, const b200::Epilogue &epi = b200::plain_epilogue(),
-                          uint32_t layout = 0, bool allow_split = true) {
+                          uint32_t layout = 0) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
     cudaError_t e;
@@ -385,40 +318,14 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
         return s;
 
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
-    // Split tail (one-consumer tiles; not for the allocation-free entry)
-    b200::SplitTail sp{static_cast<int>(tiles), 1, 0u, nullptr, nullptr};
-    int64_t items = tiles;
-    if (allow_split && Cfg::CONSUMERS == 1) {
-        int64_t num_full = tiles;
-        const int64_t num_kb = (K + Cfg::BK - 1) / Cfg::BK;
-        const int split = split_factor(tiles, st->max_clusters[cfg_id][oi], num_kb, num_full);
-        if (split > 1) {
-            const int64_t tail = tiles - num_full;
-            const size_t part_bytes = size_t(Cfg::CG) * Cfg::CONSUMERS * Cfg::BM_CTA * Cfg::BN * 4;
-            const size_t partial_bytes = size_t(tail) * split * part_bytes;
-            uint8_t *ws = nullptr;
-            gemm_status_t ws_s = split_workspace(st, partial_bytes + size_t(tail) * Cfg::CG * 8, ws, stream);
-            if (ws_s != GEMM_OK) return ws_s;
-            uint32_t epoch;
-            {
-                std::lock_guard<std::mutex> lock(g_mutex);
-                epoch = ++st->st_epoch;
-                if (epoch == 0) epoch = ++st->st_epoch;
-            }
-            sp = b200::SplitTail{static_cast<int>(num_full), split, epoch, reinterpret_cast<float *>(ws),
-                                 reinterpret_cast<unsigned long long *>(ws + partial_bytes)};
-            items = num_full + tail * split;
-        }
-    }
     // Static schedule: as many clusters as fit at once, each striding over
-    // the work items.  CLC: one cluster per item; running clusters claim the
-    // rest.
-    const int64_t clusters = Cfg::CLC ? items
-                                      : (items < st->max_clusters[cfg_id][oi] ? items : st->max_clusters[cfg_id][oi]);
+    // the tiles.  CLC: one cluster per tile; running clusters claim the rest.
+    const int64_t clusters = Cfg::CLC ? tiles
+                                      : (tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi]);
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
                            static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
-                           watchdog_ns(K), inject_flags(), epi, layout, sp);
+                           watchdog_ns(K), inject_flags(), epi, layout);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -554,28 +461,28 @@ gemm_status_t launch_zero(void *C, int64_t M, int64_t N, int64_t ldc, int sm_cou
 // The dense bf16 kernels, by configuration.
 gemm_status_t launch_dense(DeviceState *st, gemm_config_t cfg, bool f32, const void *A, const void *B, void *C,
                            int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                           cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout, bool allow_split = true) {
+                           cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout) {
     switch (cfg) {
         case GEMM_CFG_1CTA_128x256:
-            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split)
-                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split);
+            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_1CTA_128x128:
-            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split)
-                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split);
+            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_256x256:
-            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split)
-                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split);
+            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_SKINNY:
             return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_256x256_CLC:
-            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split)
-                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split);
+            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_512x256_CLC:
-            return f32 ? launch_bf16<Cfg2x512F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split)
-                       : launch_bf16<Cfg2x512B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split);
+            return f32 ? launch_bf16<Cfg2x512F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x512B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_1CTA_128x256_CLC:
-            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split)
-                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, allow_split);
+            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         default:
             return GEMM_ERR_INVALID_VALUE;
     }
@@ -910,7 +817,7 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
     gemm_config_t cfg = select_config(M, N, K);
     if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128;
     return launch_dense(st, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc, stream,
-                        b200::plain_epilogue(), 0u, /*allow_split=*/false);
+                        b200::plain_epilogue(), 0u);
 }
 
 }  // extern "C"

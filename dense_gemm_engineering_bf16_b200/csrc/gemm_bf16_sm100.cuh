@@ -73,7 +73,7 @@ constexpr uint32_t kInjectDropFirstStage = 1u;
 
 enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleScheduler = 4 };
 enum : int { kBarFull = 1, kBarEmpty = 2, kBarTmemFull = 3, kBarTmemEmpty = 4, kBarTail = 5, kBarSched = 6,
-             kBarClc = 7, kBarSplit = 10 };
+             kBarClc = 7 };
 
 __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     int p = lo;
@@ -109,10 +109,8 @@ struct GemmBf16Cfg {
     static constexpr int EPI_BUF = 32 * 128;       // one warp's 32 rows x 128 bytes
     static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
     static constexpr int TMEM_COLS = pow2_at_least(ACC_BUFS * CONSUMERS * BN, 32);
-    // full[S], empty[S], tmem_full[2], tmem_empty[2] (+ clc[2], sched_full[2], sched_empty[2]),
-    // split_stored, split_decided (split-tail parts)
-    static constexpr int SPLIT_BAR0 = 2 * STAGES + 4 + (CLC ? 6 : 0);
-    static constexpr int NUM_BARS = SPLIT_BAR0 + 2;
+    // full[S], empty[S], tmem_full[2], tmem_empty[2] (+ clc[2], sched_full[2], sched_empty[2])
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + (CLC ? 6 : 0);
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
     // after the barriers: TMEM address, abort flag, 2 tile ids, 2 CLC answers
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 64;
@@ -195,38 +193,6 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk, bool mn)
     return mn ? sw128_mnmajor_desc(base + 2048u * kk) : sw128_kmajor_desc(base + 32u * kk);
 }
 
-// Split tail ("stream-K" for the last wave): with T tiles on P resident
-// clusters, the first num_full = P * floor(T / P) tiles run whole and each
-// of the remaining T - num_full is cut into `split` K ranges, so the last
-// wave is split ways shorter instead of leaving clusters idle.  Work item i
-// < num_full is tile i; item num_full + j is part j % split of tile
-// num_full + j / split.  A part writes its fp32 accumulator to `partials`;
-// the last of a tile's parts to arrive (per CTA of the pair) sums the parts
-// in part order -- the same order whoever arrives last -- and writes C.
-// Arrival counters are 64-bit, (epoch << 32) | arrivals, as in the skinny
-// path: a new epoch per call restarts a count an aborted call left behind,
-// and the last part returns the count to zero for graph replays.
-struct SplitTail {
-    int num_full;
-    int split;                   // 1: no split
-    uint32_t epoch;
-    float *partials;             // [tail tiles][split][CG][CONSUMERS][128][BN]
-    unsigned long long *counters;  // [tail tiles][CG]
-};
-
-struct WorkItem {
-    int tile;
-    int kb0, kb1;                // K blocks [kb0, kb1)
-    int part;                    // -1: the whole tile
-};
-
-__device__ __forceinline__ WorkItem decode_item(int i, const SplitTail &sp, int num_kb) {
-    if (sp.split <= 1 || i < sp.num_full) return WorkItem{i, 0, num_kb, -1};
-    const int j = i - sp.num_full;
-    const int p = j % sp.split;
-    return WorkItem{sp.num_full + j / sp.split, p * num_kb / sp.split, (p + 1) * num_kb / sp.split, p};
-}
-
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -234,7 +200,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmC,
                        int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m,
                        DeviceStatus *status, uint64_t timeout_ns, uint32_t inject,
-                       Epilogue epi, uint32_t layout, SplitTail sp) {
+                       Epilogue epi, uint32_t layout) {
     constexpr int CG = Cfg::CG;
     const bool a_mn = (layout & kLayoutAMajorM) != 0;   // A stored K x M
     const bool b_mn = (layout & kLayoutBMajorN) != 0;   // B stored K x N
@@ -256,8 +222,6 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     auto clc_bar = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 4 + i); };
     auto sched_full = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 6 + i); };
     auto sched_empty = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 8 + i); };
-    const uint32_t split_stored = bar0 + 8u * Cfg::SPLIT_BAR0;        // 4 epilogue warps stored a part
-    const uint32_t split_decided = split_stored + 8u;                  // the part's fate is known
     const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
     const uint32_t abort_slot = tmem_slot + 4u;
     const uint32_t tile_ids = tmem_slot + 8u;              // int32 [2]
@@ -265,7 +229,6 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
     volatile uint32_t *abort_flag = tmem_slot_ptr + 1;
     volatile int32_t *tile_id_ptr = reinterpret_cast<volatile int32_t *>(tmem_slot_ptr + 2);
-    volatile uint32_t *last_part_flag = tmem_slot_ptr + 12;   // after the CLC answers
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -283,8 +246,6 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 mbar_init(sched_empty(i), Cfg::SCHED_CONSUMERS);
             }
         }
-        mbar_init(split_stored, 4);
-        mbar_init(split_decided, 1);
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -307,7 +268,6 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + Cfg::BK - 1) / Cfg::BK;
-    const int num_items = sp.split > 1 ? sp.num_full + (num_tiles - sp.num_full) * sp.split : num_tiles;
     const int cluster_id = static_cast<int>(blockIdx.x) / CG;
     const int num_clusters = static_cast<int>(gridDim.x) / CG;
 
@@ -320,7 +280,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             (void)j;
             (void)ok;
             const int n = tile + num_clusters;
-            return n < num_items ? n : -1;
+            return n < num_tiles ? n : -1;
         } else {
             (void)tile;
             const uint32_t slot = j & 1u;
@@ -344,12 +304,11 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             uint32_t fetched = 0;
 
             for (int tile = cluster_id; ok && tile >= 0;) {
-                const WorkItem item = decode_item(tile, sp, num_kb);
                 int tm, tn;
-                raster_tile(item.tile, num_m, num_n, group_m, tm, tn);
+                raster_tile(tile, num_m, num_n, group_m, tm, tn);
                 const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;   // + c * BM_MMA
                 const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
-                for (int kb = item.kb0; kb < item.kb1; ++kb) {
+                for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarEmpty);
                         ok = false;
@@ -358,7 +317,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t a_dst = base + stage * Cfg::STAGE_BYTES;
                     const uint32_t b_dst = a_dst + Cfg::A_BYTES;
                     const int kx = kb * Cfg::BK;
-                    if ((inject & kInjectDropFirstStage) && blockIdx.x == 0 && fetched == 0 && kb == item.kb0) {
+                    if ((inject & kInjectDropFirstStage) && blockIdx.x == 0 && fetched == 0 && kb == 0) {
                         // Failure-detection test: this stage's full barrier is
                         // never armed, so the MMA's bounded wait on it expires.
                         if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -420,8 +379,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + buf * Cfg::CONSUMERS * Cfg::BN;
-                const WorkItem item = decode_item(tile, sp, num_kb);
-                for (int kb = item.kb0; kb < item.kb1; ++kb) {
+                for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarFull);
                         ok = false;
@@ -436,7 +394,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         for (int c = 0; c < Cfg::CONSUMERS; ++c)   // both consumers read this B k-step
                             mma_bf16_ss<CG>(d_tmem + c * Cfg::BN,
                                             a_desc0 + soff + (c * Cfg::A_PART_BYTES >> 4) + kk * a_kstep, bd, idesc,
-                                            (kb != item.kb0 || kk != 0) ? 1u : 0u);
+                                            (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit<CG>(empty_bar(stage), 0x3);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -486,12 +444,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const bool fused = !epi.identity();
         const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
         uint32_t nstore = 0;
-        uint32_t nparts = 0;                       // split parts handled (barrier parity)
         int t = 0;
         for (int tile = cluster_id; tile >= 0; ++t) {
-            const WorkItem item = decode_item(tile, sp, num_kb);
             int tm, tn;
-            raster_tile(item.tile, num_m, num_n, group_m, tm, tn);
+            raster_tile(tile, num_m, num_n, group_m, tm, tn);
             const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
             const uint32_t acc_phase = (static_cast<uint32_t>(t) / Cfg::ACC_BUFS) & 1u;
             // One lane waits; the verdict is broadcast so the warp stays
@@ -507,188 +463,85 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             const int row_base = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
             const int col0 = tn * Cfg::BN;
             const uint32_t tbase0 = tmem_base + ((sub * 32u) << 16) + buf * Cfg::CONSUMERS * Cfg::BN;
-            if (item.part < 0) {
-                // chunk q: consumer q / EPI_CHUNKS (its own rows and accumulator),
-                // columns (q % EPI_CHUNKS) * EPI_COLS of the tile
+            // chunk q: consumer q / EPI_CHUNKS (its own rows and accumulator),
+            // columns (q % EPI_CHUNKS) * EPI_COLS of the tile
 #pragma unroll 1
-                for (int q = 0; q < Cfg::CONSUMERS * Cfg::EPI_CHUNKS; ++q) {
-                    const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
-                    const int row0 = row_base + cons * Cfg::BM_MMA;
-                    const uint32_t tbase = tbase0 + static_cast<uint32_t>(cons) * Cfg::BN;
-                    uint32_t packed[32];
-                    const int erow = row0 + static_cast<int>(lane);   // this thread's row of C
-                    if constexpr (Cfg::OUT == 0) {
-                        tmem_ld_32x32b_x32(tbase + c * 32, packed);
-                        tmem_ld_wait();
-                        if (fused) epilogue32_f32c(packed, C, ldc, erow, col0 + c * 32, M, N, epi);
-                    } else {
-                        uint32_t v0[32], v1[32];
-                        tmem_ld_32x32b_x32(tbase + c * 64, v0);
-                        tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
-                        tmem_ld_wait();
-                        if (fused) {
-                            epilogue32_bf16c(v0, C, ldc, erow, col0 + c * 64, M, N, epi);
-                            epilogue32_bf16c(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, epi);
-                        }
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
-                            packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
-                        }
+            for (int q = 0; q < Cfg::CONSUMERS * Cfg::EPI_CHUNKS; ++q) {
+                const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
+                const int row0 = row_base + cons * Cfg::BM_MMA;
+                const uint32_t tbase = tbase0 + static_cast<uint32_t>(cons) * Cfg::BN;
+                uint32_t packed[32];
+                const int erow = row0 + static_cast<int>(lane);   // this thread's row of C
+                if constexpr (Cfg::OUT == 0) {
+                    tmem_ld_32x32b_x32(tbase + c * 32, packed);
+                    tmem_ld_wait();
+                    if (fused) epilogue32_f32c(packed, C, ldc, erow, col0 + c * 32, M, N, epi);
+                } else {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_32x32b_x32(tbase + c * 64, v0);
+                    tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
+                    tmem_ld_wait();
+                    if (fused) {
+                        epilogue32_bf16c(v0, C, ldc, erow, col0 + c * 64, M, N, epi);
+                        epilogue32_bf16c(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, epi);
                     }
-                    if (q == Cfg::CONSUMERS * Cfg::EPI_CHUNKS - 1) {
-                        // This warp has read its whole slice of accumulator `buf`.
-                        tc_fence_before_sync();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if constexpr (CG == 1) mbar_arrive_local(tempty_bar(buf));
-                            else mbar_arrive_cluster(map_to_cta(tempty_bar(buf), 0));
-                        }
-                    }
-                    const int cstart = col0 + c * Cfg::EPI_COLS;
-                    if (cstart >= N) continue;                  // chunk wholly right of C
-                    if (cstart + Cfg::EPI_COLS > n_tma) {
-                        // Columns [n_tma, N) end C's rows inside a 16-byte granule:
-                        // a TMA store writes whole granules, so these few elements
-                        // (< 16 bytes per row) go out as plain predicated stores.
-                        const int row = row0 + static_cast<int>(lane);
-                        if (row < M) {
-                            uint8_t *crow = static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * (Cfg::OUT == 0 ? 4 : 2);
 #pragma unroll
-                            for (int w = 0; w < Cfg::EPI_COLS; ++w) {
-                                const int col = cstart + w;
-                                if (col >= n_tma && col < N) {
-                                    if constexpr (Cfg::OUT == 0) {
-                                        reinterpret_cast<uint32_t *>(crow)[col] = packed[w];
-                                    } else {
-                                        reinterpret_cast<uint16_t *>(crow)[col] =
-                                            static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
-                                    }
+                    for (int i = 0; i < 16; ++i) {
+                        packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+                        packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+                    }
+                }
+                if (q == Cfg::CONSUMERS * Cfg::EPI_CHUNKS - 1) {
+                    // This warp has read its whole slice of accumulator `buf`.
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (CG == 1) mbar_arrive_local(tempty_bar(buf));
+                        else mbar_arrive_cluster(map_to_cta(tempty_bar(buf), 0));
+                    }
+                }
+                const int cstart = col0 + c * Cfg::EPI_COLS;
+                if (cstart >= N) continue;                  // chunk wholly right of C
+                if (cstart + Cfg::EPI_COLS > n_tma) {
+                    // Columns [n_tma, N) end C's rows inside a 16-byte granule:
+                    // a TMA store writes whole granules, so these few elements
+                    // (< 16 bytes per row) go out as plain predicated stores.
+                    const int row = row0 + static_cast<int>(lane);
+                    if (row < M) {
+                        uint8_t *crow = static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * (Cfg::OUT == 0 ? 4 : 2);
+#pragma unroll
+                        for (int w = 0; w < Cfg::EPI_COLS; ++w) {
+                            const int col = cstart + w;
+                            if (col >= n_tma && col < N) {
+                                if constexpr (Cfg::OUT == 0) {
+                                    reinterpret_cast<uint32_t *>(crow)[col] = packed[w];
+                                } else {
+                                    reinterpret_cast<uint16_t *>(crow)[col] =
+                                        static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
                                 }
                             }
                         }
-                        if (cstart >= n_tma) continue;          // nothing left for the TMA store
                     }
-                    const uint32_t sbuf = stage_base + (nstore & 1u) * Cfg::EPI_BUF;
-                    if (lane == 0) bulk_wait_group_read<1>();   // the store that used sbuf is done reading
-                    __syncwarp();
-                    // Row `lane` of the 32 x 128-byte box; 16-byte chunk j goes to
-                    // chunk slot j ^ (row % 8) -- the TMA 128-byte swizzle.
-                    const uint32_t row_addr = sbuf + lane * 128u;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4),
-                                     packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmC, sbuf, col0 + c * Cfg::EPI_COLS, row0);
-                        bulk_commit_group();
-                    }
-                    ++nstore;
+                    if (cstart >= n_tma) continue;          // nothing left for the TMA store
                 }
-            } else {
-                // A part of a split tile: this CTA's fp32 accumulator goes to
-                // the part's slot; the last part of the tile to arrive sums
-                // all parts in part order and writes C.  The four epilogue
-                // warps meet on bounded mbarrier waits (never a named
-                // barrier), so an aborted call cannot strand one of them.
-                const size_t tile_elems = static_cast<size_t>(Cfg::BM_CTA) * Cfg::BN;
-                const int ti = item.tile - sp.num_full;
-                const int rl = static_cast<int>(sub) * 32 + static_cast<int>(lane);   // row within the CTA
-                float *my_slot = sp.partials + ((static_cast<size_t>(ti) * sp.split + item.part) * CG + rank) *
-                                                   Cfg::CONSUMERS * tile_elems;
-#pragma unroll 1
-                for (int cons = 0; cons < Cfg::CONSUMERS; ++cons) {
-                    float4 *dst = reinterpret_cast<float4 *>(my_slot + cons * tile_elems + static_cast<size_t>(rl) * Cfg::BN);
-#pragma unroll 1
-                    for (int g = 0; g < Cfg::BN / 32; ++g) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(tbase0 + static_cast<uint32_t>(cons * Cfg::BN + g * 32), v);
-                        tmem_ld_wait();
+                const uint32_t sbuf = stage_base + (nstore & 1u) * Cfg::EPI_BUF;
+                if (lane == 0) bulk_wait_group_read<1>();   // the store that used sbuf is done reading
+                __syncwarp();
+                // Row `lane` of the 32 x 128-byte box; 16-byte chunk j goes to
+                // chunk slot j ^ (row % 8) -- the TMA 128-byte swizzle.
+                const uint32_t row_addr = sbuf + lane * 128u;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            __stcg(dst + g * 8 + j, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
-                    }
+                for (int j = 0; j < 8; ++j) {
+                    st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4),
+                                 packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
                 }
-                tc_fence_before_sync();
-                __threadfence();                           // this thread's part stores, GPU-wide
+                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    if constexpr (CG == 1) mbar_arrive_local(tempty_bar(buf));
-                    else mbar_arrive_cluster(map_to_cta(tempty_bar(buf), 0));
-                    mbar_arrive_local(split_stored);
+                    tma_store_2d(&tmC, sbuf, col0 + c * Cfg::EPI_COLS, row0);
+                    bulk_commit_group();
                 }
-                const uint32_t par = nparts & 1u;
-                ++nparts;
-                uint32_t go = 1;
-                if (threadIdx.x == 64) {                   // warp 2, lane 0 decides
-                    if (!mbar_wait(split_stored, par, abort_flag, 3 * timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarSplit);
-                        go = 0;
-                        *last_part_flag = 0u;           // no fix-up from an incomplete tile
-                    } else {
-                        __threadfence();
-                        unsigned long long *ctr = sp.counters + ti * CG + rank;
-                        const unsigned long long tag = static_cast<unsigned long long>(sp.epoch) << 32;
-                        unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(ctr), seen, want;
-                        do {
-                            seen = old;
-                            want = ((seen & 0xFFFFFFFF00000000ull) == tag) ? seen + 1ull : (tag | 1ull);
-                            old = atomicCAS(ctr, seen, want);
-                        } while (old != seen);
-                        const bool last = (want & 0xFFFFFFFFull) == static_cast<unsigned long long>(sp.split);
-                        if (last) *ctr = tag;       // every part has arrived: zero arrivals for a replay
-                        *last_part_flag = last ? 1u : 0u;
-                    }
-                    mbar_arrive_local(split_decided);
-                }
-                if (lane == 0 && go && !mbar_wait(split_decided, par, abort_flag, 3 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarSplit);
-                    go = 0;
-                }
-                uint32_t last = (lane == 0 && go) ? *last_part_flag : 0u;
-                go = __shfl_sync(0xffffffffu, go, 0);
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (!go) break;
-                if (last) {
-                    __threadfence();
-                    const float *slots = sp.partials + (static_cast<size_t>(ti) * sp.split * CG + rank) *
-                                                           Cfg::CONSUMERS * tile_elems;
-                    const size_t part_stride = static_cast<size_t>(CG) * Cfg::CONSUMERS * tile_elems;
-#pragma unroll 1
-                    for (int cons = 0; cons < Cfg::CONSUMERS; ++cons) {
-                        const int row = row_base + cons * Cfg::BM_MMA + static_cast<int>(lane);
-                        if (row >= M) continue;
-                        const float *src = slots + cons * tile_elems + static_cast<size_t>(rl) * Cfg::BN;
-                        uint8_t *crow = static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * (Cfg::OUT == 0 ? 4 : 2);
-#pragma unroll 1
-                        for (int c4 = 0; c4 < Cfg::BN; c4 += 4) {
-                            const int col = col0 + c4;
-                            if (col >= N) break;
-                            float4 acc = __ldcg(reinterpret_cast<const float4 *>(src + c4));
-                            for (int p = 1; p < sp.split; ++p) {   // part order: the same sums on every run
-                                const float4 x = __ldcg(reinterpret_cast<const float4 *>(src + p * part_stride + c4));
-                                acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
-                            }
-                            float vals[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                if (col + e >= N) break;
-                                float old = 0.0f;
-                                if (epi.beta != 0.0f)
-                                    old = Cfg::OUT == 0 ? reinterpret_cast<const float *>(crow)[col + e]
-                                                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(crow)[col + e]);
-                                const float b = epi.bias ? __ldg(epi.bias + col + e) : 0.0f;
-                                const float y = fused ? finish(vals[e], old, b, epi) : vals[e];
-                                if constexpr (Cfg::OUT == 0) reinterpret_cast<float *>(crow)[col + e] = y;
-                                else reinterpret_cast<__nv_bfloat16 *>(crow)[col + e] = __float2bfloat16_rn(y);
-                            }
-                        }
-                    }
-                }
+                ++nstore;
             }
             // next tile: one lane fetches it, the warp follows
             int nt = -1;

@@ -23,8 +23,7 @@
  * Ownership: every pointer is a DEVICE pointer owned by the caller, valid
  * until the work queued on `stream` has finished.  The library keeps, per
  * device, a small status block (allocated on the first call on a device),
- * cached launch attributes and, for the skinny and block-scaled paths (and
- * the split tail of the square kernels, when B200GEMM_SPLIT turns it on), a
+ * cached launch attributes and, for the skinny and block-scaled paths, a
  * workspace that grows on demand.  A workspace that a larger one replaces
  * is kept, never freed, while the library is loaded.
  *
