@@ -356,6 +356,12 @@ def oracle_sample(problem: Problem, budget_s: float):
     return 2.0 * R * problem.N * problem.K, dt, R
 
 
+def needs_l2_flush(traffic_bytes: int) -> bool:
+    """Inputs plus output under twice the L2 would be served partly from L2
+    across back-to-back steps; those workloads flush it between steps."""
+    return traffic_bytes < 2 * L2_BYTES
+
+
 def metric_of(kind: str) -> str:
     return {"bf16": METRIC, "mxfp8": METRIC_MXFP8, "fused": METRIC_FUSED}[kind]
 
@@ -460,7 +466,7 @@ def main():
     # back-to-back steps: flush it between steps (write a buffer larger than
     # L2 outside the events) and time each step on its own.
     traffic_bytes = p.in_bytes + p.out_bytes
-    flush = traffic_bytes < 2 * L2_BYTES
+    flush = needs_l2_flush(traffic_bytes)
     scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
     sampler = ClockSampler(gpu_id)
     sampler.start()

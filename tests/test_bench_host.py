@@ -83,7 +83,7 @@ def test_workloads_match_the_named_configs():
 def test_oracle_sample_is_bounded():
     p = bench.Problem("square4096", (64, 96, 128), 0)
     flops, dt, rows = bench.oracle_sample(p, budget_s=0.05)
-    assert 4 <= rows <= 64 and flops == 2.0 * rows * 96 * 128 and dt < 5
+    assert 1 <= rows <= 64 and flops == 2.0 * rows * 96 * 128 and dt < 5
 
 
 def test_reference_arm_other_ranks_exit_without_work():
@@ -113,3 +113,26 @@ def test_kernel_hash_ignores_comments_only():
     assert bench.code_only(a) != bench.code_only(c)
     for kernel in bench.KERNEL_SOURCES:
         assert len(bench.kernel_source_hash(kernel)) == 16
+
+
+def test_only_the_8192_cubes_run_without_an_l2_flush():
+    for name in bench.WORKLOADS:
+        p = bench.Problem(name, (8, 8, 32), 0)          # the byte counts below use the full sizes
+        M, N, K, kind = bench.WORKLOADS[name][:4]
+        in_b = {"bf16": 2 * (M * K + N * K), "fused": 2 * (M * K + N * K) + 4 * N,
+                "mxfp8": M * K + N * K + (M + N) * (K // 32)}[kind]
+        out_b = 4 * M * N if kind == "bf16" else 2 * M * N
+        assert bench.needs_l2_flush(in_b + out_b) == (M != 8192), name
+        assert p.kind == kind
+
+
+def test_fused_workloads_use_their_activation_in_the_oracle_leg():
+    import numpy as np
+    import oracle
+    for name, act in (("fused8192", oracle.ACT_GELU), ("fused8192_tanh", oracle.ACT_GELU_TANH)):
+        p = bench.Problem(name, (4, 8, 64), 0)
+        got = p.oracle_rows(4)
+        base = oracle.gemm_bf16_f64(p.a[:4], p.b, K=64)
+        want = oracle.epilogue(base, None, 1.0, 0.0, p.bias.astype(np.float64), act)
+        assert np.array_equal(got, want)
+    assert bench.metric_of("fused") == bench.METRIC_FUSED and bench.metric_of("mxfp8") == bench.METRIC_MXFP8
