@@ -21,12 +21,18 @@
 //       warp 0 loads A, B and the scale chunks by TMA (for a pair, every
 //       byte counts on the leader's barrier; each CTA holds its own 128 rows
 //       of A scales and the scales of all 256 rows of B);
-//       warp 1 of the (leader) CTA copies the stage's scales into TMEM
-//       (tcgen05.cp, cta_group::2 for a pair: each CTA's SMEM to its own
-//       TMEM; two slots alternating) and issues 4 block-scaled MMAs (K = 32 each, the byte of
-//       the scale column chosen in the instruction descriptor); warps 2-5
-//       drain the accumulator to registers, release TMEM once the last
-//       columns are read, and write bf16 C with 16-byte global stores.
+//       warp 10 of the (leader) CTA copies each stage's scales into one of
+//       four TMEM scale slots (tcgen05.cp, cta_group::2 for a pair: each
+//       CTA's SMEM to its own TMEM), ordered against the MMAs only by the
+//       sf_full / sf_empty barriers, so a later stage's copy can overlap the
+//       current stage's MMAs;
+//       warp 1 of the (leader) CTA issues 4 block-scaled MMAs per stage
+//       (K = 32 each, the byte of the scale column chosen in the instruction
+//       descriptor);
+//       warps 2-9 (two per TMEM lane quarter, half of the columns each)
+//       drain the single-buffered accumulator into registers as packed
+//       bf16, release TMEM, and only then write C with 16-byte global
+//       stores, so the next tile's MMAs wait for the TMEM reads alone.
 //
 // TMEM: accumulator columns [0, 256); scale slot s at 256 + 32 s (A: 4
 // columns) and 256 + 32 s + 16 (B: 8 columns).  Every scale sits in lane
