@@ -4,6 +4,7 @@
                     [--workload square8192|square4096|ragged|skinny1000|skinny16|mxfp8_8192|fused8192
                                 |fused8192_tanh]
                     [--shape M N K] [--config auto|1cta_128x128|1cta_128x256|2cta_256x256]
+                    [--no-configs] [--config-steps S]
 
 One step = one library call over the whole M x N x K problem with the inputs
 resident in HBM.  Multi-GPU runs (torchrun, one process per GPU) are
@@ -14,8 +15,12 @@ Printed (rank 0): one JSON line with the metric, the device-timed value,
 `e2e` (the same metric through the C ABI with host buffers, copies inside
 the timed region), `roofline` of the GEMM kernel, `cpu_baseline` (the CPU
 oracle on a bounded sample of the same workload), clocks sampled during the
-timed region and the number of kernel launches.  `--impl reference` times
-the oracle alone, as the reference arm.
+timed region and the number of kernel launches.  The default run (8192^3,
+one GPU) adds `configs`: every other configuration's workload timed on its
+own after the headline (median, p90, TFLOP/s, GB/s, and the roofline, the
+larger of FLOPs / tensor peak and minimum bytes / HBM bandwidth), plus the
+single tile's CUDA-graph replay time.  `--impl reference` times the oracle
+alone, as the reference arm.
 """
 from __future__ import annotations
 
@@ -43,8 +48,11 @@ UNIT = "TFLOP/s"
 WORKLOADS = {
     "square8192": (8192, 8192, 8192, "bf16", "uniform", 3,
                    "gemm 8192x8192x8192, bf16 U[-1,1] in, fp32 accumulate + out"),
+    "single_tile128": (128, 128, 128, "bf16", "uniform", 1, "gemm 128x128x128, bf16 U[-1,1] in, fp32 out"),
     "square4096": (4096, 4096, 4096, "bf16", "normal_scaled", 2,
                    "gemm 4096x4096x4096, bf16 N(0,1)/sqrt(K) in, fp32 out"),
+    "square4096_bf16": (4096, 4096, 4096, "bf16", "normal_scaled", 2,
+                        "gemm 4096x4096x4096, bf16 N(0,1)/sqrt(K) in, bf16 out"),
     "ragged": (4000, 3000, 2000, "bf16", "normal", 4, "gemm 4000x3000x2000, bf16 N(0,1) in, fp32 out"),
     "skinny1000": (1000, 8192, 8192, "bf16", "normal", 5, "gemm 1000x8192x8192, bf16 N(0,1) in, fp32 out"),
     "skinny16": (16, 8192, 8192, "bf16", "normal", 6, "gemm 16x8192x8192, bf16 N(0,1) in, fp32 out"),
@@ -58,10 +66,32 @@ WORKLOADS = {
 }
 # activation of the fused workloads (gemm_bf16_fused's act)
 FUSED_ACT = {"fused8192": "gelu", "fused8192_tanh": "gelu_tanh"}
+# plain GEMM workloads that write bf16 C (the others write fp32)
+BF16_OUT = {"square4096_bf16"}
+# the per-config report of the default run: every workload of the five
+# configurations, each timed on its own (the headline is the main line)
+CONFIG_SET = ("single_tile128", "square4096", "square4096_bf16", "ragged", "skinny1000", "skinny16",
+              "mxfp8_8192")
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+# nominal B200 figures the fraction is also reported against
+NOMINAL = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+
+
+def roofline_of(flops: float, min_bytes: float, seconds: float, tensor_tflops: float, hbm_gbs: float) -> dict:
+    """The roofline of one launch: its time can be no lower than the larger
+    of (FLOPs / tensor peak) and (minimum bytes / HBM bandwidth); that larger
+    term names the bound, and frac = roofline time / measured time, which
+    equals achieved / peak in the bound's own unit."""
+    t_tensor = flops / (tensor_tflops * 1e12)
+    t_hbm = min_bytes / (hbm_gbs * 1e9)
+    if t_tensor >= t_hbm:
+        return {"bound": "tensor", "achieved": flops / seconds / 1e12, "peak": tensor_tflops, "unit": "TFLOP/s",
+                "frac": t_tensor / seconds, "roofline_us": t_tensor * 1e6}
+    return {"bound": "hbm", "achieved": min_bytes / seconds / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+            "frac": t_hbm / seconds, "roofline_us": t_hbm * 1e6}
 
 
 # The device sources each kernel is compiled from; an ncu traffic figure is
@@ -218,13 +248,14 @@ class Problem:
                     "fused": f"gelu(A.B + bias) {M}x{N}x{K}, bf16 U[-1,1] in, bf16 out",
                     "mxfp8": f"block-scaled gemm {M}x{N}x{K}, E4M3 U[-1,1], E8M0 per 32, bf16 out"}[kind]
         self.name, self.M, self.N, self.K, self.kind, self.desc = name, M, N, K, kind, desc
+        self.bf16_out = name in BF16_OUT
         self.act = FUSED_ACT.get(name, "gelu")
         self.flops = 2.0 * M * N * K
         if kind == "bf16":
             self.a, self.b = synth.bf16_operands(M, N, K, dist, workload=wid, base=rank)
             self.host = [self.a, self.b]
             self.in_bytes = 2 * (M * K + N * K)
-            self.out_bytes = 4 * M * N
+            self.out_bytes = (2 if self.bf16_out else 4) * M * N
         elif kind == "fused":
             self.a, self.b = synth.bf16_operands(M, N, K, dist, workload=wid, base=rank)
             self.bias = synth.normal(synth.derive_seed(wid, 4, rank), (N,)).astype(np.float32)
@@ -246,7 +277,7 @@ class Problem:
         return [torch.from_numpy(np.ascontiguousarray(x)).cuda() for x in self.host]
 
     def empty_out(self, torch, pinned=False):
-        dt = torch.float32 if self.kind == "bf16" else torch.bfloat16
+        dt = torch.float32 if self.kind == "bf16" and not self.bf16_out else torch.bfloat16
         if pinned:
             return torch.empty((self.M, self.N), dtype=dt).pin_memory()
         return torch.empty((self.M, self.N), dtype=dt, device="cuda")
@@ -255,7 +286,7 @@ class Problem:
         M, N, K = self.M, self.N, self.K
         if self.kind == "bf16":
             A, B = dev
-            G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_F32, stream=stream)
+            G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_BF16 if self.bf16_out else G.OUT_F32, stream=stream)
         elif self.kind == "fused":
             A, B, bias = dev
             G.gemm_bf16_fused(A, B, C, M, N, K, K, K, N, G.OUT_BF16, G.KMAJOR, G.KMAJOR, 1.0, 0.0, bias,
@@ -330,6 +361,104 @@ def fusion_comparison(p, G, dev, torch, stream, steps):
             "fused_over_plain_gemm_ms": fused_ms - gemm_ms,
             "ledger_saved_bytes": 2 * inter,
             "unfused_pass_gbs": (2 * inter + 4 * N) / (pass_ms * 1e-3) / 1e9, "steps": steps}
+
+
+def min_bytes(p: Problem) -> int:
+    """Operands read once plus C written once: the byte floor of one call."""
+    return p.in_bytes + p.out_bytes
+
+
+def time_steps(p: Problem, G, dev, C, torch, stream, steps: int, scratch=None):
+    """Device time of each of `steps` calls (ms).  With `scratch`, L2 is
+    flushed before every call by writing that buffer outside the events."""
+    if scratch is not None:
+        ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            scratch.zero_()
+            ev_s[i].record(stream)
+            p.call(G, dev, C, stream)
+            ev_e[i].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)], None
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        p.call(G, dev, C, stream)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)], ev[0].elapsed_time(ev[-1])
+
+
+def graph_replay_us(p: Problem, G, dev, C, torch, stream, steps: int, scratch) -> float:
+    """Median device time (us) of one call captured in a CUDA graph and
+    replayed, L2 flushed before each replay outside the events."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        p.call(G, dev, C, torch.cuda.current_stream())
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        scratch.zero_()
+        ev_s[i].record(stream)
+        g.replay()
+        ev_e[i].record(stream)
+    torch.cuda.synchronize()
+    t = statistics.median(a.elapsed_time(b) for a, b in zip(ev_s, ev_e)) * 1e3
+    del g
+    return t
+
+
+def config_report(G, torch, stream, peaks: dict, steps: int, warmup: int) -> dict:
+    """Every workload of CONFIG_SET timed on its own, on the same GPU, with
+    the same L2 rule as the headline: median and p90 of `steps` calls,
+    TFLOP/s and GB/s at the median, and the roofline (the larger of FLOPs /
+    tensor peak and minimum bytes / HBM bandwidth) against the measured
+    peaks and against the nominal B200 figures."""
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    out = {}
+    for name in CONFIG_SET:
+        p = Problem(name, None, 0)
+        dev = p.device_arrays(torch)
+        C = p.empty_out(torch)
+        for _ in range(warmup):
+            p.call(G, dev, C, stream)
+        G.gemm_check_device_status(stream)
+        flush = needs_l2_flush(min_bytes(p))
+        per_step, _ = time_steps(p, G, dev, C, torch, stream, steps, scratch if flush else None)
+        G.gemm_check_device_status(stream)
+        med = statistics.median(per_step) * 1e-3
+        ratio = FP8_OVER_BF16 if p.kind == "mxfp8" else 1.0
+        measured = roofline_of(p.flops, min_bytes(p), med, float(peaks["bf16_tflops"]) * ratio,
+                               float(peaks["hbm_gbs"]))
+        nominal = roofline_of(p.flops, min_bytes(p), med, NOMINAL["bf16_tflops"] * ratio, NOMINAL["hbm_gbs"])
+        entry = {"workload": p.desc, "M": p.M, "N": p.N, "K": p.K, "kernel_config": config_name(G, p, "auto"),
+                 "launches_per_call": p.launches(G), "steps": steps,
+                 "l2": "flushed before every call" if flush else "no flush (inputs+output > 2 x L2)",
+                 "median_us": med * 1e6, "p90_us": float(np.percentile(per_step, 90)) * 1e3,
+                 "tflops": p.flops / med / 1e12, "gbs": min_bytes(p) / med / 1e9,
+                 "bound": measured["bound"], "roofline_us": measured["roofline_us"], "frac": measured["frac"],
+                 "frac_of_nominal": nominal["frac"], "min_bytes": min_bytes(p)}
+        if name == "single_tile128":
+            # one 128 x 128 tile: launch latency, not a roofline, bounds it
+            entry["bound"] = "latency"
+            entry["graph_replay_us"] = graph_replay_us(p, G, dev, C, torch, stream, steps, scratch)
+        out[name] = entry
+        del dev, C
+    del scratch
+    return out
+
+
+def config_name(G, p: Problem, forced: str) -> str:
+    """Name of the kernel configuration a call of this problem runs."""
+    if p.kind == "mxfp8":
+        pair_tiles = ((p.M + 255) // 256) * ((p.N + 255) // 256)
+        return forced if forced.startswith("mxfp8") else \
+            ("mxfp8_2cta_256x256" if pair_tiles >= 74 else "mxfp8_1cta_128x256")
+    name = {v: k for k, v in G.CONFIGS.items()}[G.gemm_select_config(p.M, p.N, p.K)]
+    if p.kind == "fused" and forced == "auto" and name == "2cta_512x256_clc":
+        name = "2cta_256x256_clc"   # the library's choice for a non-plain epilogue
+    return name
 
 
 def oracle_sample(problem: Problem, budget_s: float):
@@ -410,6 +539,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5, help="0 skips the end-to-end leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the per-config report (default run: every configuration's workload)")
+    ap.add_argument("--config-steps", type=int, default=50)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -442,14 +574,7 @@ def main():
     dev = p.device_arrays(torch)
     C = p.empty_out(torch)
     G.gemm_force_config(args.config)
-    if p.kind == "mxfp8":
-        pair_tiles = ((p.M + 255) // 256) * ((p.N + 255) // 256)
-        cfg_name = args.config if args.config.startswith("mxfp8") else \
-            ("mxfp8_2cta_256x256" if pair_tiles >= 74 else "mxfp8_1cta_128x256")
-    else:
-        cfg_name = {v: k for k, v in G.CONFIGS.items()}[G.gemm_select_config(p.M, p.N, p.K)]
-        if p.kind == "fused" and args.config == "auto" and cfg_name == "2cta_512x256_clc":
-            cfg_name = "2cta_256x256_clc"   # the library's choice for a non-plain epilogue
+    cfg_name = config_name(G, p, args.config)
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
@@ -472,30 +597,11 @@ def main():
     sampler.start()
     barrier()
     torch.cuda.synchronize()
-    if flush:
-        ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        for i in range(args.steps):
-            scratch.zero_()
-            ev_s[i].record(stream)
-            p.call(G, dev, C, stream)
-            ev_e[i].record(stream)
-    else:
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-        ev[0].record(stream)
-        for i in range(args.steps):
-            p.call(G, dev, C, stream)
-            ev[i + 1].record(stream)
-    torch.cuda.synchronize()
+    per_step_ms, span_ms = time_steps(p, G, dev, C, torch, stream, args.steps, scratch)
     barrier()
     sampler.stop()
     G.gemm_check_device_status(stream)
-    if flush:
-        per_step_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
-        local_ms = sum(per_step_ms)
-    else:
-        per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-        local_ms = ev[0].elapsed_time(ev[-1])
+    local_ms = span_ms if span_ms is not None else sum(per_step_ms)
     t_ms = max_over_ranks(local_ms, world, "cuda")
 
     fusion = fusion_comparison(p, G, dev, torch, stream, min(args.steps, 50)) if p.kind == "fused" else None
@@ -535,25 +641,41 @@ def main():
     if rank != 0:
         return
 
-    value = whole_job_tflops(p.flops, args.steps, world, t_ms)
     peaks, peak_src = load_peaks()
+    for key, v in FALLBACK_PEAKS.items():
+        peaks.setdefault(key, v)
+    configs = None
+    if args.configs and world == 1 and args.shape is None and args.workload == "square8192":
+        G.gemm_force_config("auto")
+        csampler = ClockSampler(gpu_id)
+        csampler.start()
+        configs = config_report(G, torch, stream, peaks, args.config_steps, 5)
+        csampler.stop()
+        configs["clocks"] = csampler.summary()
+        G.gemm_force_config(args.config)
+
+    value = whole_job_tflops(p.flops, args.steps, world, t_ms)
     # per-step event time: for bf16 the step is the one GEMM launch; for
     # MXFP8 it also holds the small scale-repack launch, so `achieved` is a
     # lower bound for the GEMM kernel alone
-    mean_step_ms = sum(per_step_ms) / len(per_step_ms)
-    achieved = p.flops / (mean_step_ms * 1e-3) / 1e12
-    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    mean_step_s = sum(per_step_ms) / len(per_step_ms) * 1e-3
+    bf16_peak = float(peaks["bf16_tflops"])
+    sustained = float(peaks["bf16_tflops_sustained"])
     ratio = FP8_OVER_BF16 if p.kind == "mxfp8" else 1.0
-    peak = bf16_peak * ratio
-    peak_note = (f"{peak_src} bf16_tflops (burst, cuBLAS 8192^3)" if p.kind != "mxfp8" else
-                 f"{peak_src} bf16_tflops x {FP8_OVER_BF16:g} (nominal fp8/bf16 dense ratio)")
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profile_traffic(p.name, cfg_name),
-                "peak_source": peak_note,
-                "frac_of_sustained_peak": achieved / (sustained * ratio),
-                "algorithmic_flops_per_launch": p.flops,
-                "min_bytes_per_launch": p.in_bytes + p.out_bytes}
+    roofline = roofline_of(p.flops, min_bytes(p), mean_step_s, bf16_peak * ratio, float(peaks["hbm_gbs"]))
+    nominal = roofline_of(p.flops, min_bytes(p), mean_step_s, NOMINAL["bf16_tflops"] * ratio, NOMINAL["hbm_gbs"])
+    if roofline["bound"] == "tensor":
+        peak_note = (f"{peak_src} bf16_tflops (burst, cuBLAS 8192^3)" if p.kind != "mxfp8" else
+                     f"{peak_src} bf16_tflops x {FP8_OVER_BF16:g} (nominal fp8/bf16 dense ratio)")
+    else:
+        peak_note = f"{peak_src} hbm_gbs (copy bandwidth)"
+    roofline.update({
+        "traffic": profile_traffic(p.name, cfg_name), "peak_source": peak_note,
+        "frac_of_nominal_peak": nominal["frac"],
+        "nominal_peak": nominal["peak"],
+        "frac_of_sustained_peak": (p.flops / mean_step_s / 1e12) / (sustained * ratio),
+        "algorithmic_flops_per_launch": p.flops,
+        "min_bytes_per_launch": min_bytes(p)})
 
     cpu = None
     if not args.no_cpu_baseline:
@@ -582,8 +704,10 @@ def main():
         "clocks": sampler.summary(),
         "gpu_launches": args.steps * p.launches(G) * world,
     }
+    if configs:
+        line["configs"] = configs
     if fusion:
-        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        hbm = float(peaks["hbm_gbs"])
         fusion["ledger_saved_ms_at_hbm_peak"] = fusion["ledger_saved_bytes"] / (hbm * 1e9) * 1e3
         fusion["unfused_pass_frac_of_hbm_peak"] = fusion["unfused_pass_gbs"] / hbm
         line["fusion"] = fusion

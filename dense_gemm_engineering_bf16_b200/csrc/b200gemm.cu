@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "b200gemm.h"
@@ -53,7 +54,11 @@ struct DeviceState {
     bool ready = false;
     bool supported = false;
     int sm_count = 0;
+    // watchdog status blocks: `status` from cudaMalloc (first allocating call
+    // on the device), `noalloc_status` the device address of the library's
+    // static scratch array (first gemm_bf16_noalloc call on the device)
     DeviceStatus *status = nullptr;
+    DeviceStatus *noalloc_status = nullptr;
     // per (config, out type): smem attribute set, co-resident clusters
     bool attr_done[GEMM_CFG_COUNT_][2] = {};
     int max_clusters[GEMM_CFG_COUNT_][2] = {};
@@ -112,12 +117,20 @@ int raster_group_m() {
     return g;
 }
 
-// Test-only: B200GEMM_INJECT_TIMEOUT=1 makes the next square-kernel launches
-// drop one pipeline arrival in CTA 0 so the device watchdog fires (read at
-// every launch, so a test can switch it on and off inside one process).
+// Test-only: B200GEMM_INJECT_TIMEOUT holds one character per launch of the
+// dense bf16 kernels, in launch order; a '1' makes that launch drop one
+// pipeline arrival in CTA 0 so the device watchdog fires.  The variable is
+// read once, at the first launch; unset or empty, launches only test one
+// static flag.
 uint32_t inject_flags() {
-    const char *s = std::getenv("B200GEMM_INJECT_TIMEOUT");
-    return (s && s[0] == '1') ? b200::kInjectDropFirstStage : 0u;
+    static const std::string mask = [] {
+        const char *s = std::getenv("B200GEMM_INJECT_TIMEOUT");
+        return std::string(s ? s : "");
+    }();
+    if (mask.empty()) return 0u;
+    static std::atomic<size_t> launches{0};
+    const size_t i = launches.fetch_add(1, std::memory_order_relaxed);
+    return (i < mask.size() && mask[i] == '1') ? b200::kInjectDropFirstStage : 0u;
 }
 
 // True while `stream` is being captured into a CUDA graph (or when that
@@ -132,8 +145,8 @@ bool capturing(cudaStream_t stream) {
 }
 
 // Device of the current thread, checked to be compute capability 10.0, with
-// its status block allocated.  The one-time set-up (cudaMalloc, a blocking
-// cudaMemset) may not run inside a stream capture: GEMM_ERR_CAPTURE then.
+// the tensor-map encoder looked up.  Allocates nothing.  The one-time
+// set-up may not run inside a stream capture: GEMM_ERR_CAPTURE then.
 gemm_status_t current_device(int &dev, DeviceState *&st, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -156,8 +169,6 @@ gemm_status_t current_device(int &dev, DeviceState *&st, cudaStream_t stream) {
         }
         if ((e = cudaDeviceGetAttribute(&st->sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail(e);
-        if ((e = cudaMalloc(&st->status, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
-        if ((e = cudaMemset(st->status, 0, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
         if (!g_encode) {
             void *fn = nullptr;
             cudaDriverEntryPointQueryResult q;
@@ -168,6 +179,23 @@ gemm_status_t current_device(int &dev, DeviceState *&st, cudaStream_t stream) {
         st->ready = true;
     }
     return st->supported ? GEMM_OK : GEMM_ERR_UNSUPPORTED_DEVICE;
+}
+
+// current_device, plus the device's status block from cudaMalloc (first
+// call on the device; a blocking cudaMemset zeroes it).
+gemm_status_t current_device_alloc(int &dev, DeviceState *&st, cudaStream_t stream) {
+    gemm_status_t s = current_device(dev, st, stream);
+    if (s != GEMM_OK) return s;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!st->status) {
+        if (capturing(stream)) return GEMM_ERR_CAPTURE;
+        cudaError_t e;
+        DeviceStatus *p = nullptr;
+        if ((e = cudaMalloc(&p, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
+        if ((e = cudaMemset(p, 0, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
+        st->status = p;
+    }
+    return GEMM_OK;
 }
 
 // [begin, end) byte ranges of a row-major rows x cols matrix with leading dim ld.
@@ -257,10 +285,11 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     return GEMM_CFG_1CTA_128x128;
 }
 
+// `status`: the watchdog status block the kernel records a timeout in.
 template <class Cfg>
-gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, const void *B, void *C,
-                          int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                          cudaStream_t stream, const b200::Epilogue &epi = b200::plain_epilogue(),
+gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t cfg_id, const void *A,
+                          const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                          int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi = b200::plain_epilogue(),
                           uint32_t layout = 0) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
@@ -324,7 +353,7 @@ gemm_status_t launch_bf16(DeviceState *st, gemm_config_t cfg_id, const void *A, 
                                       : (tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi]);
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
-                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), st->status,
+                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), status,
                            watchdog_ns(K), inject_flags(), epi, layout);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
@@ -459,30 +488,32 @@ gemm_status_t launch_zero(void *C, int64_t M, int64_t N, int64_t ldc, int sm_cou
 }
 
 // The dense bf16 kernels, by configuration.
-gemm_status_t launch_dense(DeviceState *st, gemm_config_t cfg, bool f32, const void *A, const void *B, void *C,
-                           int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                           cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout) {
+// `status`: the watchdog status block (the skinny kernel, which only the
+// allocating entry points run, always uses the device's cudaMalloc'd one).
+gemm_status_t launch_dense(DeviceState *st, DeviceStatus *status, gemm_config_t cfg, bool f32, const void *A,
+                           const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                           int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout) {
     switch (cfg) {
         case GEMM_CFG_1CTA_128x256:
-            return f32 ? launch_bf16<Cfg1x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg1x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return f32 ? launch_bf16<Cfg1x256F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x256B16>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_1CTA_128x128:
-            return f32 ? launch_bf16<Cfg1x128F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg1x128B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return f32 ? launch_bf16<Cfg1x128F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x128B16>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_256x256:
-            return f32 ? launch_bf16<Cfg2x256F32>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg2x256B16>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return f32 ? launch_bf16<Cfg2x256F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_SKINNY:
             return launch_skinny_any(st, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_256x256_CLC:
-            return f32 ? launch_bf16<Cfg2x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg2x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return f32 ? launch_bf16<Cfg2x256F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_512x256_CLC:
-            return f32 ? launch_bf16<Cfg2x512F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg2x512B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return f32 ? launch_bf16<Cfg2x512F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x512B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_1CTA_128x256_CLC:
-            return f32 ? launch_bf16<Cfg1x256F32C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg1x256B16C>(st, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return f32 ? launch_bf16<Cfg1x256F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg1x256B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         default:
             return GEMM_ERR_INVALID_VALUE;
     }
@@ -494,7 +525,9 @@ gemm_status_t launch_dense(DeviceState *st, gemm_config_t cfg, bool f32, const v
 // scratch (the watchdog status block) lives in the file-scope array below
 // instead of memory obtained from cudaMalloc.  The array is part of the
 // library image: every GPU that loads the library holds its
-// kNoAllocScratchBytes until the process exits.  All calls share it.
+// kNoAllocScratchBytes until the process exits.  All calls share it.  Kernel
+// attributes and co-resident cluster counts are per kernel and device, so
+// this entry point shares them with the others (g_devices).
 
 constexpr size_t kNoAllocScratchBytes = 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -502,47 +535,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // Scratch one call needs: the status block, for every shape.
 constexpr size_t noalloc_scratch_bytes() { return sizeof(DeviceStatus); }
 
-DeviceState g_noalloc_devices[kMaxDevices];
-
-// Per-device set-up, once, with the device current: check the device, take
-// the address of the scratch array with cudaGetSymbolAddress (host code may
-// not use the array's name as a device address), and zero it.
+// Per-device set-up, once, with the device current: the device checks of
+// current_device, then the device address of the scratch array from
+// cudaGetSymbolAddress (in host code the array's name is only a host-side
+// stand-in, never a device address), zeroed once.  From then on the status
+// block there is sticky: a recorded timeout stays until
+// gemm_check_device_status() reads and clears it.
 gemm_status_t noalloc_device(int &dev, DeviceState *&st, cudaStream_t stream) {
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        g_last_cuda_error = static_cast<int>(e);
-        return GEMM_ERR_UNSUPPORTED_DEVICE;
-    }
+    gemm_status_t s = current_device(dev, st, stream);
+    if (s != GEMM_OK) return s;
     std::lock_guard<std::mutex> lock(g_mutex);
-    st = &g_noalloc_devices[dev];
-    if (!st->ready) {
+    if (!st->noalloc_status) {
         if (capturing(stream)) return GEMM_ERR_CAPTURE;
-        int major = 0, minor = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-            return GEMM_ERR_UNSUPPORTED_DEVICE;
-        st->supported = (major == 10 && minor == 0);
-        if (!st->supported) {
-            st->ready = true;
-            return GEMM_ERR_UNSUPPORTED_DEVICE;
-        }
-        if ((e = cudaDeviceGetAttribute(&st->sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-            return cuda_fail(e);
+        cudaError_t e;
         void *scratch = nullptr;
         if ((e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch)) != cudaSuccess || !scratch)
             return cuda_fail(e);
         if ((e = cudaMemset(scratch, 0, kNoAllocScratchBytes)) != cudaSuccess) return cuda_fail(e);
-        st->status = static_cast<DeviceStatus *>(scratch);
-        if (!g_encode) {
-            void *fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
-            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-        }
-        st->ready = true;
+        st->noalloc_status = static_cast<DeviceStatus *>(scratch);
     }
-    return st->supported ? GEMM_OK : GEMM_ERR_UNSUPPORTED_DEVICE;
+    return GEMM_OK;
 }
 
 // ------------------------------------------------------ block-scaled path --
@@ -683,7 +695,7 @@ gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C, int64_t M, 
     const b200::Epilogue epi{alpha, beta, bias, static_cast<uint32_t>(act)};
     int dev;
     DeviceState *st;
-    if ((s = current_device(dev, st, stream)) != GEMM_OK) return s;
+    if ((s = current_device_alloc(dev, st, stream)) != GEMM_OK) return s;
     const bool f32 = c_type == GEMM_OUT_F32;
     if (K == 0) {
         // the empty sum: C = act(beta * C + bias); plain zeros (C not read)
@@ -702,7 +714,7 @@ gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C, int64_t M, 
     // activation) the double-buffered 256 x 256 tile hides it instead.
     if (cfg == GEMM_CFG_2CTA_512x256_CLC && !epi.identity() && g_forced.load() == GEMM_CFG_AUTO)
         cfg = GEMM_CFG_2CTA_256x256_CLC;
-    return launch_dense(st, cfg, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+    return launch_dense(st, st->status, cfg, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
 }
 
 gemm_status_t gemm_bf16_ex(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
@@ -732,7 +744,7 @@ gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const
     }
     int dev;
     DeviceState *st;
-    if ((s = current_device(dev, st, stream)) != GEMM_OK) return s;
+    if ((s = current_device_alloc(dev, st, stream)) != GEMM_OK) return s;
     if (K == 0) return launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
     if (select_mx_config(M, N) == GEMM_CFG_MXFP8_2CTA_256x256)
         return launch_mxf8<CfgMxf8Pair>(st, 1, A, sfa, B, sfb, C, M, N, K, lda, ldb, ldc, stream);
@@ -744,19 +756,27 @@ gemm_status_t gemm_check_device_status(cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_fail(e);
     int dev;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GEMM_ERR_UNSUPPORTED_DEVICE;
-    DeviceStatus *status;
+    DeviceStatus *blocks[2];
     {
         std::lock_guard<std::mutex> lock(g_mutex);
-        status = g_devices[dev].status;
+        blocks[0] = g_devices[dev].status;           // allocating entry points
+        blocks[1] = g_devices[dev].noalloc_status;   // gemm_bf16_noalloc (static scratch)
     }
-    if (!status) return GEMM_OK;   // nothing ever launched on this device
-    DeviceStatus h;
-    if ((e = cudaMemcpy(&h, status, sizeof(h), cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
-    if (h.code == 0) return GEMM_OK;
-    g_last_where = h.where;
-    g_last_block = h.block;
-    if ((e = cudaMemset(status, 0, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
-    return static_cast<gemm_status_t>(h.code);
+    // Both blocks are read and cleared; the first recorded event is reported.
+    gemm_status_t result = GEMM_OK;
+    for (DeviceStatus *status : blocks) {
+        if (!status) continue;   // that entry point never ran on this device
+        DeviceStatus h;
+        if ((e = cudaMemcpy(&h, status, sizeof(h), cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
+        if (h.code == 0) continue;
+        if ((e = cudaMemset(status, 0, sizeof(DeviceStatus))) != cudaSuccess) return cuda_fail(e);
+        if (result == GEMM_OK) {
+            g_last_where = h.where;
+            g_last_block = h.block;
+            result = static_cast<gemm_status_t>(h.code);
+        }
+    }
+    return result;
 }
 
 void gemm_last_timeout_detail(int32_t *where, int32_t *block) {
@@ -809,15 +829,12 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
         return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
                                       : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
     }
-    // The status word must start at zero for the kernel to record a timeout.
-    cudaError_t e = cudaMemsetAsync(st->status, 0, noalloc_scratch_bytes(), stream);
-    if (e != cudaSuccess) return cuda_fail(e);
     // The skinny kernel needs a workspace; without one, small-M shapes run on
     // the one-CTA 128 x 128 kernel instead.
     gemm_config_t cfg = select_config(M, N, K);
     if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128;
-    return launch_dense(st, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc, stream,
-                        b200::plain_epilogue(), 0u);
+    return launch_dense(st, st->noalloc_status, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc,
+                        stream, b200::plain_epilogue(), 0u);
 }
 
 }  // extern "C"

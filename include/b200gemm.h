@@ -22,7 +22,8 @@
  *
  * Ownership: every pointer is a DEVICE pointer owned by the caller, valid
  * until the work queued on `stream` has finished.  The library keeps, per
- * device, a small status block (allocated on the first call on a device),
+ * device, a small status block (allocated on the first call on a device of
+ * every entry point except gemm_bf16_noalloc, which uses a static array),
  * cached launch attributes and, for the skinny and block-scaled paths, a
  * workspace that grows on demand.  A workspace that a larger one replaces
  * is kept, never freed, while the library is loaded.
@@ -127,7 +128,10 @@ typedef enum {
 
 /*
  * gemm_bf16: C = A . B with bf16 A and B, fp32 accumulation in tensor memory,
- * C written as fp32 or bf16 (c_type).
+ * C written as fp32 or bf16 (c_type): the matrix product C_{MxN} = A_{MxK}
+ * B_{KxN} of "GPU 执行模型", section "Tile 的容量约束", with the argument
+ * rules of that page's section "正确性契约" (shape, stride, layout, dtype,
+ * alignment, tail predicates, accumulation and rounding, aliasing).
  *
  *   A, B     device pointers to bfloat16; C device pointer to c_type
  *   M, N, K  >= 0.  M == 0 or N == 0: nothing to do (GEMM_OK).
@@ -224,22 +228,24 @@ B200GEMM_API gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const v
  * framework's caching allocator owns the whole device memory, allocator or
  * memory-pool callbacks that must not re-enter the allocator, and latency-
  * critical loops where cudaMalloc's implicit device synchronisation is not
- * allowed.  This entry point computes exactly what gemm_bf16 computes, with
- * the same arguments, checks, kernels and configuration choice, but it
- * allocates nothing: the kernels' scratch (the 16-byte watchdog status
- * block) lives in a static 256-byte device array inside the library, which
- * every GPU that loads the library holds until the process exits.  A call
- * that would need more scratch than that array is rejected with
- * GEMM_ERR_TOO_LARGE (no shape does today: the scratch does not grow with
- * M, N or K).
+ * allowed.  This entry point computes what gemm_bf16 computes, with the same
+ * arguments, checks and kernels, but it allocates nothing: the kernels'
+ * scratch (the 16-byte watchdog status block) lives in a static 256-byte
+ * device array inside the library, which every GPU that loads the library
+ * holds until the process exits.  One difference in kernel choice: the
+ * skinny split-K kernel (GEMM_CFG_SKINNY), whose workspace gemm_bf16
+ * allocates, is replaced by GEMM_CFG_1CTA_128x128, so small-M, long-K shapes
+ * run slower here.  A call that would need more scratch than that array is
+ * rejected with GEMM_ERR_TOO_LARGE (no shape does today: the scratch does
+ * not grow with M, N or K).  Each call queues exactly one kernel.
  *
  * The first call on each device does a one-time set-up with that device
  * current (it looks up the array's device address and zeroes it); make that
- * first call before any stream capture.  Each call clears the status word
- * on `stream` before its kernel.  All calls share the one array, so
- * calls that overlap on the GPU (different streams, no ordering) race on it.
- * Watchdog timeouts of this entry point are recorded in that array and are
- * not reported by gemm_check_device_status().
+ * first call before any stream capture.  The status block then keeps a
+ * recorded watchdog timeout until gemm_check_device_status() reads and
+ * clears it, exactly as for the other entry points.  All calls share the one
+ * array, so calls that overlap on the GPU (different streams, no ordering)
+ * race on it.
  */
 B200GEMM_API gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C,
                                              int64_t M, int64_t N, int64_t K,
@@ -247,16 +253,26 @@ B200GEMM_API gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void 
                                              gemm_out_t c_type, cudaStream_t stream);
 
 /* Synchronises `stream`, then reports and clears the device watchdog status
- * of the current device: GEMM_OK, or GEMM_ERR_TIMEOUT if a kernel's bounded
- * wait expired since the last check.  GEMM_ERR_LAUNCH if the stream itself
- * reports a CUDA error. */
+ * of the current device (the status blocks of every entry point, the static
+ * one of gemm_bf16_noalloc included): GEMM_OK, or GEMM_ERR_TIMEOUT if a
+ * kernel's bounded wait expired since the last check.  GEMM_ERR_LAUNCH if
+ * the stream itself reports a CUDA error.  It serves two items of the
+ * correctness contract of "GPU 执行模型", section "正确性契约": the
+ * lifetime of the stream's asynchronous work (it returns once that work has
+ * finished) and the barrier happens-before of the shared-memory stages (the
+ * kernels bound every barrier wait, and an expired one is what it reports).
+ * The device watchdog itself has no counterpart in the pages. */
 B200GEMM_API gemm_status_t gemm_check_device_status(cudaStream_t stream);
 
 /* Detail of the last watchdog event read by gemm_check_device_status():
- * which wait expired (role * 16 + barrier kind) and in which CTA; -1 if none. */
+ * which wait expired (role * 16 + barrier kind) and in which CTA; -1 if none.
+ * (No counterpart in the pages.) */
 B200GEMM_API void gemm_last_timeout_detail(int32_t *where, int32_t *block);
 
-/* Static description of a status code. */
+/* Static description of a status code.  The codes name the argument checks
+ * of the correctness contract ("GPU 执行模型", section "正确性契约": shape,
+ * stride, alignment, aliasing, stream and capture rules) plus the library's
+ * own launch and watchdog failures, which have no counterpart in the pages. */
 B200GEMM_API const char *gemm_status_string(gemm_status_t status);
 
 /* The CUDA error behind the last GEMM_ERR_LAUNCH on this host thread. */

@@ -136,3 +136,27 @@ def test_fused_workloads_use_their_activation_in_the_oracle_leg():
         want = oracle.epilogue(base, None, 1.0, 0.0, p.bias.astype(np.float64), act)
         assert np.array_equal(got, want)
     assert bench.metric_of("fused") == bench.METRIC_FUSED and bench.metric_of("mxfp8") == bench.METRIC_MXFP8
+
+
+def test_roofline_takes_the_larger_of_compute_and_bandwidth():
+    # 8192^3: 1.1e12 FLOP over 1686 TFLOP/s (652 us) outweighs 537 MB over 6549 GB/s (82 us)
+    r = bench.roofline_of(2.0 * 8192 ** 3, 536870912, 0.72e-3, 1686.0, 6549.0)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["frac"] - (2.0 * 8192 ** 3 / 1686e12) / 0.72e-3) < 1e-12
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    # 16 x 8192 x 8192: 2.1 GFLOP (1.3 us) against 135 MB (20.6 us): HBM-bound
+    nbytes = 2 * (16 * 8192 + 8192 * 8192) + 4 * 16 * 8192
+    r = bench.roofline_of(2.0 * 16 * 8192 * 8192, nbytes, 40e-6, 1686.0, 6549.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    assert 0.5 < r["frac"] < 0.53
+
+
+def test_config_set_covers_every_named_configuration():
+    shapes = {bench.WORKLOADS[n][:3] for n in bench.CONFIG_SET} | {bench.WORKLOADS["square8192"][:3]}
+    for want in [(128, 128, 128), (4096, 4096, 4096), (8192, 8192, 8192), (4000, 3000, 2000),
+                 (1000, 8192, 8192), (16, 8192, 8192)]:
+        assert want in shapes
+    assert bench.WORKLOADS["mxfp8_8192"][3] == "mxfp8" and "mxfp8_8192" in bench.CONFIG_SET
+    p = bench.Problem("square4096_bf16", (8, 8, 32), 0)
+    assert p.bf16_out and p.out_bytes == 2 * 8 * 8

@@ -6,8 +6,12 @@ kernel frees TMEM and exits, and gemm_check_device_status() reports
 GEMM_ERR_TIMEOUT with the role and CTA.  The context stays usable: the next
 call on the same stream is correct.
 
-Runs in a child process so that the short watchdog limit (read once when the
-library starts) applies only there."""
+The switch, B200GEMM_INJECT_TIMEOUT, is a per-launch mask ('1' = inject into
+that launch) that the library reads once; the short watchdog limit is read
+once too.  Both are set in a child process's environment, so they apply only
+there.  The child alternates an injected and a clean launch per
+configuration, then does the same through gemm_bf16_noalloc, whose status
+block is the library's static scratch array."""
 import os
 import subprocess
 import sys
@@ -17,6 +21,8 @@ import pytest
 
 pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CFGS = ("1cta_128x128", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc")
 
 CHILD = textwrap.dedent(r"""
     import os, sys, time
@@ -30,31 +36,33 @@ CHILD = textwrap.dedent(r"""
     A, B = to_device_bf16(a), to_device_bf16(b)
     C = torch.zeros((M, N), dtype=torch.float32, device="cuda")
     ref, s = oracle.gemm_bf16_f64(a, b, with_abs=True)
-    for cfg in ("1cta_128x128", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc"):
+    entries = [(cfg, G.gemm_bf16) for cfg in sys.argv[2].split(",")] + [("auto", G.gemm_bf16_noalloc)]
+    for cfg, fn in entries:
+        name = fn.__name__ + ":" + cfg
         G.gemm_force_config(cfg)
-        os.environ["B200GEMM_INJECT_TIMEOUT"] = "1"
         t0 = time.time()
-        G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_F32)
+        fn(A, B, C, M, N, K, K, K, N, G.OUT_F32)          # injected launch
         st = G.gemm_check_device_status(check=False)
         dt = time.time() - t0
         where, block = G.gemm_last_timeout_detail()
-        assert st == 6, (cfg, st)
-        assert where == 2 * 16 + 1 and block == 0, (cfg, where, block)   # MMA warp, full barrier, CTA 0
+        assert st == 6, (name, st)
+        assert where == 2 * 16 + 1 and block == 0, (name, where, block)   # MMA warp, full barrier, CTA 0
         assert dt < 5.0, dt
-        os.environ["B200GEMM_INJECT_TIMEOUT"] = "0"
+        assert G.gemm_check_device_status(check=False) == 0, name        # reading cleared it
         C.zero_()
-        G.gemm_bf16(A, B, C, M, N, K, K, K, N, G.OUT_F32)
-        assert G.gemm_check_device_status(check=False) == 0
+        fn(A, B, C, M, N, K, K, K, N, G.OUT_F32)          # clean launch
+        assert G.gemm_check_device_status(check=False) == 0, name
         got = C.cpu().numpy().astype(np.float64)
-        assert np.all(np.abs(got - ref) <= 1e-3 * s + 1e-6), cfg
-        print(cfg, "timeout reported in %.3f s, next call correct" % dt, flush=True)
+        assert np.all(np.abs(got - ref) <= 1e-3 * s + 1e-6), name
+        print(name, "timeout reported in %.3f s, next call correct" % dt, flush=True)
     print("watchdog ok")
 """)
 
 
 def test_dropped_arrival_times_out_cleanly_and_context_survives():
-    env = dict(os.environ, B200GEMM_WATCHDOG_MS="100")
-    out = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True,
-                         timeout=300)
+    launches = len(CFGS) + 1                  # four configurations, then gemm_bf16_noalloc
+    env = dict(os.environ, B200GEMM_WATCHDOG_MS="100", B200GEMM_INJECT_TIMEOUT="10" * launches)
+    out = subprocess.run([sys.executable, "-c", CHILD, ROOT, ",".join(CFGS)], env=env, capture_output=True,
+                         text=True, timeout=300)
     assert out.returncode == 0, out.stdout + out.stderr
     assert "watchdog ok" in out.stdout
