@@ -368,14 +368,24 @@ def min_bytes(p: Problem) -> int:
     return p.in_bytes + p.out_bytes
 
 
-def time_steps(p: Problem, G, dev, C, torch, stream, steps: int, scratch=None):
+def flush_l2(scratch, clean: bool = True):
+    """Evict L2 before a timed call: write a buffer twice the L2's size; with
+    `clean`, read it back too, so that the write-backs of the dirty lines the
+    write leaves behind happen here, outside the timed events, instead of
+    inside the next call (which would then pay for the flush's own traffic)."""
+    scratch.zero_()
+    if clean:
+        scratch.sum()
+
+
+def time_steps(p: Problem, G, dev, C, torch, stream, steps: int, scratch=None, clean: bool = True):
     """Device time of each of `steps` calls (ms).  With `scratch`, L2 is
-    flushed before every call by writing that buffer outside the events."""
+    flushed (flush_l2) before every call, outside the events."""
     if scratch is not None:
         ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         for i in range(steps):
-            scratch.zero_()
+            flush_l2(scratch, clean)
             ev_s[i].record(stream)
             p.call(G, dev, C, stream)
             ev_e[i].record(stream)
@@ -399,7 +409,7 @@ def graph_replay_us(p: Problem, G, dev, C, torch, stream, steps: int, scratch) -
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):
-        scratch.zero_()
+        flush_l2(scratch)
         ev_s[i].record(stream)
         g.replay()
         ev_e[i].record(stream)
@@ -426,6 +436,8 @@ def config_report(G, torch, stream, peaks: dict, steps: int, warmup: int) -> dic
         G.gemm_check_device_status(stream)
         flush = needs_l2_flush(min_bytes(p))
         per_step, _ = time_steps(p, G, dev, C, torch, stream, steps, scratch if flush else None)
+        # the same with the write-only flush: L2 left full of dirty lines
+        dirty = time_steps(p, G, dev, C, torch, stream, steps, scratch, clean=False)[0] if flush else None
         G.gemm_check_device_status(stream)
         med = statistics.median(per_step) * 1e-3
         ratio = FP8_OVER_BF16 if p.kind == "mxfp8" else 1.0
@@ -434,11 +446,14 @@ def config_report(G, torch, stream, peaks: dict, steps: int, warmup: int) -> dic
         nominal = roofline_of(p.flops, min_bytes(p), med, NOMINAL["bf16_tflops"] * ratio, NOMINAL["hbm_gbs"])
         entry = {"workload": p.desc, "M": p.M, "N": p.N, "K": p.K, "kernel_config": config_name(G, p, "auto"),
                  "launches_per_call": p.launches(G), "steps": steps,
-                 "l2": "flushed before every call" if flush else "no flush (inputs+output > 2 x L2)",
+                 "l2": ("flushed before every call (252 MiB written, then read back)" if flush else
+                        "no flush (inputs+output > 2 x L2)"),
                  "median_us": med * 1e6, "p90_us": float(np.percentile(per_step, 90)) * 1e3,
                  "tflops": p.flops / med / 1e12, "gbs": min_bytes(p) / med / 1e9,
                  "bound": measured["bound"], "roofline_us": measured["roofline_us"], "frac": measured["frac"],
                  "frac_of_nominal": nominal["frac"], "min_bytes": min_bytes(p)}
+        if dirty:
+            entry["median_us_after_dirty_flush"] = statistics.median(dirty) * 1e3
         if name == "single_tile128":
             # one 128 x 128 tile: launch latency, not a roofline, bounds it
             entry["bound"] = "latency"
@@ -693,7 +708,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": p.desc, "M": p.M, "N": p.N, "K": p.K, "kernel_config": cfg_name,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": (f"flushed between steps ({2 * L2_BYTES // 2**20} MiB written outside the events): "
+                   "l2": (f"flushed between steps ({2 * L2_BYTES // 2**20} MiB written, then read back, outside "
+                          f"the events): "
                           f"inputs+output {traffic_bytes / 2**20:.0f} MiB < 2 x 126 MiB L2" if flush else
                           f"no flush: inputs+output {traffic_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2"),
                    "step_ms_median": statistics.median(per_step_ms),
