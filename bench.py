@@ -404,8 +404,11 @@ def graph_replay_us(p: Problem, G, dev, C, torch, stream, steps: int, scratch) -
     """Median device time (us) of one call captured in a CUDA graph and
     replayed, L2 flushed before each replay outside the events."""
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        p.call(G, dev, C, torch.cuda.current_stream())
+    side = torch.cuda.Stream()              # capture needs a stream other than the default one
+    side.wait_stream(stream)
+    with torch.cuda.graph(g, stream=side):
+        p.call(G, dev, C, side)
+    stream.wait_stream(side)
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):

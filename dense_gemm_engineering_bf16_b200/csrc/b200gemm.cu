@@ -39,6 +39,11 @@ using Cfg1x256B16C = b200::GemmBf16Cfg<1, 256, 4, 1, true>;
 // two MMA consumers sharing B: 512 x 256 pair tiles, single-buffered TMEM
 using Cfg2x512F32C = b200::GemmBf16Cfg<2, 256, 4, 0, true, 2>;
 using Cfg2x512B16C = b200::GemmBf16Cfg<2, 256, 4, 1, true, 2>;
+// stream-K over the (tile, K block) iterations: pair tiles 256 x 256, static grid
+using Cfg2x256F32S = b200::GemmBf16Cfg<2, 256, 6, 0, false, 1, true>;
+using Cfg2x256B16S = b200::GemmBf16Cfg<2, 256, 6, 1, false, 1, true>;
+// pair tiles 256 x 224 (fp32 C: 7 chunks of 32 columns), static grid
+using Cfg2x224F32 = b200::GemmBf16Cfg<2, 224, 6, 0>;
 using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
@@ -115,6 +120,17 @@ int raster_group_m() {
         return v > 0 ? v : 8;
     }();
     return g;
+}
+
+// K order of the dense kernels' tiles: serpentine (odd waves of tiles walk K
+// backwards, reusing the K slices the previous wave left in L2) unless
+// B200GEMM_SERPENTINE=0.
+bool serpentine_k() {
+    static const bool on = [] {
+        const char *s = std::getenv("B200GEMM_SERPENTINE");
+        return !(s && s[0] == '0');
+    }();
+    return on;
 }
 
 // Test-only: B200GEMM_INJECT_TIMEOUT holds one character per launch of the
@@ -274,8 +290,21 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     // under the power cap buys clock); fewer: the double-buffered 256 x 256
     const int64_t tall_tiles = ((M + 511) / 512) * ((N + 255) / 256);
     if (tall_tiles >= 148) return GEMM_CFG_2CTA_512x256_CLC;
-    if (pair_tiles >= 148) return GEMM_CFG_2CTA_256x256_CLC;
-    if (pair_tiles >= 74) return GEMM_CFG_2CTA_256x256;
+    if (pair_tiles >= 74) {
+        // The last wave of pair tiles: when it leaves more than a tenth of
+        // the pairs idle, either 256 x 224 tiles fill the waves better
+        // (e.g. 1000 x 8192: 148 tiles, two full waves, against 128 tiles in
+        // two waves of 256 x 256), or, with operands small enough to stay in
+        // L2, stream-K gives every pair an equal share of the iterations.
+        const int64_t waves = (pair_tiles + 73) / 74;
+        if (pair_tiles * 10 < waves * 74 * 9) {
+            const int64_t tiles224 = ((M + 255) / 256) * ((N + 223) / 224);
+            const int64_t waves224 = (tiles224 + 73) / 74;
+            if (waves224 * 224 * 100 <= waves * 256 * 92) return GEMM_CFG_2CTA_256x224;
+            if (2 * (M + N) * K <= (int64_t(96) << 20) && K >= 512) return GEMM_CFG_2CTA_256x256_SK;
+        }
+        return pair_tiles >= 148 ? GEMM_CFG_2CTA_256x256_CLC : GEMM_CFG_2CTA_256x256;
+    }
     // few rows, too few tiles to fill the SMs, and a long K to split: stream-K.
     // (A short K gains nothing from splitting; the plain 128 x 128 kernel has
     // the lower fixed cost there: 4.8 vs 9.6 us at 128^3 under graph replay.)
@@ -284,6 +313,8 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     if (wide_tiles >= 148) return GEMM_CFG_1CTA_128x256;
     return GEMM_CFG_1CTA_128x128;
 }
+
+gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStream_t stream);
 
 // `status`: the watchdog status block the kernel records a timeout in.
 template <class Cfg>
@@ -349,12 +380,34 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     // Static schedule: as many clusters as fit at once, each striding over
     // the tiles.  CLC: one cluster per tile; running clusters claim the rest.
-    const int64_t clusters = Cfg::CLC ? tiles
-                                      : (tiles < st->max_clusters[cfg_id][oi] ? tiles : st->max_clusters[cfg_id][oi]);
+    // Stream-K: every co-resident cluster, each with an equal share of the
+    // (tile, K block) iterations.
+    const int64_t resident = st->max_clusters[cfg_id][oi];
+    const int64_t clusters = Cfg::CLC ? tiles : (Cfg::SK || tiles > resident ? resident : tiles);
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
+    // tiles that run at the same time: one wave (for CLC, as many clusters
+    // as fit on the SMs at once); stream-K keeps K ascending
+    const int wave_tiles = (serpentine_k() && !Cfg::SK) ? static_cast<int>(resident) : 0;
+    // Stream-K workspace: two [128][BN] fp32 partial slots per CTA (the
+    // first and the last tile of its range may be split), then one 64-bit
+    // arrival counter per (tile, CTA of the cluster).
+    float *sk_partials = nullptr;
+    unsigned long long *sk_counters = nullptr;
+    uint32_t epoch = 0;
+    if constexpr (Cfg::SK) {
+        const int64_t partial_bytes = clusters * Cfg::CG * 2 * 128 * Cfg::BN * 4;
+        uint8_t *ws = nullptr;
+        if ((s = sk_workspace(st, static_cast<size_t>(partial_bytes + tiles * Cfg::CG * 8), ws, stream)) != GEMM_OK)
+            return s;
+        sk_partials = reinterpret_cast<float *>(ws);
+        sk_counters = reinterpret_cast<unsigned long long *>(ws + partial_bytes);
+        std::lock_guard<std::mutex> lock(g_mutex);
+        epoch = ++st->sk_epoch;
+        if (epoch == 0) epoch = ++st->sk_epoch;
+    }
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
-                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), status,
-                           watchdog_ns(K), inject_flags(), epi, layout);
+                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), wave_tiles, status,
+                           watchdog_ns(K), inject_flags(), epi, layout, sk_partials, sk_counters, epoch);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -370,12 +423,12 @@ struct SkinnyLayout {
 template <class Cfg>
 SkinnyLayout skinny_layout(int64_t N, int64_t K, int sm_count) {
     SkinnyLayout l;
-    const int64_t kb = (K + Cfg::BK - 1) / Cfg::BK;
+    const int64_t kb = (K + Cfg::SK - 1) / Cfg::SK;    // iterations (stages of SK) per tile
     l.tiles = (N + Cfg::TILE_N - 1) / Cfg::TILE_N;
     const int64_t total = l.tiles * kb;
-    // at least kMinIters K blocks per CTA: a CTA with fewer barely fills its
+    // at least 8 64-wide K blocks per CTA: a CTA with fewer barely fills its
     // pipeline, and a tile cut into many slivers costs a long fix-up
-    constexpr int64_t kMinIters = 8;
+    constexpr int64_t kMinIters = 8 / Cfg::KBS > 0 ? 8 / Cfg::KBS : 1;
     const int64_t want = (total + kMinIters - 1) / kMinIters;
     l.grid = want < sm_count ? want : sm_count;
     const int64_t per = (total + l.grid - 1) / l.grid;
@@ -511,6 +564,14 @@ gemm_status_t launch_dense(DeviceState *st, DeviceStatus *status, gemm_config_t 
         case GEMM_CFG_2CTA_512x256_CLC:
             return f32 ? launch_bf16<Cfg2x512F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                        : launch_bf16<Cfg2x512B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_2CTA_256x256_SK:
+            return f32 ? launch_bf16<Cfg2x256F32S>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16S>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_2CTA_256x224:
+            // 224 columns are 3.5 chunks of 64 bf16: bf16 C takes 256 x 256
+            return f32 ? launch_bf16<Cfg2x224F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_bf16<Cfg2x256B16>(st, status, GEMM_CFG_2CTA_256x256, A, B, C, M, N, K, lda, ldb, ldc,
+                                                  stream, epi, layout);
         case GEMM_CFG_1CTA_128x256_CLC:
             return f32 ? launch_bf16<Cfg1x256F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                        : launch_bf16<Cfg1x256B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
@@ -829,10 +890,12 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
         return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
                                       : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
     }
-    // The skinny kernel needs a workspace; without one, small-M shapes run on
-    // the one-CTA 128 x 128 kernel instead.
+    // The skinny and stream-K kernels need a workspace; without one, small-M
+    // shapes run on the one-CTA 128 x 128 kernel and stream-K shapes on the
+    // CLC pair kernel instead.
     gemm_config_t cfg = select_config(M, N, K);
     if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128;
+    if (cfg == GEMM_CFG_2CTA_256x256_SK) cfg = GEMM_CFG_2CTA_256x256_CLC;   // stream-K needs a workspace too
     return launch_dense(st, st->noalloc_status, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc,
                         stream, b200::plain_epilogue(), 0u);
 }

@@ -37,16 +37,20 @@
 
 namespace b200 {
 
-template <int MP_, int STAGES_, int OUT_>
+template <int MP_, int STAGES_, int OUT_, int KBS_ = 1>
 struct GemmSkinnyCfg {
     static constexpr int MP = MP_;                 // max padded rows of A (MMA N)
     static constexpr int STAGES = STAGES_;
     static constexpr int OUT = OUT_;               // 0: f32 C, 1: bf16 C
     static constexpr int TILE_N = 128;             // rows of B per tile (MMA M)
-    static constexpr int BK = 64;
+    static constexpr int BK = 64;                  // K per box (one 128-byte swizzle row)
+    static constexpr int KBS = KBS_;               // boxes (64-wide K blocks) per stage
+    static constexpr int SK = BK * KBS;            // K per stage, the stream-K iteration unit
     static constexpr int UMMA_K = 16;
-    static constexpr int B_BYTES = TILE_N * BK * 2;
-    static constexpr int A_BYTES = MP * BK * 2;
+    static constexpr int B_BOX = TILE_N * BK * 2;
+    static constexpr int A_BOX = MP * BK * 2;
+    static constexpr int B_BYTES = KBS * B_BOX;
+    static constexpr int A_BYTES = KBS * A_BOX;
     static constexpr int STAGE_BYTES = B_BYTES + A_BYTES;
     static constexpr int TMEM_COLS = pow2_at_least(2 * MP, 32);
     static constexpr int NUM_BARS = 2 * STAGES + 4;
@@ -54,7 +58,7 @@ struct GemmSkinnyCfg {
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
     static constexpr int THREADS = 192;
     static_assert(MP % 16 == 0 && MP >= 16 && MP <= 256, "MMA N for M = 128");
-    static_assert(STAGE_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+    static_assert(STAGE_BYTES % 1024 == 0 && A_BOX % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
 };
@@ -67,10 +71,6 @@ __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t total, int64_t
 // The CTA whose range holds iteration `it`.
 __device__ __forceinline__ int64_t range_owner(int64_t it, int64_t total, int64_t g) {
     return ((it + 1) * g + total - 1) / total - 1;
-}
-
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -242,7 +242,8 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot_ptr;
 
-    const int64_t kb_per_tile = (K + Cfg::BK - 1) / Cfg::BK;
+    // iterations: (tile of 128 rows of B, stage of SK = KBS x 64 K), K fastest
+    const int64_t kb_per_tile = (K + Cfg::SK - 1) / Cfg::SK;
     const int64_t tiles = (N + Cfg::TILE_N - 1) / Cfg::TILE_N;
     const int64_t total = tiles * kb_per_tile;
     const int64_t g = gridDim.x;
@@ -254,7 +255,8 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
-            const uint32_t tx = static_cast<uint32_t>(Cfg::B_BYTES + mpad * Cfg::BK * 2);
+            const uint32_t box_tx = static_cast<uint32_t>(Cfg::B_BOX + mpad * Cfg::BK * 2);
+            const int k_boxes = (K + Cfg::BK - 1) / Cfg::BK;
             // Each byte of B is read once: evict_first keeps the stream from
             // displacing A and the split-tile partials in L2 (measured: 38.9
             // vs 43.1 us per 16 x 8192 x 8192 step).
@@ -271,10 +273,17 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 }
                 const uint32_t b_dst = base + stage * Cfg::STAGE_BYTES;
                 const uint32_t a_dst = b_dst + Cfg::B_BYTES;
-                mbar_arrive_expect_tx(full_bar(stage), tx);
-                load_operand_tile<1, true>(b_dst, &tmB, full_bar(stage), kb * Cfg::BK, t * Cfg::TILE_N, Cfg::TILE_N,
-                                           b_mn, stream_b);
-                tma_load_2d(a_dst, &tmA, full_bar(stage), kb * Cfg::BK, 0);
+                // the stage's boxes back to back: for every row of B, up to
+                // KBS adjacent 128-byte pieces are requested close together;
+                // boxes wholly past K (the last stage of a tile) are skipped
+                const int nbox = min(Cfg::KBS, k_boxes - kb * Cfg::KBS);
+                mbar_arrive_expect_tx(full_bar(stage), static_cast<uint32_t>(nbox) * box_tx);
+                for (int j = 0; j < nbox; ++j)
+                    load_operand_tile<1, true>(b_dst + j * Cfg::B_BOX, &tmB, full_bar(stage),
+                                               (kb * Cfg::KBS + j) * Cfg::BK, t * Cfg::TILE_N, Cfg::TILE_N, b_mn,
+                                               stream_b);
+                for (int j = 0; j < nbox; ++j)
+                    tma_load_2d(a_dst + j * Cfg::A_BOX, &tmA, full_bar(stage), (kb * Cfg::KBS + j) * Cfg::BK, 0);
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
             }
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
@@ -290,6 +299,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
         // --------------------------------------------------- MMA issuer --
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(Cfg::TILE_N, mpad, b_mn ? 1u : 0u, 0u);
+            const int k_boxes = (K + Cfg::BK - 1) / Cfg::BK;
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             int seg = 0;
@@ -312,12 +322,17 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t b0 = base + stage * Cfg::STAGE_BYTES;
-                    const uint32_t a0 = b0 + Cfg::B_BYTES;
+                    const uint32_t bs = base + stage * Cfg::STAGE_BYTES;
+                    const uint32_t as = bs + Cfg::B_BYTES;
+                    const int nbox = min(Cfg::KBS, k_boxes - static_cast<int>(j - t * kb_per_tile) * Cfg::KBS);
+                    for (int q = 0; q < nbox; ++q) {
+                        const uint32_t b0 = bs + q * Cfg::B_BOX;
+                        const uint32_t a0 = as + q * Cfg::A_BOX;
 #pragma unroll
-                    for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
-                        mma_bf16_ss<1>(d_tmem, operand_desc(b0, kk, b_mn), sw128_kmajor_desc(a0 + kk * 32),
-                                       idesc, (j != it || kk != 0) ? 1u : 0u);
+                        for (int kk = 0; kk < Cfg::BK / Cfg::UMMA_K; ++kk) {
+                            mma_bf16_ss<1>(d_tmem, operand_desc(b0, kk, b_mn), sw128_kmajor_desc(a0 + kk * 32),
+                                           idesc, (j != it || q != 0 || kk != 0) ? 1u : 0u);
+                        }
                     }
                     mma_commit<1>(empty_bar(stage), 0);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }

@@ -81,9 +81,13 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     return p;
 }
 
-template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1>
+template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1, bool SK_ = false>
 struct GemmBf16Cfg {
     static constexpr bool CLC = CLC_;              // tiles from Cluster Launch Control, not a fixed stride
+    // Stream-K: the (tile, K block) iterations are cut into one contiguous
+    // range per cluster; a tile split between clusters is summed from fp32
+    // partials by the last of its contributors, in contributor order.
+    static constexpr bool SK = SK_;
     static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
     static constexpr int BN = BN_;                 // tile N == MMA N
     static constexpr int STAGES = STAGES_;         // shared-memory ring depth
@@ -119,6 +123,7 @@ struct GemmBf16Cfg {
 
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
     static_assert(CONSUMERS == 1 || CONSUMERS == 2, "one or two MMA consumers");
+    static_assert(!SK || (!CLC && CONSUMERS == 1 && BN % 4 == 0), "stream-K: static schedule, one consumer");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
     static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows <= 256, whole 8-row swizzle atoms");
     static_assert(BN % EPI_COLS == 0, "epilogue chunks cover the tile");
@@ -193,14 +198,103 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk, bool mn)
     return mn ? sw128_mnmajor_desc(base + 2048u * kk) : sw128_kmajor_desc(base + 32u * kk);
 }
 
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// C[row][col .. col + 3] = finish(v, C_old, bias) for the columns below N.
+template <int OUT>
+__device__ __forceinline__ void store4_c(void *C, int64_t ldc, int row, int col, float (&v)[4], int N,
+                                         const Epilogue &epi) {
+    const int64_t i = static_cast<int64_t>(row) * ldc + col;
+    if (!epi.identity()) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (col + q >= N) break;
+            float old = 0.0f;
+            if (epi.beta != 0.0f) {
+                if constexpr (OUT == 0) old = static_cast<const float *>(C)[i + q];
+                else old = __bfloat162float(static_cast<const __nv_bfloat16 *>(C)[i + q]);
+            }
+            v[q] = finish(v[q], old, epi.bias ? __ldg(epi.bias + col + q) : 0.0f, epi);
+        }
+    }
+    if (col + 4 <= N) {
+        if constexpr (OUT == 0) {
+            *reinterpret_cast<float4 *>(static_cast<float *>(C) + i) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(C) + i) =
+                make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (col + q >= N) break;
+            if constexpr (OUT == 0) static_cast<float *>(C)[i + q] = v[q];
+            else static_cast<__nv_bfloat16 *>(C)[i + q] = __float2bfloat16_rn(v[q]);
+        }
+    }
+}
+
+// Stream-K fix-up by the last contributor of a split tile, for this CTA's
+// 128 rows: C rows [row0, row0 + 128) x columns [col0, col0 + BN) = the sum
+// of the contributors' fp32 partials ([128][BN] each, `part(cc)`) in
+// contributor order c_lo, c_lo + 1, ..., then the epilogue.  128 threads;
+// thread `tid` owns four consecutive columns and every (128 / (BN / 4))-th
+// row; each round keeps 8 rows x 2 contributors of float4 loads in flight.
+template <int OUT, int BN, class PartFn>
+__device__ __forceinline__ void sk_fixup(PartFn part, int64_t c_lo, int64_t c_hi, int row0, int col0, int M,
+                                         int N, void *C, int64_t ldc, uint32_t tid, const Epilogue &epi) {
+    constexpr int TPR = BN / 4;          // threads per row
+    constexpr int RPP = 128 / TPR;       // rows per pass of the 128 threads
+    constexpr int ROWS = 8;
+    static_assert(128 % TPR == 0 && (128 / RPP) % ROWS == 0, "fix-up thread layout");
+    const int c4 = static_cast<int>(tid % TPR) * 4;
+    const int r_first = static_cast<int>(tid / TPR);
+    const int col = col0 + c4;
+    for (int rb = 0; rb < 128 / RPP; rb += ROWS) {
+        float4 acc[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int64_t cc = c_lo; cc <= c_hi; cc += 2) {
+            const bool two = cc + 1 <= c_hi;
+            const float *p0 = part(cc) + c4;
+            const float *p1 = two ? part(cc + 1) + c4 : p0;
+            float4 v0[ROWS], v1[ROWS];
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const int lr = r_first + RPP * (rb + r);
+                v0[r] = __ldcg(reinterpret_cast<const float4 *>(p0 + static_cast<int64_t>(lr) * BN));
+                v1[r] = two ? __ldcg(reinterpret_cast<const float4 *>(p1 + static_cast<int64_t>(lr) * BN))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                acc[r].x += v0[r].x; acc[r].y += v0[r].y; acc[r].z += v0[r].z; acc[r].w += v0[r].w;
+                if (two) {
+                    acc[r].x += v1[r].x; acc[r].y += v1[r].y; acc[r].z += v1[r].z; acc[r].w += v1[r].w;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            const int row = row0 + r_first + RPP * (rb + r);
+            if (row >= M || col >= N) continue;
+            float v[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
+            store4_c<OUT>(C, ldc, row, col, v, N, epi);
+        }
+    }
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC,
-                       int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m,
+                       int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m, int wave_tiles,
                        DeviceStatus *status, uint64_t timeout_ns, uint32_t inject,
-                       Epilogue epi, uint32_t layout) {
+                       Epilogue epi, uint32_t layout,
+                       float *sk_partials, unsigned long long *sk_counters, uint32_t sk_epoch) {
     constexpr int CG = Cfg::CG;
     const bool a_mn = (layout & kLayoutAMajorM) != 0;   // A stored K x M
     const bool b_mn = (layout & kLayoutBMajorN) != 0;   // B stored K x N
@@ -229,6 +323,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
     volatile uint32_t *abort_flag = tmem_slot_ptr + 1;
     volatile int32_t *tile_id_ptr = reinterpret_cast<volatile int32_t *>(tmem_slot_ptr + 2);
+    volatile uint32_t *sk_last_flag = tmem_slot_ptr + 12;  // after the CLC answers
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -295,6 +390,50 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         }
     };
 
+    // Work units: K blocks [kb0, kb1) of one tile.  Static and CLC
+    // schedules: whole tiles from next_tile.  Stream-K: the pieces of this
+    // cluster's range [it_begin, it_end) of the (tile, K block) iterations
+    // (K fastest), one piece per tile the range touches.
+    struct Unit {
+        int tile, kb0, kb1;
+    };
+    const int64_t sk_total = static_cast<int64_t>(num_tiles) * num_kb;
+    const int64_t it_begin = Cfg::SK ? (static_cast<int64_t>(cluster_id) * sk_total) / num_clusters : 0;
+    const int64_t it_end = Cfg::SK ? (static_cast<int64_t>(cluster_id + 1) * sk_total) / num_clusters : 0;
+    auto sk_unit = [&](int64_t it) -> Unit {
+        Unit u;
+        u.tile = static_cast<int>(it / num_kb);
+        const int64_t t0 = static_cast<int64_t>(u.tile) * num_kb;
+        u.kb0 = static_cast<int>(it - t0);
+        u.kb1 = static_cast<int>(min(it_end, t0 + num_kb) - t0);
+        return u;
+    };
+    auto first_unit = [&](Unit &u) -> bool {
+        if constexpr (Cfg::SK) {
+            if (it_begin >= it_end) return false;
+            u = sk_unit(it_begin);
+            return true;
+        } else {
+            u = Unit{cluster_id, 0, num_kb};
+            return cluster_id < num_tiles;
+        }
+    };
+    // j counts the units this role has finished (the CLC ring position)
+    auto next_unit = [&](Unit &u, uint32_t j, bool &ok) -> bool {
+        if constexpr (Cfg::SK) {
+            (void)j;
+            (void)ok;
+            const int64_t it = static_cast<int64_t>(u.tile) * num_kb + u.kb1;
+            if (it >= it_end) return false;
+            u = sk_unit(it);
+            return true;
+        } else {
+            const int n = next_tile(u.tile, j, ok);
+            u = Unit{n, 0, num_kb};
+            return n >= 0;
+        }
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
@@ -303,12 +442,19 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t leader_rank = 0;
             uint32_t fetched = 0;
 
-            for (int tile = cluster_id; ok && tile >= 0;) {
+            Unit u;
+            for (bool more = first_unit(u); ok && more;) {
+                const int tile = u.tile;
                 int tm, tn;
                 raster_tile(tile, num_m, num_n, group_m, tm, tn);
                 const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;   // + c * BM_MMA
                 const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                // Serpentine K: tiles of odd waves (tile / wave_tiles) walk K
+                // backwards, so a new wave starts on the K slices of A and B
+                // that the wave before it read last, which are still in L2.
+                // The order is fixed per tile, so results stay deterministic.
+                const bool rev = !Cfg::SK && wave_tiles > 0 && ((tile / wave_tiles) & 1) != 0;
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarEmpty);
                         ok = false;
@@ -316,8 +462,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     const uint32_t a_dst = base + stage * Cfg::STAGE_BYTES;
                     const uint32_t b_dst = a_dst + Cfg::A_BYTES;
-                    const int kx = kb * Cfg::BK;
-                    if ((inject & kInjectDropFirstStage) && blockIdx.x == 0 && fetched == 0 && kb == 0) {
+                    const int kx = (rev ? num_kb - 1 - kb : kb) * Cfg::BK;
+                    if ((inject & kInjectDropFirstStage) && blockIdx.x == 0 && fetched == 0 && kb == u.kb0) {
                         // Failure-detection test: this stage's full barrier is
                         // never armed, so the MMA's bounded wait on it expires.
                         if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -339,7 +485,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tile = next_tile(tile, fetched++, ok);
+                more = next_unit(u, fetched++, ok);
                 if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarSched);
             }
             // Tail: every stage handed out must be released by the MMA before
@@ -369,7 +515,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             int t = 0;
-            for (int tile = cluster_id; ok && tile >= 0; ++t) {
+            Unit u;
+            for (bool more = first_unit(u); ok && more; ++t) {
                 const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
                 const uint32_t acc_phase = (static_cast<uint32_t>(t) / Cfg::ACC_BUFS) & 1u;
                 if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, 3 * timeout_ns)) {
@@ -379,7 +526,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + buf * Cfg::CONSUMERS * Cfg::BN;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarFull);
                         ok = false;
@@ -394,14 +541,14 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         for (int c = 0; c < Cfg::CONSUMERS; ++c)   // both consumers read this B k-step
                             mma_bf16_ss<CG>(d_tmem + c * Cfg::BN,
                                             a_desc0 + soff + (c * Cfg::A_PART_BYTES >> 4) + kk * a_kstep, bd, idesc,
-                                            (kb | kk) != 0 ? 1u : 0u);
+                                            (kb != u.kb0 || kk != 0) ? 1u : 0u);
                     }
                     mma_commit<CG>(empty_bar(stage), 0x3);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 mma_commit<CG>(tfull_bar(buf), 0x3);
-                tile = next_tile(tile, static_cast<uint32_t>(t), ok);
+                more = next_unit(u, static_cast<uint32_t>(t), ok);
                 if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarSched);
             }
         }
@@ -445,7 +592,9 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
         uint32_t nstore = 0;
         int t = 0;
-        for (int tile = cluster_id; tile >= 0; ++t) {
+        Unit u;
+        for (bool more = first_unit(u); more; ++t) {
+            const int tile = u.tile;
             int tm, tn;
             raster_tile(tile, num_m, num_n, group_m, tm, tn);
             const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
@@ -463,45 +612,30 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             const int row_base = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
             const int col0 = tn * Cfg::BN;
             const uint32_t tbase0 = tmem_base + ((sub * 32u) << 16) + buf * Cfg::CONSUMERS * Cfg::BN;
+            constexpr int NQ = Cfg::CONSUMERS * Cfg::EPI_CHUNKS;
             // chunk q: consumer q / EPI_CHUNKS (its own rows and accumulator),
             // columns (q % EPI_CHUNKS) * EPI_COLS of the tile
-#pragma unroll 1
-            for (int q = 0; q < Cfg::CONSUMERS * Cfg::EPI_CHUNKS; ++q) {
+            auto chunk_taddr = [&](int q) -> uint32_t {
+                const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
+                return tbase0 + static_cast<uint32_t>(cons) * Cfg::BN + static_cast<uint32_t>(c * Cfg::EPI_COLS);
+            };
+            // This warp has read its whole slice of accumulator `buf`.
+            auto release_tmem = [&]() {
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (CG == 1) mbar_arrive_local(tempty_bar(buf));
+                    else mbar_arrive_cluster(map_to_cta(tempty_bar(buf), 0));
+                }
+            };
+            // Write one chunk of C from registers (32 packed words: 32 fp32
+            // or 64 bf16): the ragged end of each row by plain stores, the rest
+            // through a swizzled staging buffer and a TMA store.
+            auto store_chunk = [&](uint32_t (&packed)[32], int q) {
                 const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
                 const int row0 = row_base + cons * Cfg::BM_MMA;
-                const uint32_t tbase = tbase0 + static_cast<uint32_t>(cons) * Cfg::BN;
-                uint32_t packed[32];
-                const int erow = row0 + static_cast<int>(lane);   // this thread's row of C
-                if constexpr (Cfg::OUT == 0) {
-                    tmem_ld_32x32b_x32(tbase + c * 32, packed);
-                    tmem_ld_wait();
-                    if (fused) epilogue32_f32c(packed, C, ldc, erow, col0 + c * 32, M, N, epi);
-                } else {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld_32x32b_x32(tbase + c * 64, v0);
-                    tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
-                    tmem_ld_wait();
-                    if (fused) {
-                        epilogue32_bf16c(v0, C, ldc, erow, col0 + c * 64, M, N, epi);
-                        epilogue32_bf16c(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, epi);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
-                        packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
-                    }
-                }
-                if (q == Cfg::CONSUMERS * Cfg::EPI_CHUNKS - 1) {
-                    // This warp has read its whole slice of accumulator `buf`.
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (CG == 1) mbar_arrive_local(tempty_bar(buf));
-                        else mbar_arrive_cluster(map_to_cta(tempty_bar(buf), 0));
-                    }
-                }
                 const int cstart = col0 + c * Cfg::EPI_COLS;
-                if (cstart >= N) continue;                  // chunk wholly right of C
+                if (cstart >= N) return;                    // chunk wholly right of C
                 if (cstart + Cfg::EPI_COLS > n_tma) {
                     // Columns [n_tma, N) end C's rows inside a 16-byte granule:
                     // a TMA store writes whole granules, so these few elements
@@ -522,7 +656,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                             }
                         }
                     }
-                    if (cstart >= n_tma) continue;          // nothing left for the TMA store
+                    if (cstart >= n_tma) return;            // nothing left for the TMA store
                 }
                 const uint32_t sbuf = stage_base + (nstore & 1u) * Cfg::EPI_BUF;
                 if (lane == 0) bulk_wait_group_read<1>();   // the store that used sbuf is done reading
@@ -538,19 +672,136 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmC, sbuf, col0 + c * Cfg::EPI_COLS, row0);
+                    tma_store_2d(&tmC, sbuf, cstart, row0);
                     bulk_commit_group();
                 }
                 ++nstore;
+            };
+            bool split = false;   // stream-K: this unit is one piece of a split tile
+            if constexpr (Cfg::SK) split = !(u.kb0 == 0 && u.kb1 == num_kb);
+            if (split) {
+              if constexpr (Cfg::SK) {
+                // ---- stream-K: this unit is part of a tile split between
+                // clusters.  Write this CTA's fp32 partial (row 32 sub + lane,
+                // all BN columns) to its slot, count the arrival, and let the
+                // last contributor sum every partial in contributor order.
+                const int64_t G = num_clusters;
+                auto owner = [&](int64_t it) { return ((it + 1) * G + sk_total - 1) / sk_total - 1; };
+                auto part = [&](int64_t cc) -> float * {
+                    const int64_t first = ((cc * sk_total) / G) / num_kb;   // cc's first tile
+                    const int64_t slot = (cc * CG + rank) * 2 + (tile == first ? 0 : 1);
+                    return sk_partials + slot * (128 * Cfg::BN);
+                };
+                const int64_t t0 = static_cast<int64_t>(tile) * num_kb;
+                const int64_t c_lo = owner(t0), c_hi = owner(t0 + num_kb - 1);
+                float *mine = part(cluster_id) + static_cast<int64_t>(sub * 32u + lane) * Cfg::BN;
+#pragma unroll 1
+                for (int c = 0; c < Cfg::BN / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase0 + static_cast<uint32_t>(c * 32), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        __stcg(reinterpret_cast<float4 *>(mine + c * 32 + 4 * j),
+                               make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                           __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+                }
+                release_tmem();
+                // The barrier orders the 128 threads' partial stores before
+                // thread 0's gpu-scope fence, which (being cumulative) makes
+                // them visible before its counter update.
+                const uint32_t epi_tid = threadIdx.x - 64u;
+                named_barrier_sync(1, 128);
+                if (epi_tid == 0) {
+                    __threadfence();
+                    unsigned long long *ctr = sk_counters + static_cast<int64_t>(tile) * CG + rank;
+                    const unsigned long long tag = static_cast<unsigned long long>(sk_epoch) << 32;
+                    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(ctr), seen, want;
+                    do {
+                        seen = old;
+                        want = ((seen & 0xFFFFFFFF00000000ull) == tag) ? seen + 1ull : (tag | 1ull);
+                        old = atomicCAS(ctr, seen, want);
+                    } while (old != seen);
+                    *sk_last_flag =
+                        ((want & 0xFFFFFFFFull) == static_cast<unsigned long long>(c_hi - c_lo + 1)) ? 1u : 0u;
+                }
+                named_barrier_sync(1, 128);
+                if (*sk_last_flag) {
+                    __threadfence();
+                    sk_fixup<Cfg::OUT, Cfg::BN>(part, c_lo, c_hi,
+                                                tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA, col0, M, N, C, ldc,
+                                                epi_tid, epi);
+                    // all contributors have arrived: back to zero arrivals, so
+                    // a replay of this launch (same epoch) starts clean
+                    if (epi_tid == 0) sk_counters[static_cast<int64_t>(tile) * CG + rank] = static_cast<unsigned long long>(sk_epoch) << 32;
+                }
+                named_barrier_sync(1, 128);
+              }
+            } else if constexpr (Cfg::OUT == 0) {
+                // fp32 C: one 32-column TMEM load per chunk, double-buffered in
+                // registers so chunk q + 1's load is in flight while chunk q
+                // is converted and stored
+                auto finish = [&](uint32_t (&v)[32], int q) {
+                    if (fused) {
+                        const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
+                        epilogue32_f32c(v, C, ldc, row_base + cons * Cfg::BM_MMA + static_cast<int>(lane),
+                                        col0 + c * 32, M, N, epi);
+                    }
+                    store_chunk(v, q);
+                };
+                uint32_t ra[32], rb[32];
+                tmem_ld_32x32b_x32(chunk_taddr(0), ra);
+#pragma unroll 1
+                for (int q = 0; q < NQ; q += 2) {
+                    tmem_ld_wait();
+                    if (q + 1 < NQ) tmem_ld_32x32b_x32(chunk_taddr(q + 1), rb);
+                    else release_tmem();
+                    finish(ra, q);
+                    if (q + 1 < NQ) {
+                        tmem_ld_wait();
+                        if (q + 2 < NQ) tmem_ld_32x32b_x32(chunk_taddr(q + 2), ra);
+                        else release_tmem();
+                        finish(rb, q + 1);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int q = 0; q < NQ; ++q) {
+                    const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
+                    const int erow = row_base + cons * Cfg::BM_MMA + static_cast<int>(lane);
+                    uint32_t packed[32], v0[32], v1[32];
+                    tmem_ld_32x32b_x32(chunk_taddr(q), v0);
+                    tmem_ld_32x32b_x32(chunk_taddr(q) + 32, v1);
+                    tmem_ld_wait();
+                    if (q == NQ - 1) release_tmem();
+                    if (fused) {
+                        epilogue32_bf16c(v0, C, ldc, erow, col0 + c * 64, M, N, epi);
+                        epilogue32_bf16c(v1, C, ldc, erow, col0 + c * 64 + 32, M, N, epi);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+                        packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+                    }
+                    store_chunk(packed, q);
+                }
             }
-            // next tile: one lane fetches it, the warp follows
-            int nt = -1;
-            if (lane == 0) {
+            // next unit: stream-K computes it; otherwise one lane fetches the
+            // next tile and the warp follows
+            if constexpr (Cfg::SK) {
                 bool ok = true;
-                nt = next_tile(tile, static_cast<uint32_t>(t), ok);
-                if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarSched);
+                more = next_unit(u, static_cast<uint32_t>(t), ok);
+            } else {
+                int nt = -1;
+                if (lane == 0) {
+                    bool ok = true;
+                    nt = next_tile(tile, static_cast<uint32_t>(t), ok);
+                    if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarSched);
+                }
+                nt = __shfl_sync(0xffffffffu, nt, 0);
+                u = Unit{nt, 0, num_kb};
+                more = nt >= 0;
             }
-            tile = __shfl_sync(0xffffffffu, nt, 0);
         }
         if (lane == 0) bulk_wait_group<0>();
         __syncwarp();

@@ -40,6 +40,8 @@ CONFIGS = {
     "mxfp8_1cta_128x256": 7,
     "mxfp8_2cta_256x256": 8,
     "2cta_512x256_clc": 9,
+    "2cta_256x256_sk": 10,
+    "2cta_256x224": 11,
 }
 
 STATUS_NAMES = {

@@ -123,7 +123,14 @@ typedef enum {
                                        B k-tile, one TMEM accumulator each (TMEM single-buffered);
                                        Cluster Launch Control; chosen when there are >= 148
                                        such tiles (two waves), e.g. 8192 x 8192 */
-    GEMM_CFG_COUNT_ = 10
+    GEMM_CFG_2CTA_256x256_SK = 10,  /* CTA pair per 256 x 256 tile, stream-K: every co-resident pair
+                                       takes an equal contiguous share of the (tile, 64-wide K block)
+                                       iterations; a tile split between pairs is summed from fp32
+                                       partials by its last contributor, in contributor order
+                                       (deterministic); uses the library-owned split workspace */
+    GEMM_CFG_2CTA_256x224 = 11,     /* CTA pair per 256 x 224 tile (fp32 C; bf16 C runs 2CTA_256x256),
+                                       for shapes whose 224-wide tiles fill the waves better */
+    GEMM_CFG_COUNT_ = 12
 } gemm_config_t;
 
 /*

@@ -143,12 +143,17 @@ def test_status_strings_and_config_control():
     G.gemm_force_config("auto")
     assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 512 tiles of 512 x 256
     assert G.gemm_select_config(6144, 6144, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 288
-    assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_clc"]   # 8 x 16 = 128 < 148
+    # 256 pair tiles: 3.46 waves of 74 pairs; operands (64 MiB) stay in L2 -> stream-K
+    assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_sk"]
+    assert G.gemm_select_config(4000, 3000, 2000) == G.CONFIGS["2cta_256x256_sk"]   # 192 tiles: 2.6 waves
     assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
     assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
-    assert G.gemm_select_config(1000, 8192, 8192) == G.CONFIGS["2cta_256x256"]
-    assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_clc"]
+    # 128 pair tiles of 256 x 256 (1.73 waves) against 148 of 256 x 224 (two full waves)
+    assert G.gemm_select_config(1000, 8192, 8192) == G.CONFIGS["2cta_256x224"]
+    assert G.gemm_select_config(2048, 8192, 2048) == G.CONFIGS["2cta_256x224"]     # 296 tiles: 4 full waves
+    assert G.gemm_select_config(2560, 3584, 2048) == G.CONFIGS["2cta_256x256"]     # 140 tiles: 0.95 of 2 waves
+    assert G.gemm_select_config(4096, 4608, 2048) == G.CONFIGS["2cta_256x256_clc"] # 288 tiles: 0.97 of 4 waves
     assert G.gemm_select_config(300, 1000, 64) == G.CONFIGS["1cta_128x128"]
     with pytest.raises(G.GemmError):
         G.gemm_bf16(A, B, C, -1, 1, 1, 1, 1, 1, stream=0)

@@ -49,7 +49,7 @@ def test_replays_stay_valid_after_the_workspaces_grow():
 
 
 def test_one_graph_of_several_configs_replays_like_eager_calls():
-    """One graph holding the 2-CTA CLC kernel (4096 x 4096), the skinny path
+    """One graph holding the 2-CTA stream-K kernel (4096 x 4096), the skinny path
     (64 rows), the fused epilogue (bias + ReLU, bf16 out) and the
     block-scaled path; replayed with fresh inputs, every output is
     bit-identical to the same calls made eagerly."""
@@ -72,7 +72,7 @@ def test_one_graph_of_several_configs_replays_like_eager_calls():
     A4, B4 = torch.from_numpy(am).cuda(), torch.from_numpy(bm).cuda()
     SA, SB = torch.from_numpy(sa).cuda(), torch.from_numpy(sb).cuda()
     C4 = torch.empty((M4, N4), dtype=torch.bfloat16, device="cuda")
-    assert G.gemm_select_config(M1, N1, K1) == G.CONFIGS["2cta_256x256_clc"]
+    assert G.gemm_select_config(M1, N1, K1) == G.CONFIGS["2cta_256x256_sk"]
     assert G.gemm_select_config(M2, N2, K2) == G.CONFIGS["skinny"]
 
     def calls():

@@ -14,7 +14,8 @@ from gpu_helpers import assert_close, assert_exact, sample_indices, to_device_bf
 pytestmark = pytest.mark.gpu
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 K_, MN = G.KMAJOR, G.MNMAJOR
-CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc", "skinny"]
+CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc", "skinny",
+        "2cta_256x256_sk", "2cta_256x224"]
 
 
 def _store(canon_bits: np.ndarray, mn: bool) -> np.ndarray:

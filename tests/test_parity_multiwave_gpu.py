@@ -30,7 +30,8 @@ from gpu_helpers import assert_close, assert_exact, run_gemm, run_mxfp8
 
 pytestmark = pytest.mark.gpu
 
-CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "1cta_128x256_clc", "2cta_256x256_clc", "2cta_512x256_clc"]
+CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "1cta_128x256_clc", "2cta_256x256_clc", "2cta_512x256_clc",
+        "2cta_256x256_sk", "2cta_256x224"]
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 WAVES = (4096, 4864, 256)
 
@@ -45,7 +46,8 @@ def _case(M, N, K, dist, workload, with_abs):
 
 def _tiles(cfg, M, N):
     bm, bn = {"1cta_128x128": (128, 128), "1cta_128x256": (128, 256), "2cta_256x256": (256, 256),
-              "1cta_128x256_clc": (128, 256), "2cta_256x256_clc": (256, 256), "2cta_512x256_clc": (512, 256)}[cfg]
+              "1cta_128x256_clc": (128, 256), "2cta_256x256_clc": (256, 256), "2cta_512x256_clc": (512, 256),
+              "2cta_256x256_sk": (256, 256), "2cta_256x224": (256, 224)}[cfg]
     pair = cfg.startswith("2cta")
     return -(-M // bm) * -(-N // bn), (74 if pair else 148)
 
@@ -80,7 +82,7 @@ def test_several_waves_ragged_normal(cfg):
     assert_close(got, c_ref, s_abs, F32, f"{cfg} {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("cfg", ["2cta_512x256_clc", "2cta_256x256_clc"])
+@pytest.mark.parametrize("cfg", ["2cta_512x256_clc", "2cta_256x256_clc", "2cta_256x256_sk"])
 def test_several_waves_repeat_identical(cfg):
     """A CLC schedule assigns tiles to pairs by timing, differently on every
     run; the per-element order is fixed by the tile, so results must not
