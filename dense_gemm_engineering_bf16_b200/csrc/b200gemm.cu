@@ -383,7 +383,16 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     // Stream-K: every co-resident cluster, each with an equal share of the
     // (tile, K block) iterations.
     const int64_t resident = st->max_clusters[cfg_id][oi];
-    const int64_t clusters = Cfg::CLC ? tiles : (Cfg::SK || tiles > resident ? resident : tiles);
+    int64_t clusters = Cfg::CLC ? tiles : (tiles > resident ? resident : tiles);
+    if constexpr (Cfg::SK) {
+        // Every cluster's range must hold at least one iteration (the
+        // fix-up counts a split tile's contributors as the consecutive range
+        // owners), and a range of fewer than 4 K blocks barely fills the
+        // pipeline: at most one cluster per 4 iterations.
+        const int64_t iters = tiles * ((K + Cfg::BK - 1) / Cfg::BK);
+        const int64_t want = (iters + 3) / 4;
+        clusters = want < resident ? want : resident;
+    }
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
     // tiles that run at the same time: one wave (for CLC, as many clusters
     // as fit on the SMs at once); stream-K keeps K ascending
