@@ -324,6 +324,9 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
                           uint32_t layout = 0) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
+    // MN-major tiles arrive as 64-wide boxes: whole boxes per CTA only
+    if (((layout & b200::kLayoutBMajorN) && Cfg::B_ROWS % 64) || ((layout & b200::kLayoutAMajorM) && Cfg::BM_CTA % 64))
+        return GEMM_ERR_INVALID_VALUE;
     cudaError_t e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -577,8 +580,11 @@ gemm_status_t launch_dense(DeviceState *st, DeviceStatus *status, gemm_config_t 
             return f32 ? launch_bf16<Cfg2x256F32S>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                        : launch_bf16<Cfg2x256B16S>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
         case GEMM_CFG_2CTA_256x224:
-            // 224 columns are 3.5 chunks of 64 bf16: bf16 C takes 256 x 256
-            return f32 ? launch_bf16<Cfg2x224F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
+            // 224 columns are 3.5 chunks of 64 bf16, and each CTA's 112 rows
+            // of a B stored K x N are not whole 64-wide MN-major boxes: those
+            // take 256 x 256
+            return (f32 && !(layout & b200::kLayoutBMajorN))
+                       ? launch_bf16<Cfg2x224F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                        : launch_bf16<Cfg2x256B16>(st, status, GEMM_CFG_2CTA_256x256, A, B, C, M, N, K, lda, ldb, ldc,
                                                   stream, epi, layout);
         case GEMM_CFG_1CTA_128x256_CLC:

@@ -69,6 +69,7 @@ struct GemmMxf8Cfg {
     static constexpr int TX_BYTES = CTA_BYTES * CG;  // bytes landing on the leader's full[s]
     static constexpr int STAGE_BYTES = ((CTA_BYTES + 1023) / 1024) * 1024;
     static constexpr int EPI_COLS = BN / 2;        // accumulator columns one epilogue warp drains
+    static_assert(EPI_COLS % 64 == 0, "the drain reads 64 columns per TMEM round trip");
     // Scale slots in TMEM (32 columns each, beside the accumulator): a
     // separate warp copies stage s's scales into slot s % SF_SLOTS ahead of
     // the MMAs that read them.
@@ -98,7 +99,7 @@ struct GemmMxf8Cfg {
 // memory, then writes kRepackKb consecutive 512-byte chunks with 16-byte
 // stores (thread r of a chunk writes the four words of rows r, r+32, r+64,
 // r+96).
-constexpr int kRepackKb = 32;
+constexpr int kRepackKb = 8;
 
 __global__ void __launch_bounds__(256)
 mxf8_repack_scales_kernel(const uint8_t *__restrict__ sfa, int64_t M, int64_t a_blocks,
@@ -405,14 +406,18 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const int col0 = tn * Cfg::BN + half * Cfg::EPI_COLS;
             uint16_t *crow = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * 2);
             uint32_t packed[Cfg::EPI_COLS / 2];
+            // two 32-column loads per TMEM round trip
 #pragma unroll
-            for (int g = 0; g < Cfg::EPI_COLS / 32; ++g) {
-                uint32_t v[32];
+            for (int g = 0; g < Cfg::EPI_COLS / 32; g += 2) {
+                uint32_t v[32], w[32];
                 tmem_ld_32x32b_x32(tbase + g * 32, v);
+                tmem_ld_32x32b_x32(tbase + g * 32 + 32, w);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
+                for (int i = 0; i < 16; ++i) {
                     packed[16 * g + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                    packed[16 * g + 16 + i] = pack_bf16x2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+                }
             }
             tc_fence_before_sync();
             __syncwarp();

@@ -128,8 +128,9 @@ typedef enum {
                                        iterations; a tile split between pairs is summed from fp32
                                        partials by its last contributor, in contributor order
                                        (deterministic); uses the library-owned split workspace */
-    GEMM_CFG_2CTA_256x224 = 11,     /* CTA pair per 256 x 224 tile (fp32 C; bf16 C runs 2CTA_256x256),
-                                       for shapes whose 224-wide tiles fill the waves better */
+    GEMM_CFG_2CTA_256x224 = 11,     /* CTA pair per 256 x 224 tile, for shapes whose 224-wide tiles fill
+                                       the waves better; fp32 C with B stored K-major only (bf16 C or
+                                       a B stored K x N runs 2CTA_256x256) */
     GEMM_CFG_COUNT_ = 12
 } gemm_config_t;
 
@@ -300,7 +301,8 @@ B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
  * epilogue (beta != 0, alpha != 1, a bias or an activation) they take
  * GEMM_CFG_2CTA_256x256_CLC where this returns GEMM_CFG_2CTA_512x256_CLC
  * (the 256 x 256 tile's second TMEM buffer hides the longer epilogue), and
- * an A stored K x M never takes GEMM_CFG_SKINNY. */
+ * an A stored K x M never takes GEMM_CFG_SKINNY.  Where this returns
+ * GEMM_CFG_2CTA_256x224, bf16 C or a B stored K x N runs GEMM_CFG_2CTA_256x256. */
 B200GEMM_API gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K);
 
 /* Number of kernels that one call queues for this shape: gemm_bf16 /
