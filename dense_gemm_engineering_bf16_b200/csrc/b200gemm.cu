@@ -583,10 +583,10 @@ gemm_status_t launch_dense(DeviceState *st, DeviceStatus *status, gemm_config_t 
             // 224 columns are 3.5 chunks of 64 bf16, and each CTA's 112 rows
             // of a B stored K x N are not whole 64-wide MN-major boxes: those
             // take 256 x 256
-            return (f32 && !(layout & b200::kLayoutBMajorN))
-                       ? launch_bf16<Cfg2x224F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
-                       : launch_bf16<Cfg2x256B16>(st, status, GEMM_CFG_2CTA_256x256, A, B, C, M, N, K, lda, ldb, ldc,
-                                                  stream, epi, layout);
+            if (f32 && !(layout & b200::kLayoutBMajorN))
+                return launch_bf16<Cfg2x224F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+            return launch_dense(st, status, GEMM_CFG_2CTA_256x256, f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi,
+                                layout);
         case GEMM_CFG_1CTA_128x256_CLC:
             return f32 ? launch_bf16<Cfg1x256F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                        : launch_bf16<Cfg1x256B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
