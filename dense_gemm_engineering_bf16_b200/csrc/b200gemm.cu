@@ -292,16 +292,16 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     if (tall_tiles >= 148) return GEMM_CFG_2CTA_512x256_CLC;
     if (pair_tiles >= 74) {
         // The last wave of pair tiles: when it leaves more than a tenth of
-        // the pairs idle, either 256 x 224 tiles fill the waves better
-        // (e.g. 1000 x 8192: 148 tiles, two full waves, against 128 tiles in
-        // two waves of 256 x 256), or, with operands small enough to stay in
-        // L2, stream-K gives every pair an equal share of the iterations.
+        // the pairs idle and 256 x 224 tiles fill the waves better (e.g.
+        // 1000 x 8192: 148 tiles, two full waves, against 128 tiles in two
+        // waves of 256 x 256), take those.  (Stream-K, GEMM_CFG_2CTA_256x256_SK,
+        // evens out the waves too, but its fix-up of split tiles cost more
+        // than it saved on 4096^3 and 4000 x 3000 x 2000: it is not chosen.)
         const int64_t waves = (pair_tiles + 73) / 74;
         if (pair_tiles * 10 < waves * 74 * 9) {
             const int64_t tiles224 = ((M + 255) / 256) * ((N + 223) / 224);
             const int64_t waves224 = (tiles224 + 73) / 74;
             if (waves224 * 224 * 100 <= waves * 256 * 92) return GEMM_CFG_2CTA_256x224;
-            if (2 * (M + N) * K <= (int64_t(96) << 20) && K >= 512) return GEMM_CFG_2CTA_256x256_SK;
         }
         return pair_tiles >= 148 ? GEMM_CFG_2CTA_256x256_CLC : GEMM_CFG_2CTA_256x256;
     }

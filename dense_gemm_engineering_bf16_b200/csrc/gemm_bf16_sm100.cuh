@@ -111,28 +111,19 @@ struct GemmBf16Cfg {
     static constexpr int EPI_COLS = OUT == 0 ? 32 : 64; // columns in one 128-byte staged row
     static constexpr int EPI_CHUNKS = BN / EPI_COLS;
     static constexpr int EPI_BUF = 32 * 128;       // one warp's 32 rows x 128 bytes
-    // Epilogue warps: four (one per TMEM lane quarter), or eight with two
-    // consumers (one set of four per consumer's accumulator, so the single-
-    // buffered TMEM is drained in half the time).  Eight warps single-buffer
-    // their staging rows to stay within shared memory.
-    static constexpr int EPI_WARPS = CONSUMERS == 2 ? 8 : 4;
-    static constexpr int EPI_STAGE_BUFS = EPI_WARPS == 8 ? 1 : 2;
-    static constexpr int EPI_BYTES = EPI_WARPS * EPI_STAGE_BUFS * EPI_BUF;
+    static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
     static constexpr int TMEM_COLS = pow2_at_least(ACC_BUFS * CONSUMERS * BN, 32);
     // full[S], empty[S], tmem_full[2], tmem_empty[2] (+ clc[2], sched_full[2], sched_empty[2])
     static constexpr int NUM_BARS = 2 * STAGES + 4 + (CLC ? 6 : 0);
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
     // after the barriers: TMEM address, abort flag, 2 tile ids, 2 CLC answers
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 64;
-    static constexpr int SCHED_WARP = 2 + EPI_WARPS;       // CLC scheduler warp
-    static constexpr int THREADS = 32 * (2 + EPI_WARPS + (CLC ? 1 : 0));
-    // arrivals that free a tile slot: producer, MMA (leader only), epilogue warps
-    static constexpr int SCHED_CONSUMERS = CG == 1 ? 2 + EPI_WARPS : 3 + 2 * EPI_WARPS;
+    static constexpr int THREADS = CLC ? 224 : 192;        // + one scheduler warp
+    static constexpr int SCHED_CONSUMERS = CG == 1 ? 6 : 11;  // arrivals that free a tile slot
 
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
     static_assert(CONSUMERS == 1 || CONSUMERS == 2, "one or two MMA consumers");
     static_assert(!SK || (!CLC && CONSUMERS == 1 && BN % 4 == 0), "stream-K: static schedule, one consumer");
-    static_assert(!SK || EPI_WARPS == 4, "the stream-K fix-up runs on four epilogue warps (128 threads)");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
     static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows <= 256, whole 8-row swizzle atoms");
     static_assert(BN % EPI_COLS == 0, "epilogue chunks cover the tile");
@@ -341,7 +332,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), Cfg::EPI_WARPS * CG);
+            mbar_init(tempty_bar(b), 4 * CG);
         }
         if constexpr (Cfg::CLC) {
             for (int i = 0; i < 2; ++i) {
@@ -562,7 +553,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             }
         }
         __syncwarp();
-    } else if (Cfg::CLC && warp == Cfg::SCHED_WARP) {
+    } else if (Cfg::CLC && warp == 6) {
         // ------------------------------------------- CLC scheduler (leader) --
         if constexpr (Cfg::CLC) {
             if (rank == 0 && lane == 0) {
@@ -598,9 +589,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t sub = warp & 3u;            // TMEM lanes [32*sub, 32*sub + 32)
         const uint32_t ew = warp - 2u;             // staging slot
         const bool fused = !epi.identity();
-        const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * Cfg::EPI_STAGE_BUFS * Cfg::EPI_BUF;
-        // with eight warps, warps 2-5 drain consumer 0 and warps 6-9 consumer 1
-        const int q_first = Cfg::EPI_WARPS == 8 ? static_cast<int>(ew >> 2) * Cfg::EPI_CHUNKS : 0;
+        const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
         uint32_t nstore = 0;
         int t = 0;
         Unit u;
@@ -623,12 +612,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             const int row_base = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
             const int col0 = tn * Cfg::BN;
             const uint32_t tbase0 = tmem_base + ((sub * 32u) << 16) + buf * Cfg::CONSUMERS * Cfg::BN;
-            // this warp's chunks: q_first + [0, NQ)
-            constexpr int NQ = Cfg::CONSUMERS * Cfg::EPI_CHUNKS / (Cfg::EPI_WARPS / 4);
+            constexpr int NQ = Cfg::CONSUMERS * Cfg::EPI_CHUNKS;
             // chunk q: consumer q / EPI_CHUNKS (its own rows and accumulator),
             // columns (q % EPI_CHUNKS) * EPI_COLS of the tile
             auto chunk_taddr = [&](int q) -> uint32_t {
-                q += q_first;
                 const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
                 return tbase0 + static_cast<uint32_t>(cons) * Cfg::BN + static_cast<uint32_t>(c * Cfg::EPI_COLS);
             };
@@ -645,7 +632,6 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             // or 64 bf16): the ragged end of each row by plain stores, the rest
             // through a swizzled staging buffer and a TMA store.
             auto store_chunk = [&](uint32_t (&packed)[32], int q) {
-                q += q_first;
                 const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
                 const int row0 = row_base + cons * Cfg::BM_MMA;
                 const int cstart = col0 + c * Cfg::EPI_COLS;
@@ -672,8 +658,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     if (cstart >= n_tma) return;            // nothing left for the TMA store
                 }
-                const uint32_t sbuf = stage_base + (nstore % Cfg::EPI_STAGE_BUFS) * Cfg::EPI_BUF;
-                if (lane == 0) bulk_wait_group_read<Cfg::EPI_STAGE_BUFS - 1>();   // sbuf's last store has read it
+                const uint32_t sbuf = stage_base + (nstore & 1u) * Cfg::EPI_BUF;
+                if (lane == 0) bulk_wait_group_read<1>();   // the store that used sbuf is done reading
                 __syncwarp();
                 // Row `lane` of the 32 x 128-byte box; 16-byte chunk j goes to
                 // chunk slot j ^ (row % 8) -- the TMA 128-byte swizzle.
@@ -757,8 +743,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 // is converted and stored
                 auto finish = [&](uint32_t (&v)[32], int q) {
                     if (fused) {
-                        const int qq = q + q_first;
-                        const int cons = qq / Cfg::EPI_CHUNKS, c = qq - cons * Cfg::EPI_CHUNKS;
+                        const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
                         epilogue32_f32c(v, C, ldc, row_base + cons * Cfg::BM_MMA + static_cast<int>(lane),
                                         col0 + c * 32, M, N, epi);
                     }
@@ -782,8 +767,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             } else {
 #pragma unroll 1
                 for (int q = 0; q < NQ; ++q) {
-                    const int qq = q + q_first;
-                    const int cons = qq / Cfg::EPI_CHUNKS, c = qq - cons * Cfg::EPI_CHUNKS;
+                    const int cons = q / Cfg::EPI_CHUNKS, c = q - cons * Cfg::EPI_CHUNKS;
                     const int erow = row_base + cons * Cfg::BM_MMA + static_cast<int>(lane);
                     uint32_t packed[32], v0[32], v1[32];
                     tmem_ld_32x32b_x32(chunk_taddr(q), v0);

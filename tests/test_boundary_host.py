@@ -143,9 +143,9 @@ def test_status_strings_and_config_control():
     G.gemm_force_config("auto")
     assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 512 tiles of 512 x 256
     assert G.gemm_select_config(6144, 6144, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 288
-    # 256 pair tiles: 3.46 waves of 74 pairs; operands (64 MiB) stay in L2 -> stream-K
-    assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_sk"]
-    assert G.gemm_select_config(4000, 3000, 2000) == G.CONFIGS["2cta_256x256_sk"]   # 192 tiles: 2.6 waves
+    # 256 pair tiles (3.46 waves of 74 pairs), 192 (2.6): CLC, since 224-wide tiles do no better
+    assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_clc"]
+    assert G.gemm_select_config(4000, 3000, 2000) == G.CONFIGS["2cta_256x256_clc"]
     assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
     assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]

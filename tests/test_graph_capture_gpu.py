@@ -49,7 +49,7 @@ def test_replays_stay_valid_after_the_workspaces_grow():
 
 
 def test_one_graph_of_several_configs_replays_like_eager_calls():
-    """One graph holding the 2-CTA stream-K kernel (4096 x 4096), the skinny path
+    """One graph holding the 2-CTA CLC kernel (4096 x 4096), the skinny path
     (64 rows), the fused epilogue (bias + ReLU, bf16 out) and the
     block-scaled path; replayed with fresh inputs, every output is
     bit-identical to the same calls made eagerly."""
@@ -72,7 +72,7 @@ def test_one_graph_of_several_configs_replays_like_eager_calls():
     A4, B4 = torch.from_numpy(am).cuda(), torch.from_numpy(bm).cuda()
     SA, SB = torch.from_numpy(sa).cuda(), torch.from_numpy(sb).cuda()
     C4 = torch.empty((M4, N4), dtype=torch.bfloat16, device="cuda")
-    assert G.gemm_select_config(M1, N1, K1) == G.CONFIGS["2cta_256x256_sk"]
+    assert G.gemm_select_config(M1, N1, K1) == G.CONFIGS["2cta_256x256_clc"]
     assert G.gemm_select_config(M2, N2, K2) == G.CONFIGS["skinny"]
 
     def calls():
@@ -110,3 +110,41 @@ def test_one_graph_of_several_configs_replays_like_eager_calls():
     tol = 1e-3 * s_abs + 1e-6 + 2.0 ** -8 * np.abs(want)
     assert np.all(np.abs(C3.cpu().float().numpy()[rows] - want) <= tol)
     assert G.gemm_check_device_status() == 0
+
+
+def test_stream_k_replays_match_eager_and_oracle():
+    """The stream-K kernel in a graph: its split-tile counters are left at
+    zero arrivals by each launch, so replays (same epoch) stay correct."""
+    s = torch.cuda.Stream()
+    M, N, K = 1000, 1500, 1000                 # 4 x 6 = 24 pair tiles x 16 K blocks over <= 74 pairs
+    a, b = synth.bf16_operands(M, N, K, "normal", workload=430)
+    A, B = to_device_bf16(a), to_device_bf16(b)
+    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    G.gemm_force_config("2cta_256x256_sk")
+    try:
+        call = lambda: G.gemm_bf16(A, B, C, M, N, K, K, K, N, stream=s)  # noqa: E731
+        with torch.cuda.stream(s):
+            call()
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            call()
+        for rep in range(3):
+            a2, b2 = synth.bf16_operands(M, N, K, "normal", workload=431 + rep)
+            A.copy_(to_device_bf16(a2))
+            B.copy_(to_device_bf16(b2))
+            C.fill_(float("nan"))
+            g.replay()
+            torch.cuda.synchronize()
+            got = C.clone()
+            with torch.cuda.stream(s):
+                call()
+            s.synchronize()
+            assert torch.equal(got, C)
+            rows = np.arange(0, M, 37)
+            c_ref, s_abs = oracle.gemm_bf16_f64(a2, b2, rows=rows, with_abs=True)
+            err = np.abs(got.cpu().numpy()[rows].astype(np.float64) - c_ref)
+            assert np.all(err <= 1e-3 * s_abs + 1e-6)
+    finally:
+        G.gemm_force_config("auto")
+    G.gemm_check_device_status()
