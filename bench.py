@@ -554,7 +554,7 @@ def main():
     ap.add_argument("--shape", type=int, nargs=3, metavar=("M", "N", "K"),
                     help="override the workload's shape (U[-1,1] inputs), e.g. for profiling")
     ap.add_argument("--config", default="auto")
-    ap.add_argument("--e2e-steps", type=int, default=5, help="0 skips the end-to-end leg")
+    ap.add_argument("--e2e-steps", type=int, default=20, help="0 skips the end-to-end leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", dest="configs", action="store_false",

@@ -101,15 +101,17 @@ __device__ __forceinline__ void store_c(void *C, int64_t ldc, int m, int n, floa
 // The last contributor of a split tile sums the contributors' fp32 partials
 // ([m][128] each) in contributor order and writes C rows [0, M) x the tile's
 // 128 columns.  Thread t handles four consecutive columns (t % 32) * 4 of
-// rows m = 4 j + t / 32; per round every thread has 8 rows x 2 contributors
-// of float4 loads in flight, and each element is summed c_lo, c_lo+1, ...
-// exactly as a sequential loop would.
+// rows m = 4 j + t / 32.  Each round issues the loads of 4 rows x up to 4
+// contributors before summing, so a tile split between up to four CTAs (the
+// usual case) costs one round trip to L2 per round; each element is summed
+// c_lo, c_lo+1, ... exactly as a sequential loop would.
 template <int OUT>
 __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_elems, int slots_per_cta,
                                            int64_t c_lo, int64_t c_hi, int64_t t, int64_t total, int64_t g,
                                            int64_t kb_per_tile, int M, int N, void *C, int64_t ldc,
                                            uint32_t epi_tid, const Epilogue &epi) {
-    constexpr int ROWS = 8;                      // rows per round for this thread
+    constexpr int ROWS = 4;                      // rows per round for this thread
+    constexpr int CPR = 4;                       // contributors per round
     const int n4 = static_cast<int>(epi_tid & 31u) * 4;
     const int msub = static_cast<int>(epi_tid >> 5);
     const int n = static_cast<int>(t) * 128 + n4;
@@ -121,26 +123,25 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
         float4 acc[ROWS];
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-        int64_t cc = c_lo;
-        for (; cc <= c_hi; cc += 2) {
-            const bool two = cc + 1 <= c_hi;
-            const float *p0 = slot_ptr(cc);
-            const float *p1 = two ? slot_ptr(cc + 1) : p0;
-            float4 v0[ROWS], v1[ROWS];
+        for (int64_t cc = c_lo; cc <= c_hi; cc += CPR) {
+            float4 v[CPR][ROWS];
 #pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                const int m = m0 + 4 * r;
-                const bool in = m < M;
-                v0[r] = in ? __ldcg(reinterpret_cast<const float4 *>(p0 + static_cast<int64_t>(m) * 128))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                v1[r] = (in && two) ? __ldcg(reinterpret_cast<const float4 *>(p1 + static_cast<int64_t>(m) * 128))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < CPR; ++q) {
+                const bool have = cc + q <= c_hi;
+                const float *p = slot_ptr(have ? cc + q : cc);
+#pragma unroll
+                for (int r = 0; r < ROWS; ++r) {
+                    const int m = m0 + 4 * r;
+                    v[q][r] = (have && m < M) ? __ldcg(reinterpret_cast<const float4 *>(p + static_cast<int64_t>(m) * 128))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
 #pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                acc[r].x += v0[r].x; acc[r].y += v0[r].y; acc[r].z += v0[r].z; acc[r].w += v0[r].w;
-                if (two) {
-                    acc[r].x += v1[r].x; acc[r].y += v1[r].y; acc[r].z += v1[r].z; acc[r].w += v1[r].w;
+            for (int q = 0; q < CPR; ++q) {
+                if (cc + q > c_hi) break;
+#pragma unroll
+                for (int r = 0; r < ROWS; ++r) {
+                    acc[r].x += v[q][r].x; acc[r].y += v[q][r].y; acc[r].z += v[q][r].z; acc[r].w += v[q][r].w;
                 }
             }
         }

@@ -393,25 +393,45 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     // Work units: K blocks [kb0, kb1) of one tile.  Static and CLC
     // schedules: whole tiles from next_tile.  Stream-K: the pieces of this
     // cluster's range [it_begin, it_end) of the (tile, K block) iterations
-    // (K fastest), one piece per tile the range touches.
+    // (K fastest), one piece per tile the range touches.  The split pieces
+    // (a range boundary inside the tile: at most the first and the last)
+    // run first, so the tiles shared with the neighbouring clusters are
+    // complete early and their fix-ups overlap this cluster's whole tiles
+    // instead of ending the launch.
     struct Unit {
         int tile, kb0, kb1;
     };
     const int64_t sk_total = static_cast<int64_t>(num_tiles) * num_kb;
     const int64_t it_begin = Cfg::SK ? (static_cast<int64_t>(cluster_id) * sk_total) / num_clusters : 0;
     const int64_t it_end = Cfg::SK ? (static_cast<int64_t>(cluster_id + 1) * sk_total) / num_clusters : 0;
-    auto sk_unit = [&](int64_t it) -> Unit {
+    const int64_t sk_tile0 = it_begin / num_kb;
+    const int sk_units = it_end > it_begin ? static_cast<int>((it_end - 1) / num_kb - sk_tile0 + 1) : 0;
+    auto sk_range_unit = [&](int i) -> Unit {        // the i-th piece in range order
         Unit u;
-        u.tile = static_cast<int>(it / num_kb);
+        u.tile = static_cast<int>(sk_tile0 + i);
         const int64_t t0 = static_cast<int64_t>(u.tile) * num_kb;
-        u.kb0 = static_cast<int>(it - t0);
-        u.kb1 = static_cast<int>(min(it_end, t0 + num_kb) - t0);
+        u.kb0 = static_cast<int>(max(it_begin - t0, int64_t(0)));
+        u.kb1 = static_cast<int>(min(it_end - t0, static_cast<int64_t>(num_kb)));
         return u;
+    };
+    auto whole = [&](const Unit &u) { return u.kb0 == 0 && u.kb1 == num_kb; };
+    const bool sk_split_first = Cfg::SK && sk_units > 0 && !whole(sk_range_unit(0));
+    const bool sk_split_last = Cfg::SK && sk_units > 1 && !whole(sk_range_unit(sk_units - 1));
+    auto sk_order = [&](int j) -> int {              // range position of the j-th piece run
+        if (sk_split_last) {
+            if (j == 0) return sk_units - 1;
+            --j;
+        }
+        if (sk_split_first) {
+            if (j == 0) return 0;
+            --j;
+        }
+        return (sk_split_first ? 1 : 0) + j;
     };
     auto first_unit = [&](Unit &u) -> bool {
         if constexpr (Cfg::SK) {
-            if (it_begin >= it_end) return false;
-            u = sk_unit(it_begin);
+            if (sk_units == 0) return false;
+            u = sk_range_unit(sk_order(0));
             return true;
         } else {
             u = Unit{cluster_id, 0, num_kb};
@@ -421,11 +441,9 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     // j counts the units this role has finished (the CLC ring position)
     auto next_unit = [&](Unit &u, uint32_t j, bool &ok) -> bool {
         if constexpr (Cfg::SK) {
-            (void)j;
             (void)ok;
-            const int64_t it = static_cast<int64_t>(u.tile) * num_kb + u.kb1;
-            if (it >= it_end) return false;
-            u = sk_unit(it);
+            if (static_cast<int>(j) + 1 >= sk_units) return false;
+            u = sk_range_unit(sk_order(static_cast<int>(j) + 1));
             return true;
         } else {
             const int n = next_tile(u.tile, j, ok);

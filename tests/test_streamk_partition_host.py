@@ -38,3 +38,36 @@ def test_stream_k_ranges_contributors_and_slots(tiles, nkb, resident):
             for c in contrib:
                 first, last = ranges[c][0] // nkb, (ranges[c][1] - 1) // nkb
                 assert t in (first, last)
+
+
+def run_order(lo, hi, nkb):
+    """The order a cluster runs the pieces of its range [lo, hi): split
+    pieces (the last, then the first) before the whole tiles, the rest in
+    range order -- the sequence the kernel's producer, MMA and epilogue
+    roles all walk."""
+    t0 = lo // nkb
+    units = (hi - 1) // nkb - t0 + 1
+
+    def piece(i):
+        t = t0 + i
+        return t, max(lo - t * nkb, 0), min(hi - t * nkb, nkb)
+
+    whole = lambda p: p[1] == 0 and p[2] == nkb  # noqa: E731
+    split_first = units > 0 and not whole(piece(0))
+    split_last = units > 1 and not whole(piece(units - 1))
+    order = ([units - 1] if split_last else []) + ([0] if split_first else [])
+    order += list(range(1 if split_first else 0, units - 1 if split_last else units))
+    return [piece(i) for i in order], split_first, split_last
+
+
+@pytest.mark.parametrize("tiles,nkb", [(1, 2), (3, 5), (7, 3), (128, 128), (192, 32), (256, 64)])
+def test_stream_k_runs_each_piece_once_split_pieces_first(tiles, nkb):
+    T, G, ranges = partition(tiles, nkb, 74)
+    for lo, hi in ranges:
+        pieces, split_first, split_last = run_order(lo, hi, nkb)
+        covered = sorted((t * nkb + a, t * nkb + b) for t, a, b in pieces)
+        assert covered[0][0] == lo and covered[-1][1] == hi
+        assert all(x[1] == y[0] for x, y in zip(covered, covered[1:]))      # each iteration once
+        n_split = int(split_first) + int(split_last)
+        assert all(not (a == 0 and b == nkb) for _, a, b in pieces[:n_split])
+        assert all(a == 0 and b == nkb for _, a, b in pieces[n_split:])
