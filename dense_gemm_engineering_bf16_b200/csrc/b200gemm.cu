@@ -44,6 +44,10 @@ using Cfg2x256F32S = b200::GemmBf16Cfg<2, 256, 6, 0, false, 1, true>;
 using Cfg2x256B16S = b200::GemmBf16Cfg<2, 256, 6, 1, false, 1, true>;
 // pair tiles 256 x 224 (fp32 C: 7 chunks of 32 columns), static grid
 using Cfg2x224F32 = b200::GemmBf16Cfg<2, 224, 6, 0>;
+// the 256 x 256 CLC pair kernel storing every chunk to further copies of C
+// (gemm_bf16_allgather)
+using Cfg2x256F32CP = b200::GemmBf16Cfg<2, 256, 6, 0, true, 1, false, true>;
+using Cfg2x256B16CP = b200::GemmBf16Cfg<2, 256, 6, 1, true, 1, false, true>;
 using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
@@ -54,6 +58,8 @@ using CfgSk256F32 = b200::GemmSkinnyCfg<256, 4, 0>;
 using CfgSk256B16 = b200::GemmSkinnyCfg<256, 4, 1>;
 
 constexpr int kMaxDevices = 64;
+// internal configuration slot of the CLC pair kernel with further copies of C
+constexpr gemm_config_t kCfgAllgather = static_cast<gemm_config_t>(GEMM_CFG_COUNT_);
 
 struct DeviceState {
     bool ready = false;
@@ -65,8 +71,8 @@ struct DeviceState {
     DeviceStatus *status = nullptr;
     DeviceStatus *noalloc_status = nullptr;
     // per (config, out type): smem attribute set, co-resident clusters
-    bool attr_done[GEMM_CFG_COUNT_][2] = {};
-    int max_clusters[GEMM_CFG_COUNT_][2] = {};
+    bool attr_done[GEMM_CFG_COUNT_ + 1][2] = {};     // + the all-gather kernel (kCfgAllgather)
+    int max_clusters[GEMM_CFG_COUNT_ + 1][2] = {};
     // block-scaled path: kernel attributes (1-CTA, pair), repacked-scale workspace
     bool mx_attr_done[2] = {};
     int mx_max_clusters[2] = {};
@@ -318,12 +324,20 @@ gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStre
 
 // `status`: the watchdog status block the kernel records a timeout in.
 template <class Cfg>
+// `peers`: the further copies of C of a PEERS configuration (else unused).
 gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t cfg_id, const void *A,
                           const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
                           int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi = b200::plain_epilogue(),
-                          uint32_t layout = 0) {
+                          uint32_t layout = 0, const b200::PeerC *peers = nullptr) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
+    typename Cfg::PeerArg peer_arg{};
+    if constexpr (Cfg::PEERS) {
+        if (!peers) return GEMM_ERR_INVALID_VALUE;
+        peer_arg = *peers;
+    } else {
+        (void)peers;
+    }
     // MN-major tiles arrive as 64-wide boxes: whole boxes per CTA only
     if (((layout & b200::kLayoutBMajorN) && Cfg::B_ROWS % 64) || ((layout & b200::kLayoutAMajorM) && Cfg::BM_CTA % 64))
         return GEMM_ERR_INVALID_VALUE;
@@ -419,7 +433,7 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     }
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
                            static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), wave_tiles, status,
-                           watchdog_ns(K), inject_flags(), epi, layout, sk_partials, sk_counters, epoch);
+                           watchdog_ns(K), inject_flags(), epi, layout, sk_partials, sk_counters, epoch, peer_arg);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }
@@ -804,6 +818,54 @@ gemm_status_t gemm_bf16(const void *A, const void *B, void *C, int64_t M, int64_
                         int64_t lda, int64_t ldb, int64_t ldc, gemm_out_t c_type, cudaStream_t stream) {
     return gemm_bf16_ex(A, B, C, M, N, K, lda, ldb, ldc, c_type, GEMM_LAYOUT_KMAJOR, GEMM_LAYOUT_KMAJOR, 1.0f, 0.0f,
                         stream);
+}
+
+gemm_status_t gemm_bf16_allgather(const void *A, const void *B, void *const *C_dst, int n_dst, int64_t M,
+                                  int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int64_t row0,
+                                  gemm_out_t c_type, cudaStream_t stream) {
+    if (c_type != GEMM_OUT_F32 && c_type != GEMM_OUT_BF16) return GEMM_ERR_INVALID_VALUE;
+    if (!C_dst || n_dst < 1 || n_dst > 1 + b200::kMaxPeerC || row0 < 0) return GEMM_ERR_INVALID_VALUE;
+    const int64_t ec = c_type == GEMM_OUT_F32 ? 4 : 2;
+    if (row0 > kMaxDim - M) return GEMM_ERR_TOO_LARGE;
+    // each destination's slab: rows [row0, row0 + M) of a C with leading dimension ldc
+    void *slab[1 + b200::kMaxPeerC];
+    gemm_status_t s = GEMM_OK;
+    for (int d = 0; d < n_dst; ++d) {
+        if (!C_dst[d]) return GEMM_ERR_INVALID_VALUE;
+        if (!aligned16(C_dst[d])) return GEMM_ERR_MISALIGNED;
+        slab[d] = static_cast<uint8_t *>(C_dst[d]) + row0 * ldc * ec;
+        if ((s = check_args(A, B, slab[d], M, N, K, lda, ldb, ldc, 2, 2, ec)) != GEMM_OK) return s;
+        for (int e = 0; e < d; ++e)   // two destinations may not share bytes of the slab
+            if (overlaps(slab[d], M, N, ldc, ec, slab[e], M, N, ldc, ec)) return GEMM_ERR_ALIAS;
+    }
+    if (M == 0 || N == 0) return GEMM_OK;
+    int dev;
+    DeviceState *st;
+    if ((s = current_device_alloc(dev, st, stream)) != GEMM_OK) return s;
+    const bool f32 = c_type == GEMM_OUT_F32;
+    if (K == 0) {
+        for (int d = 0; d < n_dst && s == GEMM_OK; ++d)
+            s = f32 ? launch_zero<uint32_t>(slab[d], M, N, ldc, st->sm_count, stream)
+                    : launch_zero<uint16_t>(slab[d], M, N, ldc, st->sm_count, stream);
+        return s;
+    }
+    // The copies beyond the first: a tensor map of the slab in each (the same
+    // box as the kernel's own C map) and the slab's base for the row ends.
+    b200::PeerC peers{};
+    peers.count = n_dst - 1;
+    const int64_t n_tma = (N * ec / 16) * 16 / ec;
+    const CUtensorMapDataType cdt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint32_t box_cols = f32 ? Cfg2x256F32CP::EPI_COLS : Cfg2x256B16CP::EPI_COLS;
+    for (int d = 1; d < n_dst; ++d) {
+        if ((s = encode_2d(&peers.map[d - 1], cdt, slab[d], n_tma > 0 ? n_tma : 16 / ec, M, ldc * ec, box_cols, 32)) !=
+            GEMM_OK)
+            return s;
+        peers.base[d - 1] = slab[d];
+    }
+    return f32 ? launch_bf16<Cfg2x256F32CP>(st, st->status, kCfgAllgather, A, B, slab[0], M, N, K, lda, ldb, ldc,
+                                             stream, b200::plain_epilogue(), 0u, &peers)
+               : launch_bf16<Cfg2x256B16CP>(st, st->status, kCfgAllgather, A, B, slab[0], M, N, K, lda, ldb, ldc,
+                                             stream, b200::plain_epilogue(), 0u, &peers);
 }
 
 gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const void *B, const uint8_t *sfb, void *C,

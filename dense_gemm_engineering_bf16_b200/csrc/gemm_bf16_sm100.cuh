@@ -49,6 +49,7 @@
 #include <cuda_bf16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -81,13 +82,30 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     return p;
 }
 
-template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1, bool SK_ = false>
+// More copies of C for the row-sharded GEMM with its all-gather fused in:
+// the epilogue stores every finished chunk of the slab to up to kMaxPeerC
+// further destinations (other GPUs' C through their mapped pointers), each
+// described by a tensor map of the slab in that C and the slab's base
+// pointer there (for the plain stores of each row's ragged end).
+constexpr int kMaxPeerC = 7;
+struct PeerC {
+    CUtensorMap map[kMaxPeerC];
+    void *base[kMaxPeerC];
+    int count;
+};
+struct NoPeerC {};
+
+template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1, bool SK_ = false,
+          bool PEERS_ = false>
 struct GemmBf16Cfg {
     static constexpr bool CLC = CLC_;              // tiles from Cluster Launch Control, not a fixed stride
     // Stream-K: the (tile, K block) iterations are cut into one contiguous
     // range per cluster; a tile split between clusters is summed from fp32
     // partials by the last of its contributors, in contributor order.
     static constexpr bool SK = SK_;
+    // PEERS: every chunk of C is also stored to the destinations of a PeerC
+    static constexpr bool PEERS = PEERS_;
+    using PeerArg = std::conditional_t<PEERS_, PeerC, NoPeerC>;
     static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
     static constexpr int BN = BN_;                 // tile N == MMA N
     static constexpr int STAGES = STAGES_;         // shared-memory ring depth
@@ -124,6 +142,7 @@ struct GemmBf16Cfg {
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
     static_assert(CONSUMERS == 1 || CONSUMERS == 2, "one or two MMA consumers");
     static_assert(!SK || (!CLC && CONSUMERS == 1 && BN % 4 == 0), "stream-K: static schedule, one consumer");
+    static_assert(!PEERS || !SK, "a stream-K fix-up writes C with plain stores to one C only");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
     static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows <= 256, whole 8-row swizzle atoms");
     static_assert(BN % EPI_COLS == 0, "epilogue chunks cover the tile");
@@ -294,7 +313,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m, int wave_tiles,
                        DeviceStatus *status, uint64_t timeout_ns, uint32_t inject,
                        Epilogue epi, uint32_t layout,
-                       float *sk_partials, unsigned long long *sk_counters, uint32_t sk_epoch) {
+                       float *sk_partials, unsigned long long *sk_counters, uint32_t sk_epoch,
+                       const __grid_constant__ typename Cfg::PeerArg peers) {
     constexpr int CG = Cfg::CG;
     const bool a_mn = (layout & kLayoutAMajorM) != 0;   // A stored K x M
     const bool b_mn = (layout & kLayoutBMajorN) != 0;   // B stored K x N
@@ -660,19 +680,25 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     // (< 16 bytes per row) go out as plain predicated stores.
                     const int row = row0 + static_cast<int>(lane);
                     if (row < M) {
-                        uint8_t *crow = static_cast<uint8_t *>(C) + static_cast<int64_t>(row) * ldc * (Cfg::OUT == 0 ? 4 : 2);
+                        const int64_t roff = static_cast<int64_t>(row) * ldc * (Cfg::OUT == 0 ? 4 : 2);
+                        auto tail = [&](void *dst) {
+                            uint8_t *crow = static_cast<uint8_t *>(dst) + roff;
 #pragma unroll
-                        for (int w = 0; w < Cfg::EPI_COLS; ++w) {
-                            const int col = cstart + w;
-                            if (col >= n_tma && col < N) {
-                                if constexpr (Cfg::OUT == 0) {
-                                    reinterpret_cast<uint32_t *>(crow)[col] = packed[w];
-                                } else {
-                                    reinterpret_cast<uint16_t *>(crow)[col] =
-                                        static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
+                            for (int w = 0; w < Cfg::EPI_COLS; ++w) {
+                                const int col = cstart + w;
+                                if (col >= n_tma && col < N) {
+                                    if constexpr (Cfg::OUT == 0) {
+                                        reinterpret_cast<uint32_t *>(crow)[col] = packed[w];
+                                    } else {
+                                        reinterpret_cast<uint16_t *>(crow)[col] =
+                                            static_cast<uint16_t>(packed[w >> 1] >> (16 * (w & 1)));
+                                    }
                                 }
                             }
-                        }
+                        };
+                        tail(C);
+                        if constexpr (Cfg::PEERS)
+                            for (int d = 0; d < peers.count; ++d) tail(peers.base[d]);
                     }
                     if (cstart >= n_tma) return;            // nothing left for the TMA store
                 }
@@ -691,6 +717,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 __syncwarp();
                 if (lane == 0) {
                     tma_store_2d(&tmC, sbuf, cstart, row0);
+                    if constexpr (Cfg::PEERS)   // the same staged chunk to every other C
+                        for (int d = 0; d < peers.count; ++d) tma_store_2d(&peers.map[d], sbuf, cstart, row0);
                     bulk_commit_group();
                 }
                 ++nstore;

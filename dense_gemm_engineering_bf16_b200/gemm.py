@@ -64,6 +64,9 @@ lib.gemm_bf16_ex.restype = _int
 lib.gemm_bf16_fused.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int,
                                 ctypes.c_float, ctypes.c_float, _vp, _int, _vp]
 lib.gemm_bf16_fused.restype = _int
+lib.gemm_bf16_allgather.argtypes = [_vp, _vp, ctypes.POINTER(_vp), _int, _i64, _i64, _i64, _i64, _i64, _i64,
+                                    _i64, _int, _vp]
+lib.gemm_bf16_allgather.restype = _int
 lib.gemm_mxfp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]
 lib.gemm_mxfp8.restype = _int
 lib.gemm_check_device_status.argtypes = [_vp]
@@ -150,6 +153,18 @@ def gemm_bf16_fused(A, B, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: in
                              int(b_layout), float(alpha), float(beta), _ptr(bias) if bias is not None else None,
                              int(act), _stream(stream))
     return _check(st, "gemm_bf16_fused", check)
+
+
+def gemm_bf16_allgather(A, B, C_dst, M: int, N: int, K: int, lda: int, ldb: int, ldc: int, row0: int,
+                        c_type: int = OUT_F32, stream=None, check: bool = True) -> int:
+    """This GPU's slab C[row0:row0+M] = A.B written into every C of C_dst
+    (this GPU's own C first, then other GPUs' mapped C buffers): a row-
+    sharded GEMM with its all-gather in the write-back (see
+    include/b200gemm.h, gemm_bf16_allgather)."""
+    ptrs = (_vp * len(C_dst))(*[_ptr(c) for c in C_dst])
+    st = lib.gemm_bf16_allgather(_ptr(A), _ptr(B), ptrs, len(C_dst), M, N, K, lda, ldb, ldc, row0, int(c_type),
+                                 _stream(stream))
+    return _check(st, "gemm_bf16_allgather", check)
 
 
 def gemm_mxfp8(A, sfa, B, sfb, C, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,

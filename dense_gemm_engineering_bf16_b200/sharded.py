@@ -9,11 +9,18 @@ the distributed step the tile ledger of "GPU 执行模型" (section "Tile
 only C's slabs cross the interconnect.
 
 One process per GPU (torch.distributed, NCCL over NVLink / NVSwitch on a GPU
-node; gloo for host-side tests).  The slab compute is one ``gemm_bf16`` call
-writing straight into this rank's rows of C (no staging copy); the gather is
-one broadcast per rank of that rank's rows, in rank order, so slabs of
-unequal height need no padding.  Every rank issues the same collectives in
-the same order.
+node; gloo for host-side tests).  Two forms:
+
+* collective: the slab compute is one ``gemm_bf16`` call writing straight
+  into this rank's rows of C (no staging copy); the gather is one broadcast
+  per rank of that rank's rows, in rank order, so slabs of unequal height
+  need no padding.  Every rank issues the same collectives in the same order.
+* fused (``peer_c`` given): one ``gemm_bf16_allgather`` kernel computes the
+  slab and its epilogue stores every finished chunk into this rank's C and
+  into every other rank's C (their buffers mapped into this process, e.g. by
+  CUDA IPC or symmetric memory), so the transfer overlaps the math; a barrier
+  then tells every rank that all slabs have landed.  No TMA load reads another
+  GPU's memory: only the epilogue's stores cross NVLink.
 """
 from __future__ import annotations
 
@@ -75,7 +82,7 @@ def gather_rows(C, parts: Sequence[Tuple[int, int]], rank: int, group=None) -> N
 
 
 def gemm_bf16_msharded(A_slab, B, C, M: int, N: int, K: int, c_type: int = 0, group=None, stream=None,
-                       slab_gemm: Callable | None = None) -> Tuple[int, int]:
+                       slab_gemm: Callable | None = None, peer_c: Sequence | None = None) -> Tuple[int, int]:
     """C = A.B with A's rows sharded over the ranks of `group`.
 
     A_slab  this rank's rows [m0, m1) of A, a (m1 - m0) x K bf16 tensor,
@@ -86,6 +93,11 @@ def gemm_bf16_msharded(A_slab, B, C, M: int, N: int, K: int, c_type: int = 0, gr
             holds all of C.
     stream  the CUDA stream of the slab GEMM (None: the current stream); the
             gather is ordered after it.
+    peer_c  fused form: the other ranks' C buffers (tensors or device
+            pointers mapped into this process, same shape and leading
+            dimension as C), in any order.  This rank's slab is written into
+            C and into each of them by one kernel; the call then waits at a
+            barrier of `group` until every rank's kernel has finished.
     The slab boundaries are row_partition(M, world).  Returns (m0, m1).
 
     `slab_gemm(A_slab, B, C_rows, m, N, K, lda, ldb, ldc, c_type, stream)`
@@ -101,6 +113,22 @@ def gemm_bf16_msharded(A_slab, B, C, M: int, N: int, K: int, c_type: int = 0, gr
         raise ValueError(f"rank {rank} holds {A_slab.shape[0]} rows of A; its slab is rows [{m0}, {m1})")
     if C.shape[0] != M or C.shape[1] < N:
         raise ValueError("C must be the whole M x N output on every rank")
+    if peer_c is not None:
+        import torch
+        from . import gemm as G
+        if len(peer_c) > 7:
+            raise ValueError("the fused form reaches at most 7 other ranks per kernel")
+        if m1 > m0:
+            G.gemm_bf16_allgather(A_slab, B, [C] + list(peer_c), m1 - m0, N, K, A_slab.stride(0), B.stride(0),
+                                  C.stride(0), m0, c_type, stream)
+        # every rank's kernel must have finished writing before anyone reads C
+        cur = torch.cuda.current_stream()
+        if stream is not None and stream != cur:
+            cur.wait_stream(stream)
+        if dist.get_backend(group) != "nccl":
+            cur.synchronize()
+        dist.barrier(group=group)
+        return m0, m1
     if slab_gemm is None:
         from . import gemm as G
         slab_gemm = G.gemm_bf16

@@ -200,6 +200,40 @@ B200GEMM_API gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C
                                            cudaStream_t stream);
 
 /*
+ * gemm_bf16_allgather: one GPU's part of a row-sharded C = A . B with the
+ * all-gather of C fused into the GEMM's write-back.
+ *
+ * With A's rows split over G GPUs (each holding its slab of A and all of B),
+ * every GPU computes its rows of C and every GPU needs all of C: the GEMM is
+ * followed by an all-gather.  Here one kernel does both: each finished chunk
+ * of this GPU's slab goes from shared memory straight into every destination
+ * C by TMA stores, so the transfer to the other GPUs overlaps the next tiles'
+ * math instead of following the whole GEMM.  (The row-sharded GEMM is the
+ * distributed step the tile ledger of "GPU 执行模型", section "Tile 小账本",
+ * leaves to a later chapter; fusing its gather into the epilogue is this
+ * library's design.)
+ *
+ *   A, B      this GPU's slab of A (M rows, row-major, lda >= K) and all of B
+ *             (stored N x K, ldb >= K), bf16, on this GPU.
+ *   C_dst     HOST array of n_dst (1 .. 8) pointers, each the base of a whole
+ *             C (c_type, leading dimension ldc >= N, at least row0 + M rows):
+ *             this GPU's own C first, then the other GPUs' C buffers mapped
+ *             into this process (CUDA IPC or symmetric memory).  The slab is
+ *             written to rows [row0, row0 + M) of every one of them.
+ *   M, N, K   the slab's rows, C's columns, the reduction length.
+ *   row0      the slab's first row in C.
+ *   Other rules (alignment, leading dimensions, tails, K == 0) as gemm_bf16;
+ *   no destination's slab may overlap A, B or another destination's slab.
+ * It runs the 256 x 256 CTA-pair kernel with Cluster Launch Control.  The
+ * call orders nothing across GPUs: a GPU may read its C only after every
+ * GPU's call has finished (for example a barrier on each stream after the
+ * call).  No TMA load ever reads another GPU's memory; only stores cross.
+ */
+B200GEMM_API gemm_status_t gemm_bf16_allgather(const void *A, const void *B, void *const *C_dst, int n_dst,
+                                               int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                                               int64_t ldc, int64_t row0, gemm_out_t c_type, cudaStream_t stream);
+
+/*
  * gemm_mxfp8: block-scaled C = (sa . A) . (sb . B) with FP8 E4M3 A and B and
  * one E8M0 scale per 32 consecutive K elements of every row of A and of the
  * K-major B -- the block-scaled MMA with its scale factors in tensor memory

@@ -65,3 +65,29 @@ def test_two_ranks_on_one_gpu_gather_the_whole_product(dist_name):
             assert np.array_equal(got, oracle.round_f32(c_ref).astype(np.float64)), f"rank {rank}"
         else:
             assert np.all(np.abs(got - c_ref) <= 1e-3 * s_abs + 1e-6), f"rank {rank}"
+
+
+def test_fused_form_writes_every_copy_on_one_rank():
+    """The fused form's Python path, one rank (gloo): this rank's slab (all of
+    C) goes into C and into two more buffers standing in for other ranks' C."""
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from dense_gemm_engineering_bf16_b200 import sharded, synth
+    import os
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        M, N, K = 700, 520, 512
+        a_bits, b_bits = synth.bf16_operands(M, N, K, "ints", workload=132)
+        A = torch.from_numpy(a_bits.view(np.int16)).cuda().view(torch.bfloat16)
+        B = torch.from_numpy(b_bits.view(np.int16)).cuda().view(torch.bfloat16)
+        C = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        peers = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(2)]
+        assert sharded.gemm_bf16_msharded(A, B, C, M, N, K, peer_c=peers) == (0, M)
+        want = oracle.round_f32(oracle.gemm_bf16_f64(a_bits, b_bits, K=K))
+        for t in [C] + peers:
+            assert np.array_equal(t.cpu().numpy().view(np.uint32), want.view(np.uint32))
+    finally:
+        dist.destroy_process_group()
