@@ -628,6 +628,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t ew = warp - 2u;             // staging slot
         const bool fused = !epi.identity();
         const uint32_t stage_base = base + Cfg::STAGES * Cfg::STAGE_BYTES + ew * 2u * Cfg::EPI_BUF;
+        const uint64_t c_policy = l2_policy_evict_first();
         uint32_t nstore = 0;
         int t = 0;
         Unit u;
@@ -716,7 +717,9 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmC, sbuf, cstart, row0);
+                    // C is written once and never read back by this kernel:
+                    // its lines go first, so the A and B panels stay in L2
+                    tma_store_2d_hint(&tmC, sbuf, cstart, row0, c_policy);
                     if constexpr (Cfg::PEERS)   // the same staged chunk to every other C
                         for (int d = 0; d < peers.count; ++d) tma_store_2d(&peers.map[d], sbuf, cstart, row0);
                     bulk_commit_group();
