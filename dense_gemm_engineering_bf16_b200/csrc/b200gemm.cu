@@ -283,41 +283,70 @@ gemm_status_t encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void 
 
 // --------------------------------------------------------------- launches --
 
+// Predicted time (us) of one launch of a dense configuration on a B200 (148
+// SMs): a fixed cost plus, per wave of tiles, the work one SM does in it
+// (tile rows x columns x K, a pair tile's split over its two SMs), at the
+// configuration's own rate.  The constants are least-squares fits to event
+// timings of every configuration over about 60 shapes from 64 x 4096 x 4096
+// to 4096^3 (fp32 C, L2 flushed before each call): the autotuning search
+// over tile shape and persistent strategy ("GPU 执行模型", section "编译与
+// autotune"), run once offline so that no call pays for it.  They rank the
+// candidates; they are not a performance claim.
+struct CostModel {
+    int tile_m, tile_n, slots;   // tile, co-resident tiles (one per SM or per pair)
+    double fixed_us, us_per_gunit;
+};
+double predicted_us(const CostModel &c, int64_t M, int64_t N, int64_t K) {
+    const int64_t tiles = ((M + c.tile_m - 1) / c.tile_m) * ((N + c.tile_n - 1) / c.tile_n);
+    const int64_t waves = (tiles + c.slots - 1) / c.slots;
+    const double per_sm = static_cast<double>(c.tile_m) * c.tile_n / (c.slots == 74 ? 2.0 : 1.0);
+    return c.fixed_us + c.us_per_gunit * 1e-9 * static_cast<double>(waves) * per_sm * static_cast<double>(K);
+}
+
 gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     const int forced = g_forced.load(std::memory_order_relaxed);
     if (forced != GEMM_CFG_AUTO && forced != GEMM_CFG_MXFP8_1CTA_128x256 && forced != GEMM_CFG_MXFP8_2CTA_256x256)
         return static_cast<gemm_config_t>(forced);
-    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    const int64_t wide_tiles = ((M + 127) / 128) * ((N + 255) / 256);
-    // two or more waves of pair tiles: Cluster Launch Control evens out the
-    // tail; a single wave: the static persistent schedule
-    // two or more waves of 512 x 256 tiles: two MMA consumers share each B
-    // k-tile (25% fewer operand bytes into shared memory per FLOP, which
-    // under the power cap buys clock); fewer: the double-buffered 256 x 256
-    const int64_t tall_tiles = ((M + 511) / 512) * ((N + 255) / 256);
-    if (tall_tiles >= 148) return GEMM_CFG_2CTA_512x256_CLC;
-    if (pair_tiles >= 74) {
-        // The last wave of pair tiles: when it leaves more than a tenth of
-        // the pairs idle and 256 x 224 tiles fill the waves better (e.g.
-        // 1000 x 8192: 148 tiles, two full waves, against 128 tiles in two
-        // waves of 256 x 256), take those.  (Stream-K, GEMM_CFG_2CTA_256x256_SK,
-        // evens out the waves too, but its fix-up of split tiles cost more
-        // than it saved on 4096^3 and 4000 x 3000 x 2000: it is not chosen.)
-        const int64_t waves = (pair_tiles + 73) / 74;
-        if (pair_tiles * 10 < waves * 74 * 9) {
-            const int64_t tiles224 = ((M + 255) / 256) * ((N + 223) / 224);
-            const int64_t waves224 = (tiles224 + 73) / 74;
-            if (waves224 * 224 * 100 <= waves * 256 * 92) return GEMM_CFG_2CTA_256x224;
+    // A few rows and a long K: swap A and B and split K over every SM (the
+    // skinny stream-K kernel).  Its fix-up of 128 x MP fp32 partials grows
+    // with M, so past 64 rows (or with a shorter K) whole tiles win.
+    if (M <= 64 && K >= 8192) return GEMM_CFG_SKINNY;
+    if (M <= 32 && K >= 4096) return GEMM_CFG_SKINNY;
+    // Every 128 x 128 tile on an SM of its own: the most SMs streaming.
+    if (((M + 127) / 128) * ((N + 127) / 128) <= 148) return GEMM_CFG_1CTA_128x128;
+    struct Candidate {
+        gemm_config_t cfg;
+        CostModel cost;
+    };
+    static constexpr Candidate kCandidates[] = {
+        {GEMM_CFG_1CTA_128x256, {128, 256, 148, 9.51, 192.3}},
+        {GEMM_CFG_2CTA_256x256, {256, 256, 74, 11.90, 178.6}},
+        {GEMM_CFG_2CTA_256x256_CLC, {256, 256, 74, 12.78, 169.5}},
+        {GEMM_CFG_2CTA_512x256_CLC, {512, 256, 74, 16.90, 151.95}},
+        {GEMM_CFG_1CTA_128x256_CLC, {128, 256, 148, 9.19, 198.7}},
+    };
+    gemm_config_t best = GEMM_CFG_1CTA_128x128;
+    double best_us = 0.0;
+    for (const Candidate &c : kCandidates) {
+        const CostModel &m = c.cost;
+        const int64_t waves = (((M + m.tile_m - 1) / m.tile_m) * ((N + m.tile_n - 1) / m.tile_n) + m.slots - 1) / m.slots;
+        // One-CTA 256-wide tiles load 50 % more operand bytes per FLOP than
+        // a pair's: past two waves L2 cannot feed them.  The 512 x 256 tile
+        // holds one tile in TMEM, so its drain is not hidden behind the
+        // next tile's MMAs: it pays off only over a long K.
+        if ((c.cfg == GEMM_CFG_1CTA_128x256 || c.cfg == GEMM_CFG_1CTA_128x256_CLC) && waves > 2) continue;
+        if ((c.cfg == GEMM_CFG_2CTA_512x256_CLC || c.cfg == GEMM_CFG_1CTA_128x256_CLC) && K < 8192) continue;
+        // a later candidate must win by more than the model's noise
+        const double us = predicted_us(m, M, N, K);
+        if (best_us == 0.0 || us < best_us * 0.98) {
+            best = c.cfg;
+            best_us = us;
         }
-        return pair_tiles >= 148 ? GEMM_CFG_2CTA_256x256_CLC : GEMM_CFG_2CTA_256x256;
     }
-    // few rows, too few tiles to fill the SMs, and a long K to split: stream-K.
-    // (A short K gains nothing from splitting; the plain 128 x 128 kernel has
-    // the lower fixed cost there: 4.8 vs 9.6 us at 128^3 under graph replay.)
-    const int64_t small_tiles = ((M + 127) / 128) * ((N + 127) / 128);
-    if (M <= 256 && K >= 1024 && small_tiles < 148) return GEMM_CFG_SKINNY;
-    if (wide_tiles >= 148) return GEMM_CFG_1CTA_128x256;
-    return GEMM_CFG_1CTA_128x128;
+    // Over a short K, the static pair schedule beats Cluster Launch Control:
+    // a tile is too short for the scheduler round trip to hide.
+    if (best == GEMM_CFG_2CTA_256x256_CLC && K <= 2048) best = GEMM_CFG_2CTA_256x256;
+    return best;
 }
 
 gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStream_t stream);

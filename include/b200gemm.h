@@ -104,8 +104,9 @@ typedef enum {
                                        tanh approximation (PTX tanh.approx.f32) */
 } gemm_act_t;
 
-/* Kernel configurations.  GEMM_CFG_AUTO picks by shape; the others force a
- * configuration (for tests and benchmarks) through gemm_force_config(). */
+/* Kernel configurations.  GEMM_CFG_AUTO picks by shape (gemm_select_config);
+ * the others force a configuration (for tests and benchmarks) through
+ * gemm_force_config(). */
 typedef enum {
     GEMM_CFG_AUTO = 0,
     GEMM_CFG_1CTA_128x256 = 1,      /* one CTA per tile, tile 128 x 256, tcgen05 cta_group::1 */
@@ -121,16 +122,17 @@ typedef enum {
     GEMM_CFG_MXFP8_2CTA_256x256 = 8,/* gemm_mxfp8: CTA pair per 256 x 256 tile, cta_group::2 */
     GEMM_CFG_2CTA_512x256_CLC = 9,  /* CTA pair per 512 x 256 tile, two MMA consumers sharing each
                                        B k-tile, one TMEM accumulator each (TMEM single-buffered);
-                                       Cluster Launch Control; chosen when there are >= 148
-                                       such tiles (two waves), e.g. 8192 x 8192 */
+                                       Cluster Launch Control; chosen by shape only for K >= 8192,
+                                       e.g. 8192 x 8192 x 8192 */
     GEMM_CFG_2CTA_256x256_SK = 10,  /* CTA pair per 256 x 256 tile, stream-K: every co-resident pair
                                        takes an equal contiguous share of the (tile, 64-wide K block)
                                        iterations; a tile split between pairs is summed from fp32
                                        partials by its last contributor, in contributor order
-                                       (deterministic); uses the library-owned split workspace */
-    GEMM_CFG_2CTA_256x224 = 11,     /* CTA pair per 256 x 224 tile, for shapes whose 224-wide tiles fill
-                                       the waves better; fp32 C with B stored K-major only (bf16 C or
-                                       a B stored K x N runs 2CTA_256x256) */
+                                       (deterministic); uses the library-owned split workspace;
+                                       never chosen by shape */
+    GEMM_CFG_2CTA_256x224 = 11,     /* CTA pair per 256 x 224 tile (fills the waves of some shapes
+                                       better); fp32 C with B stored K-major only (bf16 C or a B
+                                       stored K x N runs 2CTA_256x256); never chosen by shape */
     GEMM_CFG_COUNT_ = 12
 } gemm_config_t;
 
@@ -331,12 +333,21 @@ B200GEMM_API int gemm_last_cuda_error(void);
 B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
 
 /* The configuration the next gemm_bf16 call with this shape would use.
+ * M <= 64 with K >= 8192, or M <= 32 with K >= 4096: GEMM_CFG_SKINNY.
+ * Every 128 x 128 tile on an SM of its own: GEMM_CFG_1CTA_128x128.
+ * Otherwise the configuration with the lowest predicted time among the
+ * 1-CTA 128 x 256 (up to two waves), the 256 x 256 pair (static, or with
+ * Cluster Launch Control when K > 2048) and, for K >= 8192, the 512 x 256
+ * pair tile and the 1-CTA 128 x 256 CLC kernel.  The prediction is a fixed
+ * cost plus the waves of tiles times each SM's work per wave, at rates
+ * measured on a B200: the autotuning search over tile shape and persistent
+ * strategy ("GPU 执行模型", section "编译与 autotune"), done once offline so
+ * that no call pays for it.
  * gemm_bf16_ex and gemm_bf16_fused use it too, except that with a non-plain
  * epilogue (beta != 0, alpha != 1, a bias or an activation) they take
  * GEMM_CFG_2CTA_256x256_CLC where this returns GEMM_CFG_2CTA_512x256_CLC
  * (the 256 x 256 tile's second TMEM buffer hides the longer epilogue), and
- * an A stored K x M never takes GEMM_CFG_SKINNY.  Where this returns
- * GEMM_CFG_2CTA_256x224, bf16 C or a B stored K x N runs GEMM_CFG_2CTA_256x256. */
+ * an A stored K x M never takes GEMM_CFG_SKINNY. */
 B200GEMM_API gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K);
 
 /* Number of kernels that one call queues for this shape: gemm_bf16 /

@@ -66,7 +66,7 @@ def growth_after_capture():
     res = {}
     s = torch.cuda.Stream()
     # skinny: small problem captured, then a large one grows the workspace
-    m, n, k = 16, 256, 1024
+    m, n, k = 16, 256, 4096
     a_bits, b_bits = synth.bf16_operands(m, n, k, "normal", workload=410)
     A, B = dev_bf16(a_bits), dev_bf16(b_bits)
     C = torch.zeros((m, n), dtype=torch.float32, device="cuda")
@@ -76,7 +76,7 @@ def growth_after_capture():
         res["skinny_warm_up"] = call()
     s.synchronize()
     g_sk, res["skinny_capture"] = capture(call, s)
-    big_m, big_n, big_k = 256, 8192, 8192
+    big_m, big_n, big_k = 32, 8192, 8192
     A2 = torch.zeros((big_m, big_k), dtype=torch.bfloat16, device="cuda")
     B2 = torch.zeros((big_n, big_k), dtype=torch.bfloat16, device="cuda")
     C2 = torch.empty((big_m, big_n), dtype=torch.float32, device="cuda")

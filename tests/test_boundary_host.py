@@ -141,20 +141,34 @@ def test_status_strings_and_config_control():
     G.gemm_force_config("mxfp8_2cta_256x256")          # a block-scaled choice leaves bf16 on auto
     assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]
     G.gemm_force_config("auto")
-    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 512 tiles of 512 x 256
-    assert G.gemm_select_config(6144, 6144, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 288
-    # 256 pair tiles (3.46 waves of 74 pairs), 192 (2.6): CLC, since 224-wide tiles do no better
+    # long K, >= a wave of 512 x 256 tiles: the two-consumer tile
+    assert G.gemm_select_config(8192, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]
+    assert G.gemm_select_config(6144, 6144, 8192) == G.CONFIGS["2cta_512x256_clc"]
+    assert G.gemm_select_config(1000, 8192, 8192) == G.CONFIGS["2cta_512x256_clc"]   # 64 tiles, 0.86 wave
+    # K < 8192: its unhidden drain costs more than the shared B saves
     assert G.gemm_select_config(4096, 4096, 4096) == G.CONFIGS["2cta_256x256_clc"]
-    assert G.gemm_select_config(4000, 3000, 2000) == G.CONFIGS["2cta_256x256_clc"]
+    assert G.gemm_select_config(1536, 8192, 8192) == G.CONFIGS["2cta_256x256_clc"]   # 96 tall tiles: 2 waves
+    # K <= 2048: the static pair schedule
+    assert G.gemm_select_config(4000, 3000, 2000) == G.CONFIGS["2cta_256x256"]
+    assert G.gemm_select_config(2048, 8192, 2048) == G.CONFIGS["2cta_256x256"]
+    assert G.gemm_select_config(8192, 8192, 1024) == G.CONFIGS["2cta_256x256"]
+    # up to two waves of one-CTA 128 x 256 tiles: their lower fixed cost wins
+    assert G.gemm_select_config(2048, 2048, 2048) == G.CONFIGS["1cta_128x256"]
+    assert G.gemm_select_config(2560, 3584, 2048) == G.CONFIGS["1cta_128x256"]
+    # every 128 x 128 tile on an SM of its own
     assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
+    assert G.gemm_select_config(300, 1000, 64) == G.CONFIGS["1cta_128x128"]
+    assert G.gemm_select_config(512, 4096, 4096) == G.CONFIGS["1cta_128x128"]
+    assert G.gemm_select_config(256, 8192, 8192) == G.CONFIGS["1cta_128x128"]
+    # a few rows and a long K: the skinny stream-K kernel
     assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
-    # 128 pair tiles of 256 x 256 (1.73 waves) against 148 of 256 x 224 (two full waves)
-    assert G.gemm_select_config(1000, 8192, 8192) == G.CONFIGS["2cta_256x224"]
-    assert G.gemm_select_config(2048, 8192, 2048) == G.CONFIGS["2cta_256x224"]     # 296 tiles: 4 full waves
-    assert G.gemm_select_config(2560, 3584, 2048) == G.CONFIGS["2cta_256x256"]     # 140 tiles: 0.95 of 2 waves
-    assert G.gemm_select_config(4096, 4608, 2048) == G.CONFIGS["2cta_256x256_clc"] # 288 tiles: 0.97 of 4 waves
-    assert G.gemm_select_config(300, 1000, 64) == G.CONFIGS["1cta_128x128"]
+    assert G.gemm_select_config(64, 8192, 8192) == G.CONFIGS["skinny"]
+    assert G.gemm_select_config(64, 4096, 4096) == G.CONFIGS["1cta_128x128"]
+    # the 256 x 224 and stream-K configurations are never chosen by shape
+    seen = {G.gemm_select_config(m, n, k) for m in (1, 100, 300, 1000, 3000, 8192)
+            for n in (64, 1000, 3000, 8192) for k in (16, 1000, 5000, 16384)}
+    assert G.CONFIGS["2cta_256x224"] not in seen and G.CONFIGS["2cta_256x256_sk"] not in seen
     with pytest.raises(G.GemmError):
         G.gemm_bf16(A, B, C, -1, 1, 1, 1, 1, 1, stream=0)
 

@@ -1,4 +1,4 @@
-"""GPU parity of the skinny path (M <= 256): A and B swapped so 128 rows of B
+"""GPU parity of the skinny path (M <= 256, chosen by shape for M <= 64): A and B swapped so 128 rows of B
 fill the MMA, stream-K over every SM, split tiles finished by the last
 contributor in contributor order.  Compared with the oracle element by
 element; integer inputs bit-exact."""
@@ -30,7 +30,11 @@ def _check(M, N, K, dist, workload, c_type=F32, lda=None, config="skinny", repea
 
 def test_auto_selects_skinny_for_small_m():
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
-    assert G.gemm_select_config(256, 4096, 4096) == G.CONFIGS["skinny"]
+    assert G.gemm_select_config(64, 8192, 8192) == G.CONFIGS["skinny"]
+    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
+    # past 64 rows the fp32 partials of the split tiles cost more than the
+    # split saves: whole 128 x 128 tiles, one per SM
+    assert G.gemm_select_config(256, 4096, 4096) == G.CONFIGS["1cta_128x128"]
 
 
 @pytest.mark.parametrize("c_type", [F32, BF16])
