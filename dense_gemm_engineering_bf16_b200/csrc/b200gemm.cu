@@ -48,6 +48,12 @@ using Cfg2x224F32 = b200::GemmBf16Cfg<2, 224, 6, 0>;
 // (gemm_bf16_allgather)
 using Cfg2x256F32CP = b200::GemmBf16Cfg<2, 256, 6, 0, true, 1, false, true>;
 using Cfg2x256B16CP = b200::GemmBf16Cfg<2, 256, 6, 1, true, 1, false, true>;
+// cluster split-K: 2-8 CTAs per tile, each over a share of K, partials summed
+// through distributed shared memory
+using Cfg1x128F32K = b200::GemmBf16Cfg<1, 128, 6, 0, false, 1, false, false, true>;
+using Cfg1x128B16K = b200::GemmBf16Cfg<1, 128, 6, 1, false, 1, false, false, true>;
+using Cfg1x256F32K = b200::GemmBf16Cfg<1, 256, 4, 0, false, 1, false, false, true>;
+using Cfg1x256B16K = b200::GemmBf16Cfg<1, 256, 4, 1, false, 1, false, false, true>;
 using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
@@ -73,6 +79,8 @@ struct DeviceState {
     // per (config, out type): smem attribute set, co-resident clusters
     bool attr_done[GEMM_CFG_COUNT_ + 1][2] = {};     // + the all-gather kernel (kCfgAllgather)
     int max_clusters[GEMM_CFG_COUNT_ + 1][2] = {};
+    // split-K configurations: co-resident CTAs with clusters of 2, 4 and 8
+    int splitk_ctas[GEMM_CFG_COUNT_ + 1][2][3] = {};
     // block-scaled path: kernel attributes (1-CTA, pair), repacked-scale workspace
     bool mx_attr_done[2] = {};
     int mx_max_clusters[2] = {};
@@ -126,6 +134,18 @@ int raster_group_m() {
         return v > 0 ? v : 8;
     }();
     return g;
+}
+
+// Split factor of the split-K configurations: B200GEMM_KSPLIT = 2, 4 or 8
+// forces it (tests: every factor, including shares with no K block); unset,
+// choose_ksplit picks it by shape.  Read once.
+int forced_ksplit() {
+    static const int v = [] {
+        const char *s = std::getenv("B200GEMM_KSPLIT");
+        const int k = s ? std::atoi(s) : 0;
+        return (k == 2 || k == 4 || k == 8) ? k : 0;
+    }();
+    return v;
 }
 
 // K order of the dense kernels' tiles: serpentine (odd waves of tiles walk K
@@ -309,11 +329,16 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
         return static_cast<gemm_config_t>(forced);
     // A few rows and a long K: swap A and B and split K over every SM (the
     // skinny stream-K kernel).  Its fix-up of 128 x MP fp32 partials grows
-    // with M, so past 64 rows (or with a shorter K) whole tiles win.
-    if (M <= 64 && K >= 8192) return GEMM_CFG_SKINNY;
-    if (M <= 32 && K >= 4096) return GEMM_CFG_SKINNY;
+    // with M: past 32 rows the cluster split-K kernels win.
+    if (M <= 32 && K >= 8192) return GEMM_CFG_SKINNY;
+    // Tiles for at most half the SMs and a long K: split each tile's K over
+    // a cluster (2-8 CTAs), the partials summed on chip.
+    const int64_t tiles128 = ((M + 127) / 128) * ((N + 127) / 128);
+    const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
+    if (K >= 2048 && tiles128 <= 74) return GEMM_CFG_1CTA_128x128_SPLITK;
+    if (K >= 2048 && tiles256 <= 74) return GEMM_CFG_1CTA_128x256_SPLITK;
     // Every 128 x 128 tile on an SM of its own: the most SMs streaming.
-    if (((M + 127) / 128) * ((N + 127) / 128) <= 148) return GEMM_CFG_1CTA_128x128;
+    if (tiles128 <= 148) return GEMM_CFG_1CTA_128x128;
     struct Candidate {
         gemm_config_t cfg;
         CostModel cost;
@@ -351,13 +376,105 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
 
 gemm_status_t sk_workspace(DeviceState *st, size_t bytes, uint8_t *&ws, cudaStream_t stream);
 
-// `status`: the watchdog status block the kernel records a timeout in.
+// First launch of a configuration on a device: its shared-memory attribute
+// and how many of its clusters fit on the SMs at once (for split-K, with
+// clusters of 2, 4 and 8 CTAs).  Refused inside a stream capture.
 template <class Cfg>
-// `peers`: the further copies of C of a PEERS configuration (else unused).
+gemm_status_t setup_attrs(DeviceState *st, gemm_config_t cfg_id, cudaStream_t stream) {
+    auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
+    const int oi = Cfg::OUT;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (st->attr_done[cfg_id][oi]) return GEMM_OK;
+    if (capturing(stream)) return GEMM_ERR_CAPTURE;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES)) !=
+        cudaSuccess)
+        return cuda_fail(e);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Cfg::CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.blockDim = dim3(Cfg::THREADS, 1, 1);
+    lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    lc.stream = stream;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int clusters = st->sm_count / Cfg::CG;
+    if (Cfg::CG > 1 && !Cfg::CLC) {
+        lc.gridDim = dim3(Cfg::CG * clusters, 1, 1);
+        int n = 0;
+        if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
+        if (n > 0) clusters = n;
+    }
+    if constexpr (Cfg::SPLITK) {
+        for (int li = 0; li < 3; ++li) {
+            const int S = 2 << li;
+            attr[0].val.clusterDim.x = S;
+            lc.gridDim = dim3(S * (st->sm_count / S), 1, 1);
+            int n = 0;
+            if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
+            st->splitk_ctas[cfg_id][oi][li] = n * S;
+        }
+    }
+    st->max_clusters[cfg_id][oi] = clusters;
+    st->attr_done[cfg_id][oi] = true;
+    return GEMM_OK;
+}
+
+// Cluster size of a split-K launch: the largest S of 8, 4, 2 whose clusters
+// all fit on the SMs at once (one tile per cluster), that leaves every member
+// at least two 64-wide K blocks, and whose column slices (BN / S) are whole
+// store chunks.  1: no split pays (the caller runs the unsplit kernel).
+template <class Cfg>
+int choose_ksplit(const DeviceState *st, gemm_config_t cfg_id, int64_t M, int64_t N, int64_t K) {
+    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
+    const int64_t num_kb = (K + Cfg::BK - 1) / Cfg::BK;
+    for (int li = 2; li >= 0; --li) {
+        const int S = 2 << li;
+        if ((Cfg::BN / S) % Cfg::EPI_COLS != 0) continue;
+        if (num_kb < 2 * S) continue;
+        if (tiles * S > st->splitk_ctas[cfg_id][Cfg::OUT][li]) continue;
+        // the other members' partials of a slice fit in the operand ring
+        if (static_cast<int64_t>(S - 1) * 128 * (Cfg::BN / S) * 4 > static_cast<int64_t>(Cfg::STAGES) * Cfg::STAGE_BYTES)
+            continue;
+        return S;
+    }
+    return 1;
+}
+
+// `status`: the watchdog status block the kernel records a timeout in;
+// `peers`: the further copies of C of a PEERS configuration (else unused);
+// `ksplit`: the cluster size of a split-K configuration (else unused).
+template <class Cfg>
 gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t cfg_id, const void *A,
                           const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
                           int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi = b200::plain_epilogue(),
-                          uint32_t layout = 0, const b200::PeerC *peers = nullptr) {
+                          uint32_t layout = 0, const b200::PeerC *peers = nullptr, int ksplit = 1);
+
+// A split-K configuration: the cluster size by shape (or forced); where no
+// split pays, the same tile without one (`plain_id`, config CfgPlain).
+template <class CfgK, class CfgPlain>
+gemm_status_t launch_splitk(DeviceState *st, DeviceStatus *status, gemm_config_t cfg_id, gemm_config_t plain_id,
+                            const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda,
+                            int64_t ldb, int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi,
+                            uint32_t layout) {
+    gemm_status_t s;
+    if ((s = setup_attrs<CfgK>(st, cfg_id, stream)) != GEMM_OK) return s;
+    int S = forced_ksplit();
+    if (S == 0 || (CfgK::BN / S) % CfgK::EPI_COLS) S = choose_ksplit<CfgK>(st, cfg_id, M, N, K);
+    if (S < 2)
+        return launch_bf16<CfgPlain>(st, status, plain_id, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout,
+                                     nullptr, 1);
+    return launch_bf16<CfgK>(st, status, cfg_id, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout, nullptr, S);
+}
+
+template <class Cfg>
+gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t cfg_id, const void *A,
+                          const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                          int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout,
+                          const b200::PeerC *peers, int ksplit) {
     auto kernel = b200::gemm_bf16_sm100_kernel<Cfg>;
     const int oi = Cfg::OUT;
     typename Cfg::PeerArg peer_arg{};
@@ -370,10 +487,20 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     // MN-major tiles arrive as 64-wide boxes: whole boxes per CTA only
     if (((layout & b200::kLayoutBMajorN) && Cfg::B_ROWS % 64) || ((layout & b200::kLayoutAMajorM) && Cfg::BM_CTA % 64))
         return GEMM_ERR_INVALID_VALUE;
+    // split-K: 2, 4 or 8 CTAs per cluster, one cluster per tile; the column
+    // slices are whole store chunks, and the others' partials of a slice fit
+    // in the operand ring they are received in
+    if (Cfg::SPLITK && (ksplit < 2 || ksplit > 8 || (ksplit & (ksplit - 1)) || (Cfg::BN / ksplit) % Cfg::EPI_COLS ||
+                        static_cast<int64_t>(ksplit - 1) * 128 * (Cfg::BN / ksplit) * 4 >
+                            static_cast<int64_t>(Cfg::STAGES) * Cfg::STAGE_BYTES))
+        return GEMM_ERR_INVALID_VALUE;
     cudaError_t e;
+    gemm_status_t s;
+    if ((s = setup_attrs<Cfg>(st, cfg_id, stream)) != GEMM_OK) return s;
+    const int cluster_ctas = Cfg::SPLITK ? ksplit : Cfg::CG;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = Cfg::CG;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster_ctas);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cudaLaunchConfig_t lc = {};
@@ -382,28 +509,9 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     lc.stream = stream;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    {
-        std::lock_guard<std::mutex> lock(g_mutex);
-        if (!st->attr_done[cfg_id][oi]) {
-            if (capturing(stream)) return GEMM_ERR_CAPTURE;
-            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          Cfg::SMEM_BYTES)) != cudaSuccess)
-                return cuda_fail(e);
-            int clusters = st->sm_count / Cfg::CG;
-            if (Cfg::CG > 1 && !Cfg::CLC) {
-                lc.gridDim = dim3(Cfg::CG * clusters, 1, 1);
-                int n = 0;
-                if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
-                if (n > 0) clusters = n;
-            }
-            st->max_clusters[cfg_id][oi] = clusters;
-            st->attr_done[cfg_id][oi] = true;
-        }
-    }
     const CUtensorMapDataType cdt = Cfg::OUT == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int64_t ec = Cfg::OUT == 0 ? 4 : 2;
     alignas(64) CUtensorMap tmA, tmB, tmC;
-    gemm_status_t s;
     // K-major operands: boxes of 64 (K) x rows; MN-major (stored K x M / K x N):
     // boxes of 64 (MN) x 64 (K)
     if (layout & b200::kLayoutAMajorM)
@@ -426,10 +534,11 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     // Static schedule: as many clusters as fit at once, each striding over
     // the tiles.  CLC: one cluster per tile; running clusters claim the rest.
-    // Stream-K: every co-resident cluster, each with an equal share of the
-    // (tile, K block) iterations.
+    // Split-K: one cluster of `ksplit` CTAs per tile.  Stream-K: every
+    // co-resident cluster, each with an equal share of the (tile, K block)
+    // iterations.
     const int64_t resident = st->max_clusters[cfg_id][oi];
-    int64_t clusters = Cfg::CLC ? tiles : (tiles > resident ? resident : tiles);
+    int64_t clusters = (Cfg::CLC || Cfg::SPLITK) ? tiles : (tiles > resident ? resident : tiles);
     if constexpr (Cfg::SK) {
         // Every cluster's range must hold at least one iteration (the
         // fix-up counts a split tile's contributors as the consecutive range
@@ -439,10 +548,10 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
         const int64_t want = (iters + 3) / 4;
         clusters = want < resident ? want : resident;
     }
-    lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
+    lc.gridDim = dim3(static_cast<unsigned>(clusters * cluster_ctas), 1, 1);
     // tiles that run at the same time: one wave (for CLC, as many clusters
     // as fit on the SMs at once); stream-K keeps K ascending
-    const int wave_tiles = (serpentine_k() && !Cfg::SK) ? static_cast<int>(resident) : 0;
+    const int wave_tiles = (serpentine_k() && !Cfg::SK && !Cfg::SPLITK) ? static_cast<int>(resident) : 0;
     // Stream-K workspace: two [128][BN] fp32 partial slots per CTA (the
     // first and the last tile of its range may be split), then one 64-bit
     // arrival counter per (tile, CTA of the cluster).
@@ -633,6 +742,16 @@ gemm_status_t launch_dense(DeviceState *st, DeviceStatus *status, gemm_config_t 
         case GEMM_CFG_1CTA_128x256_CLC:
             return f32 ? launch_bf16<Cfg1x256F32C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                        : launch_bf16<Cfg1x256B16C>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_1CTA_128x128_SPLITK:
+            return f32 ? launch_splitk<Cfg1x128F32K, Cfg1x128F32>(st, status, cfg, GEMM_CFG_1CTA_128x128, A, B, C, M,
+                                                                   N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_splitk<Cfg1x128B16K, Cfg1x128B16>(st, status, cfg, GEMM_CFG_1CTA_128x128, A, B, C, M,
+                                                                   N, K, lda, ldb, ldc, stream, epi, layout);
+        case GEMM_CFG_1CTA_128x256_SPLITK:
+            return f32 ? launch_splitk<Cfg1x256F32K, Cfg1x256F32>(st, status, cfg, GEMM_CFG_1CTA_128x256, A, B, C, M,
+                                                                   N, K, lda, ldb, ldc, stream, epi, layout)
+                       : launch_splitk<Cfg1x256B16K, Cfg1x256B16>(st, status, cfg, GEMM_CFG_1CTA_128x256, A, B, C, M,
+                                                                   N, K, lda, ldb, ldc, stream, epi, layout);
         default:
             return GEMM_ERR_INVALID_VALUE;
     }
@@ -997,10 +1116,10 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
                                       : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
     }
     // The skinny and stream-K kernels need a workspace; without one, small-M
-    // shapes run on the one-CTA 128 x 128 kernel and stream-K shapes on the
-    // CLC pair kernel instead.
+    // shapes run on the cluster split-K kernel (its partials meet in shared
+    // memory) and stream-K shapes on the CLC pair kernel instead.
     gemm_config_t cfg = select_config(M, N, K);
-    if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128;
+    if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128_SPLITK;
     if (cfg == GEMM_CFG_2CTA_256x256_SK) cfg = GEMM_CFG_2CTA_256x256_CLC;   // stream-K needs a workspace too
     return launch_dense(st, st->noalloc_status, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc,
                         stream, b200::plain_epilogue(), 0u);

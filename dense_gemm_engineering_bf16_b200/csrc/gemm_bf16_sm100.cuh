@@ -34,6 +34,17 @@
 //               of idling) and hands the tile id to every role of both CTAs
 //               through a 2-deep shared-memory ring.
 //
+// Cluster split-K (SPLITK, one-CTA tiles): a cluster of S = 2, 4 or 8 CTAs
+// owns one tile, member r accumulating K blocks [r kb / S, (r+1) kb / S).
+// Once its MMAs are done, each member tells the others that its operand
+// ring is free.  It then sends column slice j of its fp32 partial into a
+// slot of member j's ring, through distributed shared memory, with a
+// cluster-scope release arrive on j's rx_full.  Member j adds the S partials
+// of its slice in member order and writes them to C through the usual store
+// path.  The split-K schedule of the pages' autotune search space ("GPU
+// 执行模型", section "编译与 autotune"), with the reduction on chip: no
+// workspace, no atomics, and a fixed summation order.
+//
 // Operands may be K-major (A as M x K, B as N x K) or MN-major (A as K x M,
 // B as K x N): MN-major tiles arrive as 64-wide boxes and the MMA reads them
 // through MN-major descriptors.  The epilogue computes
@@ -74,7 +85,7 @@ constexpr uint32_t kInjectDropFirstStage = 1u;
 
 enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleEpilogue = 3, kRoleScheduler = 4 };
 enum : int { kBarFull = 1, kBarEmpty = 2, kBarTmemFull = 3, kBarTmemEmpty = 4, kBarTail = 5, kBarSched = 6,
-             kBarClc = 7 };
+             kBarClc = 7, kBarPeerFree = 10, kBarRxFull = 11 };
 
 __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
     int p = lo;
@@ -96,7 +107,7 @@ struct PeerC {
 struct NoPeerC {};
 
 template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1, bool SK_ = false,
-          bool PEERS_ = false>
+          bool PEERS_ = false, bool SPLITK_ = false>
 struct GemmBf16Cfg {
     static constexpr bool CLC = CLC_;              // tiles from Cluster Launch Control, not a fixed stride
     // Stream-K: the (tile, K block) iterations are cut into one contiguous
@@ -105,6 +116,12 @@ struct GemmBf16Cfg {
     static constexpr bool SK = SK_;
     // PEERS: every chunk of C is also stored to the destinations of a PeerC
     static constexpr bool PEERS = PEERS_;
+    // SPLITK: cluster split-K.  The S CTAs of a cluster (S = 2, 4 or 8, the
+    // launch's cluster size) compute one tile together, each over its own
+    // contiguous share of the K blocks.  Member j then sums column slice j
+    // of the tile from every member's fp32 partial, in member order, the
+    // partials crossing between the CTAs' shared memories (DSMEM).
+    static constexpr bool SPLITK = SPLITK_;
     using PeerArg = std::conditional_t<PEERS_, PeerC, NoPeerC>;
     static constexpr int CG = CG_;                 // CTAs per tile (cta_group)
     static constexpr int BN = BN_;                 // tile N == MMA N
@@ -132,7 +149,8 @@ struct GemmBf16Cfg {
     static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
     static constexpr int TMEM_COLS = pow2_at_least(ACC_BUFS * CONSUMERS * BN, 32);
     // full[S], empty[S], tmem_full[2], tmem_empty[2] (+ clc[2], sched_full[2], sched_empty[2])
-    static constexpr int NUM_BARS = 2 * STAGES + 4 + (CLC ? 6 : 0);
+    // (+ split-K: peer_free, rx_full)
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + (CLC ? 6 : 0) + (SPLITK ? 2 : 0);
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES + EPI_BYTES;
     // after the barriers: TMEM address, abort flag, 2 tile ids, 2 CLC answers
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 64;
@@ -143,6 +161,8 @@ struct GemmBf16Cfg {
     static_assert(CONSUMERS == 1 || CONSUMERS == 2, "one or two MMA consumers");
     static_assert(!SK || (!CLC && CONSUMERS == 1 && BN % 4 == 0), "stream-K: static schedule, one consumer");
     static_assert(!PEERS || !SK, "a stream-K fix-up writes C with plain stores to one C only");
+    static_assert(!SPLITK || (CG == 1 && !CLC && CONSUMERS == 1 && !SK && !PEERS),
+                  "cluster split-K: one-CTA tiles, one tile per cluster, one C");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N: multiple of 16 in [16, 256]");
     static_assert(B_ROWS % 8 == 0 && B_ROWS <= 256, "TMA box rows <= 256, whole 8-row swizzle atoms");
     static_assert(BN % EPI_COLS == 0, "epilogue chunks cover the tile");
@@ -168,9 +188,9 @@ __device__ __forceinline__ void raster_tile(int tile, int num_m, int num_n, int 
 // A bounded wait failed.  If it failed because this CTA was already told to
 // abort, someone else has recorded the cause: just leave.  Otherwise record
 // the first expired wait of the grid (role, barrier, CTA), then tell this CTA
-// and its pair partner to abort.
+// and the other `cluster_ctas - 1` CTAs of its cluster to abort.
 __device__ __forceinline__ void record_timeout(DeviceStatus *status, volatile uint32_t *abort_flag,
-                                               uint32_t abort_smem, int cg, int where) {
+                                               uint32_t abort_smem, int cluster_ctas, int where) {
     if (*abort_flag) return;
     if (atomicCAS(&status->code, 0u, kStatusTimeout) == 0u) {
         status->where = where;
@@ -178,7 +198,11 @@ __device__ __forceinline__ void record_timeout(DeviceStatus *status, volatile ui
         __threadfence();
     }
     *abort_flag = 1u;
-    if (cg == 2) store_cluster_u32(map_to_cta(abort_smem, cluster_cta_rank() ^ 1u), 1u);
+    if (cluster_ctas > 1) {
+        const uint32_t me = cluster_cta_rank();
+        for (uint32_t r = 0; r < static_cast<uint32_t>(cluster_ctas); ++r)
+            if (r != me) store_cluster_u32(map_to_cta(abort_smem, r), 1u);
+    }
 }
 
 // Operand layouts in global memory (kernel `layout` word).
@@ -327,6 +351,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint32_t warp = threadIdx.x / 32;
     const uint32_t lane = threadIdx.x % 32;
     const uint32_t rank = (CG == 2) ? cluster_cta_rank() : 0u;
+    // cluster split-K: this CTA's member index and the number of members
+    const uint32_t kr = Cfg::SPLITK ? cluster_cta_rank() : 0u;
+    const uint32_t ksplit = Cfg::SPLITK ? cluster_num_ctas() : 1u;
+    const int cluster_ctas = Cfg::SPLITK ? static_cast<int>(ksplit) : CG;
 
     const uint32_t bar0 = base + Cfg::BAR_OFF;
     auto full_bar = [&](uint32_t s) { return bar0 + 8u * s; };
@@ -336,6 +364,9 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     auto clc_bar = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 4 + i); };
     auto sched_full = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 6 + i); };
     auto sched_empty = [&](uint32_t i) { return bar0 + 8u * (2 * Cfg::STAGES + 8 + i); };
+    // split-K: the other members' rings are free / their partials have arrived
+    const uint32_t peer_free_bar = bar0 + 8u * (2 * Cfg::STAGES + 4 + (Cfg::CLC ? 6 : 0));
+    const uint32_t rx_full_bar = peer_free_bar + 8u;
     const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
     const uint32_t abort_slot = tmem_slot + 4u;
     const uint32_t tile_ids = tmem_slot + 8u;              // int32 [2]
@@ -361,6 +392,12 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 mbar_init(sched_empty(i), Cfg::SCHED_CONSUMERS);
             }
         }
+        if constexpr (Cfg::SPLITK) {
+            if (ksplit > 1) {
+                mbar_init(peer_free_bar, ksplit - 1);            // one arrival per other member
+                mbar_init(rx_full_bar, (ksplit - 1) * 128u);     // every epilogue thread of every other member
+            }
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -375,7 +412,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     tc_fence_before_sync();
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync_all();
+    if constexpr (CG == 2 || Cfg::SPLITK) cluster_sync_all();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot_ptr;
 
@@ -383,8 +420,12 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + Cfg::BK - 1) / Cfg::BK;
-    const int cluster_id = static_cast<int>(blockIdx.x) / CG;
-    const int num_clusters = static_cast<int>(gridDim.x) / CG;
+    const int cluster_id = static_cast<int>(blockIdx.x) / cluster_ctas;
+    const int num_clusters = static_cast<int>(gridDim.x) / cluster_ctas;
+    // K blocks of every tile this CTA works on: all of them, or for split-K
+    // this member's contiguous share
+    const int kb_lo = Cfg::SPLITK ? static_cast<int>((static_cast<int64_t>(kr) * num_kb) / ksplit) : 0;
+    const int kb_hi = Cfg::SPLITK ? static_cast<int>((static_cast<int64_t>(kr + 1) * num_kb) / ksplit) : num_kb;
 
     // The tile sequence every role of this CTA (and of its pair) walks.
     // Static: cluster_id, + num_clusters, ...  CLC: the first tile is the
@@ -454,7 +495,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             u = sk_range_unit(sk_order(0));
             return true;
         } else {
-            u = Unit{cluster_id, 0, num_kb};
+            u = Unit{cluster_id, kb_lo, kb_hi};
             return cluster_id < num_tiles;
         }
     };
@@ -467,7 +508,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             return true;
         } else {
             const int n = next_tile(u.tile, j, ok);
-            u = Unit{n, 0, num_kb};
+            u = Unit{n, kb_lo, kb_hi};
             return n >= 0;
         }
     };
@@ -491,10 +532,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 // backwards, so a new wave starts on the K slices of A and B
                 // that the wave before it read last, which are still in L2.
                 // The order is fixed per tile, so results stay deterministic.
-                const bool rev = !Cfg::SK && wave_tiles > 0 && ((tile / wave_tiles) & 1) != 0;
+                const bool rev = !Cfg::SK && !Cfg::SPLITK && wave_tiles > 0 && ((tile / wave_tiles) & 1) != 0;
                 for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarEmpty);
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleProducer * 16 + kBarEmpty);
                         ok = false;
                         break;
                     }
@@ -524,13 +565,13 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 if (!ok) break;
                 more = next_unit(u, fetched++, ok);
-                if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarSched);
+                if (!ok) record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleProducer * 16 + kBarSched);
             }
             // Tail: every stage handed out must be released by the MMA before
             // this CTA may exit (its empty barriers still receive arrivals).
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, CG, kRoleProducer * 16 + kBarTail);
+                    record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleProducer * 16 + kBarTail);
                     ok = false;
                 }
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -558,7 +599,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
                 const uint32_t acc_phase = (static_cast<uint32_t>(t) / Cfg::ACC_BUFS) & 1u;
                 if (!mbar_wait(tempty_bar(buf), acc_phase ^ 1u, abort_flag, 3 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarTmemEmpty);
+                    record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleMma * 16 + kBarTmemEmpty);
                     ok = false;
                     break;
                 }
@@ -566,7 +607,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t d_tmem = tmem_base + buf * Cfg::CONSUMERS * Cfg::BN;
                 for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarFull);
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleMma * 16 + kBarFull);
                         ok = false;
                         break;
                     }
@@ -587,7 +628,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (!ok) break;
                 mma_commit<CG>(tfull_bar(buf), 0x3);
                 more = next_unit(u, static_cast<uint32_t>(t), ok);
-                if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleMma * 16 + kBarSched);
+                if (!ok) record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleMma * 16 + kBarSched);
             }
         }
         __syncwarp();
@@ -598,13 +639,13 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 for (uint32_t j = 0;; ++j) {
                     const uint32_t slot = j & 1u, ph = (j >> 1) & 1u;
                     if (!mbar_wait(sched_empty(slot), ph ^ 1u, abort_flag, 3 * timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, CG, kRoleScheduler * 16 + kBarSched);
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleScheduler * 16 + kBarSched);
                         break;
                     }
                     mbar_arrive_expect_tx(clc_bar(slot), 16);
                     clc_try_cancel(clc_resp + 16u * slot, clc_bar(slot));
                     if (!mbar_wait(clc_bar(slot), ph, abort_flag, 3 * timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, CG, kRoleScheduler * 16 + kBarClc);
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleScheduler * 16 + kBarClc);
                         break;
                     }
                     uint32_t first_x = 0;
@@ -642,7 +683,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             // converged for the .sync.aligned TMEM loads below.
             uint32_t ready = 1;
             if (lane == 0 && !mbar_wait(tfull_bar(buf), acc_phase, abort_flag, 3 * timeout_ns)) {
-                record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarTmemFull);
+                record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarTmemFull);
                 ready = 0;
             }
             ready = __shfl_sync(0xffffffffu, ready, 0);
@@ -728,7 +769,129 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             };
             bool split = false;   // stream-K: this unit is one piece of a split tile
             if constexpr (Cfg::SK) split = !(u.kb0 == 0 && u.kb1 == num_kb);
-            if (split) {
+            if constexpr (Cfg::SPLITK) {
+                // ---- cluster split-K: this member's accumulator holds the
+                // fp32 partial over K blocks [u.kb0, u.kb1) (none: zeros).
+                // Member j sums column slice j (SW columns) of the tile from
+                // every member's partial, in member order, and writes it to
+                // C.  Slice j of the others' partials crosses into member j's
+                // operand ring, which its MMAs no longer read.
+                const uint32_t S = ksplit;
+                const int SW = Cfg::BN / static_cast<int>(S);      // a multiple of EPI_COLS (host)
+                const bool has_k = u.kb1 > u.kb0;
+                const uint32_t arow = sub * 32u + lane;            // accumulator row (TMEM lane)
+                const uint32_t slot_bytes = 128u * static_cast<uint32_t>(SW) * 4u;
+                const uint32_t epi_tid = threadIdx.x - 64u;
+                auto load32 = [&](uint32_t col, uint32_t (&v)[32]) {
+                    if (has_k) {
+                        tmem_ld_32x32b_x32(tbase0 + col, v);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0u;
+                    }
+                };
+                bool xok = true;
+                if (S > 1) {
+                    // this CTA's MMAs are done: its ring may take the others' partials
+                    if (epi_tid == 0)
+                        for (uint32_t j = 0; j < S; ++j)
+                            if (j != kr) mbar_arrive_cluster(map_to_cta(peer_free_bar, j));
+                    uint32_t fr = 1;
+                    if (lane == 0 && !mbar_wait(peer_free_bar, 0, abort_flag, 3 * timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarPeerFree);
+                        fr = 0;
+                    }
+                    xok = __shfl_sync(0xffffffffu, fr, 0) != 0;
+                    if (xok) {
+                        // slice j of this partial, row `arow`, to this member's slot
+                        // at member j; 16-byte pieces swizzled by the row, so a
+                        // warp's stores (and the reads back) are conflict-free
+                        for (uint32_t j = 0; j < S; ++j) {
+                            if (j == kr) continue;
+                            const uint32_t slot = kr < j ? kr : kr - 1u;
+                            const uint32_t dst_row =
+                                map_to_cta(base + slot * slot_bytes + arow * static_cast<uint32_t>(SW) * 4u, j);
+#pragma unroll 1
+                            for (int c = 0; c < SW / 32; ++c) {
+                                uint32_t v[32];
+                                load32(j * static_cast<uint32_t>(SW) + static_cast<uint32_t>(c * 32), v);
+#pragma unroll
+                                for (int p = 0; p < 8; ++p) {
+                                    const uint32_t piece = static_cast<uint32_t>(c * 8 + p) ^ (lane & 7u);
+                                    store_cluster_v4(dst_row + (piece << 4), v[4 * p], v[4 * p + 1], v[4 * p + 2],
+                                                     v[4 * p + 3]);
+                                }
+                            }
+                            mbar_arrive_cluster(map_to_cta(rx_full_bar, j));   // release: the stores come first
+                        }
+                        uint32_t rf = 1;
+                        if (lane == 0 && !mbar_wait(rx_full_bar, 0, abort_flag, 3 * timeout_ns)) {
+                            record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarRxFull);
+                            rf = 0;
+                        }
+                        xok = __shfl_sync(0xffffffffu, rf, 0) != 0;
+                    }
+                }
+                // 32 columns of slice kr (from slice column c * 32): the
+                // members' partials added in member order
+                auto slice_sum = [&](int c, uint32_t (&v)[32]) {
+                    uint32_t own[32];
+                    load32(kr * static_cast<uint32_t>(SW) + static_cast<uint32_t>(c * 32), own);
+#pragma unroll 1
+                    for (uint32_t m = 0; m < S; ++m) {
+                        uint32_t x[32];
+                        if (m == kr) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) x[i] = own[i];
+                        } else {
+                            const uint32_t slot = m < kr ? m : m - 1u;
+                            const uint32_t src_row = base + slot * slot_bytes + arow * static_cast<uint32_t>(SW) * 4u;
+#pragma unroll
+                            for (int p = 0; p < 8; ++p) {
+                                const uint32_t piece = static_cast<uint32_t>(c * 8 + p) ^ (lane & 7u);
+                                ld_shared_v4(src_row + (piece << 4), x[4 * p], x[4 * p + 1], x[4 * p + 2], x[4 * p + 3]);
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            v[i] = m == 0 ? x[i] : __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(x[i]));
+                    }
+                };
+                if (xok) {
+                    const int erow = row_base + static_cast<int>(lane);
+                    if constexpr (Cfg::OUT == 0) {
+#pragma unroll 1
+                        for (int c = 0; c < SW / 32; ++c) {
+                            uint32_t v[32];
+                            slice_sum(c, v);
+                            const int q = static_cast<int>(kr) * SW / 32 + c;
+                            if (fused) epilogue32_f32c(v, C, ldc, erow, col0 + q * 32, M, N, epi);
+                            store_chunk(v, q);
+                        }
+                    } else {
+#pragma unroll 1
+                        for (int c = 0; c < SW / 32; c += 2) {
+                            uint32_t v0[32], v1[32], packed[32];
+                            slice_sum(c, v0);
+                            slice_sum(c + 1, v1);
+                            const int q = static_cast<int>(kr) * SW / 64 + c / 2;
+                            if (fused) {
+                                epilogue32_bf16c(v0, C, ldc, erow, col0 + q * 64, M, N, epi);
+                                epilogue32_bf16c(v1, C, ldc, erow, col0 + q * 64 + 32, M, N, epi);
+                            }
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                packed[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+                                packed[16 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+                            }
+                            store_chunk(packed, q);
+                        }
+                    }
+                }
+                release_tmem();
+                if (!xok) break;
+            } else if (split) {
               if constexpr (Cfg::SK) {
                 // ---- stream-K: this unit is part of a tile split between
                 // clusters.  Write this CTA's fp32 partial (row 32 sub + lane,
@@ -845,10 +1008,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (lane == 0) {
                     bool ok = true;
                     nt = next_tile(tile, static_cast<uint32_t>(t), ok);
-                    if (!ok) record_timeout(status, abort_flag, abort_slot, CG, kRoleEpilogue * 16 + kBarSched);
+                    if (!ok) record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarSched);
                 }
                 nt = __shfl_sync(0xffffffffu, nt, 0);
-                u = Unit{nt, 0, num_kb};
+                u = Unit{nt, kb_lo, kb_hi};
                 more = nt >= 0;
             }
         }
@@ -859,7 +1022,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     // -------------------------------------------------------- teardown --
     tc_fence_before_sync();
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync_all();
+    if constexpr (CG == 2 || Cfg::SPLITK) cluster_sync_all();
     if (*abort_flag) {
         // A wait expired somewhere: give in-flight TMA copies and MMAs time
         // to land before the TMEM and shared memory are released.
@@ -867,7 +1030,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
     }
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync_all();
+    if constexpr (CG == 2 || Cfg::SPLITK) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);

@@ -42,6 +42,8 @@ CONFIGS = {
     "2cta_512x256_clc": 9,
     "2cta_256x256_sk": 10,
     "2cta_256x224": 11,
+    "1cta_128x128_splitk": 12,
+    "1cta_128x256_splitk": 13,
 }
 
 STATUS_NAMES = {

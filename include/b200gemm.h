@@ -133,7 +133,15 @@ typedef enum {
     GEMM_CFG_2CTA_256x224 = 11,     /* CTA pair per 256 x 224 tile (fills the waves of some shapes
                                        better); fp32 C with B stored K-major only (bf16 C or a B
                                        stored K x N runs 2CTA_256x256); never chosen by shape */
-    GEMM_CFG_COUNT_ = 12
+    GEMM_CFG_1CTA_128x128_SPLITK = 12, /* cluster split-K: a cluster of S = 2, 4 or 8 CTAs per 128 x 128
+                                       tile, each over a contiguous share of K; member j sums
+                                       column slice j from every member's fp32 partial in member
+                                       order (deterministic), the partials crossing through
+                                       distributed shared memory (no workspace).  S: the largest
+                                       whose clusters all fit at once and give every member two
+                                       64-wide K blocks (else the unsplit 1CTA_128x128) */
+    GEMM_CFG_1CTA_128x256_SPLITK = 13, /* the same with 128 x 256 tiles (else 1CTA_128x256) */
+    GEMM_CFG_COUNT_ = 14
 } gemm_config_t;
 
 /*
@@ -278,8 +286,9 @@ B200GEMM_API gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const v
  * device array inside the library, which every GPU that loads the library
  * holds until the process exits.  One difference in kernel choice: the
  * skinny split-K kernel (GEMM_CFG_SKINNY), whose workspace gemm_bf16
- * allocates, is replaced by GEMM_CFG_1CTA_128x128, so small-M, long-K shapes
- * run slower here.  A call that would need more scratch than that array is
+ * allocates, is replaced by GEMM_CFG_1CTA_128x128_SPLITK (which needs no
+ * workspace: its partials meet in shared memory), so the few shapes that
+ * take the skinny kernel (M <= 32, K >= 8192) run somewhat slower here.  A call that would need more scratch than that array is
  * rejected with GEMM_ERR_TOO_LARGE (no shape does today: the scratch does
  * not grow with M, N or K).  Each call queues exactly one kernel.
  *
@@ -326,15 +335,17 @@ B200GEMM_API int gemm_last_cuda_error(void);
  * (GEMM_CFG_AUTO restores shape-based selection).  A bf16 configuration
  * applies to gemm_bf16, gemm_bf16_ex and gemm_bf16_fused (except that an A
  * stored K x M never runs on GEMM_CFG_SKINNY) and to gemm_bf16_noalloc
- * (which runs GEMM_CFG_SKINNY as GEMM_CFG_1CTA_128x128); an MXFP8 one
+ * (which runs GEMM_CFG_SKINNY as GEMM_CFG_1CTA_128x128_SPLITK); an MXFP8 one
  * applies to gemm_mxfp8, and leaves the bf16 entry points choosing by shape.
  * A forced GEMM_CFG_SKINNY with M > 256 fails with GEMM_ERR_INVALID_VALUE.
  * Returns GEMM_ERR_INVALID_VALUE for an unknown configuration. */
 B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
 
 /* The configuration the next gemm_bf16 call with this shape would use.
- * M <= 64 with K >= 8192, or M <= 32 with K >= 4096: GEMM_CFG_SKINNY.
- * Every 128 x 128 tile on an SM of its own: GEMM_CFG_1CTA_128x128.
+ * M <= 32 with K >= 8192: GEMM_CFG_SKINNY.  K >= 2048 with at most 74
+ * tiles of 128 x 128 (else of 128 x 256): GEMM_CFG_1CTA_128x128_SPLITK
+ * (GEMM_CFG_1CTA_128x256_SPLITK).  Every 128 x 128 tile on an SM of its
+ * own: GEMM_CFG_1CTA_128x128.
  * Otherwise the configuration with the lowest predicted time among the
  * 1-CTA 128 x 256 (up to two waves), the 256 x 256 pair (static, or with
  * Cluster Launch Control when K > 2048) and, for K >= 8192, the 512 x 256

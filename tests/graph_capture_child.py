@@ -66,7 +66,7 @@ def growth_after_capture():
     res = {}
     s = torch.cuda.Stream()
     # skinny: small problem captured, then a large one grows the workspace
-    m, n, k = 16, 256, 4096
+    m, n, k = 16, 256, 8192
     a_bits, b_bits = synth.bf16_operands(m, n, k, "normal", workload=410)
     A, B = dev_bf16(a_bits), dev_bf16(b_bits)
     C = torch.zeros((m, n), dtype=torch.float32, device="cuda")

@@ -58,7 +58,7 @@ def test_one_graph_of_several_configs_replays_like_eager_calls():
     a1, b1 = synth.bf16_operands(M1, N1, K1, "uniform", workload=420)
     A1, B1 = to_device_bf16(a1), to_device_bf16(b1)
     C1 = torch.empty((M1, N1), dtype=torch.float32, device="cuda")
-    M2, N2, K2 = 32, 2048, 4096
+    M2, N2, K2 = 32, 2048, 8192
     a2, b2 = synth.bf16_operands(M2, N2, K2, "normal", workload=421)
     A2, B2 = to_device_bf16(a2), to_device_bf16(b2)
     C2 = torch.empty((M2, N2), dtype=torch.float32, device="cuda")
@@ -148,3 +148,38 @@ def test_stream_k_replays_match_eager_and_oracle():
     finally:
         G.gemm_force_config("auto")
     G.gemm_check_device_status()
+
+
+def test_cluster_split_k_replays_match_eager_and_oracle():
+    """The cluster split-K kernel in a graph: its cluster barriers start each
+    launch afresh, so replays with new inputs give the eager bits."""
+    s = torch.cuda.Stream()
+    M, N, K = 256, 2048, 4096                  # 32 tiles of 128 x 128: clusters of four over K
+    assert G.gemm_select_config(M, N, K) == G.CONFIGS["1cta_128x128_splitk"]
+    a, b = synth.bf16_operands(M, N, K, "normal", workload=440)
+    A, B = to_device_bf16(a), to_device_bf16(b)
+    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    call = lambda: G.gemm_bf16(A, B, C, M, N, K, K, K, N, stream=s)  # noqa: E731
+    with torch.cuda.stream(s):
+        call()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call()
+    for rep in range(3):
+        a2, b2 = synth.bf16_operands(M, N, K, "normal", workload=441 + rep)
+        A.copy_(to_device_bf16(a2))
+        B.copy_(to_device_bf16(b2))
+        C.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        got = C.clone()
+        with torch.cuda.stream(s):
+            call()
+        s.synchronize()
+        assert torch.equal(got, C)
+    rows = np.arange(0, M, 5)
+    c_ref, s_abs = oracle.gemm_bf16_f64(a2, b2, rows=rows, with_abs=True)
+    assert np.all(np.abs(C.cpu().numpy()[rows].astype(np.float64) - c_ref) <= 1e-3 * s_abs + 1e-6)
+    del g
+    assert G.gemm_check_device_status() == 0

@@ -22,7 +22,7 @@ from gpu_helpers import (assert_close, assert_exact, run_gemm, sample_indices)
 pytestmark = pytest.mark.gpu
 
 CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "1cta_128x256_clc", "2cta_256x256_clc", "2cta_512x256_clc",
-        "2cta_256x256_sk", "2cta_256x224"]
+        "2cta_256x256_sk", "2cta_256x224", "1cta_128x128_splitk", "1cta_128x256_splitk"]
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 
 

@@ -14,7 +14,7 @@ from gpu_helpers import assert_exact, to_device_bf16
 pytestmark = pytest.mark.gpu
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc", "skinny",
-        "2cta_256x256_sk", "2cta_256x224"]
+        "2cta_256x256_sk", "2cta_256x224", "1cta_128x128_splitk", "1cta_128x256_splitk"]
 ACTS = {"none": G.ACT_NONE, "relu": G.ACT_RELU, "gelu": G.ACT_GELU, "gelu_tanh": G.ACT_GELU_TANH}
 
 

@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 F32, BF16 = G.OUT_F32, G.OUT_BF16
 K_, MN = G.KMAJOR, G.MNMAJOR
 CFGS = ["1cta_128x128", "1cta_128x256", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc", "skinny",
-        "2cta_256x256_sk", "2cta_256x224"]
+        "2cta_256x256_sk", "2cta_256x224", "1cta_128x128_splitk", "1cta_128x256_splitk"]
 
 
 def _store(canon_bits: np.ndarray, mn: bool) -> np.ndarray:

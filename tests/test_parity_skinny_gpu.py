@@ -30,11 +30,11 @@ def _check(M, N, K, dist, workload, c_type=F32, lda=None, config="skinny", repea
 
 def test_auto_selects_skinny_for_small_m():
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
-    assert G.gemm_select_config(64, 8192, 8192) == G.CONFIGS["skinny"]
-    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
-    # past 64 rows the fp32 partials of the split tiles cost more than the
-    # split saves: whole 128 x 128 tiles, one per SM
-    assert G.gemm_select_config(256, 4096, 4096) == G.CONFIGS["1cta_128x128"]
+    assert G.gemm_select_config(32, 2048, 8192) == G.CONFIGS["skinny"]
+    # past 32 rows (or over a shorter K) the skinny kernel's fp32 partials
+    # cost more than the cluster split-K kernel's on-chip sum
+    assert G.gemm_select_config(64, 8192, 8192) == G.CONFIGS["1cta_128x128_splitk"]
+    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["1cta_128x128_splitk"]
 
 
 @pytest.mark.parametrize("c_type", [F32, BF16])

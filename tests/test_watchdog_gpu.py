@@ -22,7 +22,7 @@ import pytest
 pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-CFGS = ("1cta_128x128", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc")
+CFGS = ("1cta_128x128", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc", "1cta_128x256_splitk")
 
 CHILD = textwrap.dedent(r"""
     import os, sys, time
@@ -60,7 +60,7 @@ CHILD = textwrap.dedent(r"""
 
 
 def test_dropped_arrival_times_out_cleanly_and_context_survives():
-    launches = len(CFGS) + 1                  # four configurations, then gemm_bf16_noalloc
+    launches = len(CFGS) + 1                  # each configuration, then gemm_bf16_noalloc
     env = dict(os.environ, B200GEMM_WATCHDOG_MS="100", B200GEMM_INJECT_TIMEOUT="10" * launches)
     out = subprocess.run([sys.executable, "-c", CHILD, ROOT, ",".join(CFGS)], env=env, capture_output=True,
                          text=True, timeout=300)

@@ -93,6 +93,29 @@ def test_noalloc_runs_the_cluster_launch_control_kernel():
     assert np.all(np.abs(got - c64) <= tolerance(c64, s_abs, G.OUT_BF16))
 
 
+def test_noalloc_small_m_runs_the_split_k_kernel():
+    """Where gemm_bf16 takes the skinny kernel (whose partials live in an
+    allocated workspace), the allocation-free entry point runs the cluster
+    split-K kernel, whose partials meet in shared memory: same result within
+    the tolerance, no device memory taken."""
+    M, N, K = 16, 1024, 8192
+    assert G.gemm_select_config(M, N, K) == G.CONFIGS["skinny"]
+    a_bits, b_bits = synth.bf16_operands(M, N, K, "normal", workload=74)
+    A, B = to_device_bf16(a_bits), to_device_bf16(b_bits)
+    C = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    G.gemm_bf16_noalloc(A, B, C, M, N, K, K, K, N, G.OUT_F32)     # first use of this kernel: loads it
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    C.fill_(float("nan"))
+    G.gemm_bf16_noalloc(A, B, C, M, N, K, K, K, N, G.OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free_before
+    G.gemm_check_device_status()
+    c64, s_abs = oracle.gemm_bf16_f64(a_bits, b_bits, with_abs=True)
+    got = C.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - c64) <= tolerance(c64, s_abs, G.OUT_F32))
+
+
 def test_noalloc_argument_checks_match():
     ptr = 0x7F0000000000
     for args in [(-1, 8, 8, 8, 8, 8, 0), (8, 8, 8, 4, 8, 8, 0), (8, 8, 8, 8, 8, 8, 9)]:
