@@ -452,6 +452,10 @@ def config_report(G, torch, stream, peaks: dict, steps: int, warmup: int) -> dic
                  "l2": ("flushed before every call (252 MiB written, then read back)" if flush else
                         "no flush (inputs+output > 2 x L2)"),
                  "median_us": med * 1e6, "p90_us": float(np.percentile(per_step, 90)) * 1e3,
+                 # CUDA events on this GPU tick in 2.048 us steps, so a
+                 # per-call median is a whole number of ticks; the mean of
+                 # the calls resolves finer
+                 "mean_us": statistics.fmean(per_step) * 1e3,
                  "tflops": p.flops / med / 1e12, "gbs": min_bytes(p) / med / 1e9,
                  "bound": measured["bound"], "roofline_us": measured["roofline_us"], "frac": measured["frac"],
                  "frac_of_nominal": nominal["frac"], "min_bytes": min_bytes(p)}
