@@ -58,6 +58,9 @@ using CfgMxf8 = b200::GemmMxf8Cfg<1, 4>;
 using CfgMxf8Pair = b200::GemmMxf8Cfg<2, 6>;
 using CfgSk64F32 = b200::GemmSkinnyCfg<64, 8, 0>;
 using CfgSk64B16 = b200::GemmSkinnyCfg<64, 8, 1>;
+// the skinny tile with its K split over a cluster (partials in DSMEM)
+using CfgSk64F32C = b200::GemmSkinnyCfg<64, 8, 0, 1, true>;
+using CfgSk64B16C = b200::GemmSkinnyCfg<64, 8, 1, 1, true>;
 using CfgSk128F32 = b200::GemmSkinnyCfg<128, 6, 0>;
 using CfgSk128B16 = b200::GemmSkinnyCfg<128, 6, 1>;
 using CfgSk256F32 = b200::GemmSkinnyCfg<256, 4, 0>;
@@ -86,8 +89,12 @@ struct DeviceState {
     int mx_max_clusters[2] = {};
     uint8_t *mx_ws = nullptr;
     size_t mx_ws_bytes = 0;
-    // skinny path: kernel attributes (per template), split-tile workspace
+    // skinny path: kernel attributes (per template), split-tile workspace;
+    // the cluster-split templates (fp32, bf16 C): co-resident CTAs with
+    // clusters of 2 and 4
     bool sk_attr_done[6] = {};
+    bool skc_attr_done[2] = {};
+    int skc_ctas[2][2] = {};
     uint8_t *sk_ws = nullptr;
     size_t sk_ws_bytes = 0;
     uint32_t sk_epoch = 0;
@@ -327,10 +334,10 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     const int forced = g_forced.load(std::memory_order_relaxed);
     if (forced != GEMM_CFG_AUTO && forced != GEMM_CFG_MXFP8_1CTA_128x256 && forced != GEMM_CFG_MXFP8_2CTA_256x256)
         return static_cast<gemm_config_t>(forced);
-    // A few rows and a long K: swap A and B and split K over every SM (the
-    // skinny stream-K kernel).  Its fix-up of 128 x MP fp32 partials grows
-    // with M: past 32 rows the cluster split-K kernels win.
-    if (M <= 32 && K >= 8192) return GEMM_CFG_SKINNY;
+    // A few rows and a long K: swap A and B, so 128 rows of B fill the MMA,
+    // and split K (over a cluster per tile of B, else stream-K over every
+    // SM).  Past 32 rows the split-K tile kernels win.
+    if (M <= 32 && K >= 4096) return GEMM_CFG_SKINNY;
     // Tiles for at most half the SMs and a long K: split each tile's K over
     // a cluster (2-8 CTAs), the partials summed on chip.
     const int64_t tiles128 = ((M + 127) / 128) * ((N + 127) / 128);
@@ -666,14 +673,98 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
     return GEMM_OK;
 }
 
+// The skinny tile with K split over a cluster of S CTAs per 128-row tile of
+// B (no workspace: the partials meet in shared memory).  S: 4 or 2, the
+// largest whose clusters all fit at once, leave every member two 64-wide K
+// blocks and keep at least 96 SMs streaming; 1 = none qualifies (the caller
+// runs the stream-K kernel).
+template <class Cfg>
+gemm_status_t launch_skinny_cluster(DeviceState *st, int slot, const void *A, const void *B, void *C, int64_t M,
+                                    int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
+                                    const b200::Epilogue &epi, uint32_t layout, bool &launched) {
+    launched = false;
+    auto kernel = b200::gemm_bf16_skinny_sm100_kernel<Cfg>;
+    cudaError_t e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.blockDim = dim3(Cfg::THREADS, 1, 1);
+    lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    lc.stream = stream;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!st->skc_attr_done[slot]) {
+            if (capturing(stream)) return GEMM_ERR_CAPTURE;
+            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES)) !=
+                cudaSuccess)
+                return cuda_fail(e);
+            for (int li = 0; li < 2; ++li) {
+                const int S = 2 << li;
+                attr[0].val.clusterDim.x = S;
+                lc.gridDim = dim3(S * (st->sm_count / S), 1, 1);
+                int n = 0;
+                if ((e = cudaOccupancyMaxActiveClusters(&n, kernel, &lc)) != cudaSuccess) return cuda_fail(e);
+                st->skc_ctas[slot][li] = n * S;
+            }
+            st->skc_attr_done[slot] = true;
+        }
+    }
+    const int64_t tiles = (N + Cfg::TILE_N - 1) / Cfg::TILE_N;
+    const int64_t kb = (K + Cfg::BK - 1) / Cfg::BK;
+    int S = 1;
+    for (int li = 1; li >= 0; --li) {
+        const int cand = 2 << li;
+        if (tiles * cand <= st->skc_ctas[slot][li] && kb >= 2 * cand && tiles * cand >= 96) {
+            S = cand;
+            break;
+        }
+    }
+    if (S < 2) return GEMM_OK;                    // not launched: the caller runs stream-K
+    const int64_t mpad = (M + 15) / 16 * 16;
+    alignas(64) CUtensorMap tmB, tmA;
+    gemm_status_t s;
+    if (layout & b200::kLayoutBMajorN)
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, K, ldb * 2, 64, Cfg::BK);
+    else
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N);
+    if (s != GEMM_OK) return s;
+    if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK,
+                       static_cast<uint32_t>(mpad))) != GEMM_OK)
+        return s;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    lc.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
+    float *no_partials = nullptr;
+    unsigned long long *no_counters = nullptr;
+    e = cudaLaunchKernelEx(&lc, kernel, tmB, tmA, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                           static_cast<int>(mpad), C, ldc, no_partials, no_counters, 0, 0u, st->status, watchdog_ns(K),
+                           epi, layout);
+    if (e != cudaSuccess) return cuda_fail(e);
+    launched = true;
+    return GEMM_OK;
+}
+
 gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const void *B, void *C, int64_t M,
                                 int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
                                 const b200::Epilogue &epi = b200::plain_epilogue(), uint32_t layout = 0) {
     // the skinny kernel reads A K-major only (A stored M x K)
     if (M > 256 || (layout & b200::kLayoutAMajorM)) return GEMM_ERR_INVALID_VALUE;
-    if (M <= 64)
+    if (M <= 64) {
+        // enough 128-row tiles of B to keep most SMs streaming with K split
+        // over a cluster: the partials stay on chip; otherwise stream-K
+        bool launched = false;
+        gemm_status_t s = f32 ? launch_skinny_cluster<CfgSk64F32C>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream,
+                                                                   epi, layout, launched)
+                              : launch_skinny_cluster<CfgSk64B16C>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream,
+                                                                   epi, layout, launched);
+        if (s != GEMM_OK || launched) return s;
         return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                    : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+    }
     if (M <= 128)
         return f32 ? launch_skinny<CfgSk128F32>(st, 2, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                    : launch_skinny<CfgSk128B16>(st, 3, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);

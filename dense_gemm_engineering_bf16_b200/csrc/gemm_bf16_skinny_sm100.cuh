@@ -37,8 +37,13 @@
 
 namespace b200 {
 
-template <int MP_, int STAGES_, int OUT_, int KBS_ = 1>
+template <int MP_, int STAGES_, int OUT_, int KBS_ = 1, bool CSPLIT_ = false>
 struct GemmSkinnyCfg {
+    // CSPLIT: instead of stream-K over all SMs, a cluster of S = 2 or 4 CTAs
+    // per 128-row tile of B, each over its own share of K; the partials meet
+    // in shared memory (DSMEM), and the CTA that owns a quarter or half of
+    // the tile's columns sums them in member order and writes C.
+    static constexpr bool CSPLIT = CSPLIT_;
     static constexpr int MP = MP_;                 // max padded rows of A (MMA N)
     static constexpr int STAGES = STAGES_;
     static constexpr int OUT = OUT_;               // 0: f32 C, 1: bf16 C
@@ -53,7 +58,7 @@ struct GemmSkinnyCfg {
     static constexpr int A_BYTES = KBS * A_BOX;
     static constexpr int STAGE_BYTES = B_BYTES + A_BYTES;
     static constexpr int TMEM_COLS = pow2_at_least(2 * MP, 32);
-    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + (CSPLIT ? 2 : 0);   // (+ peer_free, rx_full)
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 16;
     static constexpr int THREADS = 192;
@@ -61,6 +66,10 @@ struct GemmSkinnyCfg {
     static_assert(STAGE_BYTES % 1024 == 0 && A_BOX % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
+    static_assert(!CSPLIT || KBS == 1, "cluster split: one 64-wide K block per stage");
+    // the other members' partials of a member's columns (at most 3 x 32 rows
+    // of mpad fp32, S = 4) fit in the operand ring
+    static_assert(!CSPLIT || 96 * MP * 4 <= STAGES * STAGE_BYTES, "cluster split: receive slots in the ring");
 };
 
 // First iteration of CTA c's range when `total` iterations are cut into `g`.
@@ -205,12 +214,18 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
     const uint32_t base = smem_addr(smem);
     const uint32_t warp = threadIdx.x / 32;
     const uint32_t lane = threadIdx.x % 32;
+    // cluster split: this CTA's member index and the number of members
+    const uint32_t kr = Cfg::CSPLIT ? cluster_cta_rank() : 0u;
+    const uint32_t ksplit = Cfg::CSPLIT ? cluster_num_ctas() : 1u;
+    const int cluster_ctas = static_cast<int>(ksplit);
 
     const uint32_t bar0 = base + Cfg::BAR_OFF;
     auto full_bar = [&](uint32_t s) { return bar0 + 8u * s; };
     auto empty_bar = [&](uint32_t s) { return bar0 + 8u * (Cfg::STAGES + s); };
     auto tfull_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + b); };
     auto tempty_bar = [&](uint32_t b) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + b); };
+    const uint32_t peer_free_bar = bar0 + 8u * (2 * Cfg::STAGES + 4);   // the others' rings are free
+    const uint32_t rx_full_bar = peer_free_bar + 8u;                     // the others' partials are in
     const uint32_t tmem_slot = bar0 + 8u * Cfg::NUM_BARS;
     const uint32_t abort_slot = tmem_slot + 4u;
     volatile uint32_t *tmem_slot_ptr = reinterpret_cast<volatile uint32_t *>(smem + Cfg::BAR_OFF + 8 * Cfg::NUM_BARS);
@@ -227,6 +242,12 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
             mbar_init(tfull_bar(b), 1);
             mbar_init(tempty_bar(b), 4);
         }
+        if constexpr (Cfg::CSPLIT) {
+            if (ksplit > 1) {
+                mbar_init(peer_free_bar, ksplit - 1);                  // one arrival per other member
+                mbar_init(rx_full_bar, (ksplit - 1) * (128u / ksplit)); // their threads holding my columns
+            }
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -240,6 +261,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
     }
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (Cfg::CSPLIT) cluster_sync_all();   // the others' barriers exist before any remote arrive
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot_ptr;
 
@@ -249,9 +271,14 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
     const int64_t total = tiles * kb_per_tile;
     const int64_t g = gridDim.x;
     const int64_t c = blockIdx.x;
-    const int64_t it_begin = range_begin(c, total, g);
-    const int64_t it_end = range_begin(c + 1, total, g);
-    const int64_t first_tile = it_begin / kb_per_tile;
+    // stream-K: an equal contiguous share of all iterations per CTA; cluster
+    // split: cluster t takes tile t, member kr its share of the tile's K
+    const int64_t ctile = static_cast<int64_t>(blockIdx.x) / ksplit;
+    const int64_t it_begin = Cfg::CSPLIT ? ctile * kb_per_tile + (static_cast<int64_t>(kr) * kb_per_tile) / ksplit
+                                         : range_begin(c, total, g);
+    const int64_t it_end = Cfg::CSPLIT ? ctile * kb_per_tile + (static_cast<int64_t>(kr + 1) * kb_per_tile) / ksplit
+                                       : range_begin(c + 1, total, g);
+    const int64_t first_tile = Cfg::CSPLIT ? ctile : it_begin / kb_per_tile;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -268,7 +295,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 const int t = static_cast<int>(it / kb_per_tile);
                 const int kb = static_cast<int>(it - static_cast<int64_t>(t) * kb_per_tile);
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarEmpty);
+                    record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleProducer * 16 + kBarEmpty);
                     ok = false;
                     break;
                 }
@@ -289,7 +316,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
             }
             for (int i = 0; ok && i < Cfg::STAGES; ++i) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, 1, kRoleProducer * 16 + kBarTail);
+                    record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleProducer * 16 + kBarTail);
                     ok = false;
                 }
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -311,14 +338,14 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 const uint32_t buf = static_cast<uint32_t>(seg) & 1u;
                 if (!mbar_wait(tempty_bar(buf), ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u, abort_flag,
                                3 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarTmemEmpty);
+                    record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleMma * 16 + kBarTmemEmpty);
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + buf * Cfg::MP;
                 for (int64_t j = it; j < seg_end; ++j) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
-                        record_timeout(status, abort_flag, abort_slot, 1, kRoleMma * 16 + kBarFull);
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleMma * 16 + kBarFull);
                         ok = false;
                         break;
                     }
@@ -353,6 +380,117 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
         const int64_t slot_elems = static_cast<int64_t>(Cfg::TILE_N) * Cfg::MP;
         int seg = 0;
         int64_t it = it_begin;
+        if constexpr (Cfg::CSPLIT) {
+            // ---- cluster split: member kr holds the fp32 partial of its
+            // share of K (none: zeros).  Each warp's 32 columns of C belong to
+            // member owner = its lane quarter / (4 / S): the other members'
+            // warps on those columns send their partials (all mpad rows) to
+            // a slot of the owner's operand ring, and the owner's warp adds
+            // the S partials in member order and writes C.
+            const uint32_t S = ksplit;
+            const bool has_k = it_end > it_begin;
+            bool ok = true;
+            if (has_k) {
+                if (epi_tid == 0) {
+                    uint32_t r = 1;
+                    if (!mbar_wait(tfull_bar(0), 0, abort_flag, 3 * timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarTmemFull);
+                        r = 0;
+                    }
+                    *ready_flag = r;
+                }
+                named_barrier_sync(1, 128);
+                ok = *ready_flag != 0;
+                tc_fence_after_sync();
+            }
+            const uint32_t lanes_per = 128u / S;
+            const uint32_t owner = (sub * 32u) / lanes_per;
+            const uint32_t tbase = tmem_base + ((sub * 32u) << 16);          // accumulator buffer 0
+            const uint32_t row_bytes = static_cast<uint32_t>(mpad) * 4u;
+            const uint32_t slot_bytes = lanes_per * row_bytes;
+            const uint32_t r_in = sub * 32u + lane - owner * lanes_per;      // row in the owner's slots
+            // 16-byte pieces of a row (mpad / 4 of them, a multiple of 4)
+            // rotated within groups of four by the row: fewer bank conflicts
+            auto piece_addr = [&](uint32_t row_base, int m0, int p) {
+                return row_base + (((static_cast<uint32_t>(m0 / 4 + p)) ^ (lane & 3u)) << 4);
+            };
+            auto load16 = [&](int m0, uint32_t (&v)[16]) {
+                if (has_k) {
+                    tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(m0), v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0u;
+                }
+            };
+            if (ok && S > 1) {
+                // this CTA's MMAs are done: its ring may take the others' partials
+                if (epi_tid == 0)
+                    for (uint32_t j = 0; j < S; ++j)
+                        if (j != kr) mbar_arrive_cluster(map_to_cta(peer_free_bar, j));
+                uint32_t wok = 1;
+                if (owner != kr) {
+                    if (lane == 0 && !mbar_wait(peer_free_bar, 0, abort_flag, 3 * timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarPeerFree);
+                        wok = 0;
+                    }
+                    wok = __shfl_sync(0xffffffffu, wok, 0);
+                    if (wok) {
+                        const uint32_t slot = kr < owner ? kr : kr - 1u;
+                        const uint32_t dst_row = map_to_cta(base + slot * slot_bytes + r_in * row_bytes, owner);
+                        for (int m0 = 0; m0 < mpad; m0 += 16) {
+                            uint32_t v[16];
+                            load16(m0, v);
+#pragma unroll
+                            for (int p = 0; p < 4; ++p)
+                                store_cluster_v4(piece_addr(dst_row, m0, p), v[4 * p], v[4 * p + 1], v[4 * p + 2],
+                                                 v[4 * p + 3]);
+                        }
+                        mbar_arrive_cluster(map_to_cta(rx_full_bar, owner));   // release: the stores come first
+                    }
+                } else {
+                    if (lane == 0 && !mbar_wait(rx_full_bar, 0, abort_flag, 3 * timeout_ns)) {
+                        record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarRxFull);
+                        wok = 0;
+                    }
+                    wok = __shfl_sync(0xffffffffu, wok, 0);
+                }
+                ok = wok != 0;
+            }
+            if (ok && owner == kr) {
+                const int n = static_cast<int>(first_tile) * Cfg::TILE_N + n_local;
+                for (int m0 = 0; m0 < mpad; m0 += 16) {
+                    uint32_t own[16];
+                    load16(m0, own);
+                    float acc[16];
+                    for (uint32_t mm = 0; mm < S; ++mm) {
+                        uint32_t x[16];
+                        if (mm == kr) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) x[i] = own[i];
+                        } else {
+                            const uint32_t slot = mm < kr ? mm : mm - 1u;
+                            const uint32_t src_row = base + slot * slot_bytes + r_in * row_bytes;
+#pragma unroll
+                            for (int p = 0; p < 4; ++p)
+                                ld_shared_v4(piece_addr(src_row, m0, p), x[4 * p], x[4 * p + 1], x[4 * p + 2],
+                                             x[4 * p + 3]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[i] = mm == 0 ? __uint_as_float(x[i]) : acc[i] + __uint_as_float(x[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int m = m0 + i;
+                        if (m < M && n < N) store_c<Cfg::OUT>(C, ldc, m, n, acc[i], epi);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(tempty_bar(0));
+            it = it_end;                              // one tile per cluster: nothing further
+        }
         while (it < it_end) {
             const int64_t t = it / kb_per_tile;
             const int64_t seg_end = min(it_end, (t + 1) * kb_per_tile);
@@ -365,7 +503,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
             if (epi_tid == 0) {
                 uint32_t ok = 1;
                 if (!mbar_wait(tfull_bar(buf), (static_cast<uint32_t>(seg) >> 1) & 1u, abort_flag, 3 * timeout_ns)) {
-                    record_timeout(status, abort_flag, abort_slot, 1, kRoleEpilogue * 16 + kBarTmemFull);
+                    record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarTmemFull);
                     ok = 0;
                 }
                 *ready_flag = ok;
@@ -433,11 +571,13 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
 
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (Cfg::CSPLIT) cluster_sync_all();
     if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
     }
     __syncthreads();
+    if constexpr (Cfg::CSPLIT) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc<1>(tmem_base, Cfg::TMEM_COLS);

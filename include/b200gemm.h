@@ -112,9 +112,12 @@ typedef enum {
     GEMM_CFG_1CTA_128x256 = 1,      /* one CTA per tile, tile 128 x 256, tcgen05 cta_group::1 */
     GEMM_CFG_1CTA_128x128 = 2,      /* one CTA per tile, tile 128 x 128 */
     GEMM_CFG_2CTA_256x256 = 3,      /* CTA pair per tile, tile 256 x 256, cta_group::2 */
-    GEMM_CFG_SKINNY = 4,            /* M <= 256: swap A/B (128 rows of B per MMA), stream-K over
-                                       all SMs, deterministic fix-up of split tiles; uses a
-                                       library-owned workspace (cudaMalloc on first use) */
+    GEMM_CFG_SKINNY = 4,            /* M <= 256: swap A/B (128 rows of B per MMA).  For M <= 64
+                                       with enough 128-row tiles of B, K split over a cluster of 2
+                                       or 4 CTAs per tile, partials summed through shared memory;
+                                       otherwise stream-K over all SMs with a deterministic fix-up
+                                       of split tiles in a library-owned workspace (cudaMalloc on
+                                       first use) */
     GEMM_CFG_2CTA_256x256_CLC = 5,  /* as 2CTA_256x256, tiles handed out by Cluster Launch Control:
                                        one cluster per tile, running pairs claim pending ones */
     GEMM_CFG_1CTA_128x256_CLC = 6,  /* as 1CTA_128x256 with Cluster Launch Control */
@@ -342,7 +345,7 @@ B200GEMM_API int gemm_last_cuda_error(void);
 B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
 
 /* The configuration the next gemm_bf16 call with this shape would use.
- * M <= 32 with K >= 8192: GEMM_CFG_SKINNY.  K >= 2048 with at most 74
+ * M <= 32 with K >= 4096: GEMM_CFG_SKINNY.  K >= 2048 with at most 74
  * tiles of 128 x 128 (else of 128 x 256): GEMM_CFG_1CTA_128x128_SPLITK
  * (GEMM_CFG_1CTA_128x256_SPLITK).  Every 128 x 128 tile on an SM of its
  * own: GEMM_CFG_1CTA_128x128.

@@ -161,13 +161,16 @@ def test_status_strings_and_config_control():
     assert G.gemm_select_config(1000, 1000, 1000) == G.CONFIGS["1cta_128x128"]   # K < 2048: no split
     # tiles for at most half the SMs and K >= 2048: cluster split-K
     assert G.gemm_select_config(64, 4096, 4096) == G.CONFIGS["1cta_128x128_splitk"]
+    assert G.gemm_select_config(48, 8192, 4096) == G.CONFIGS["1cta_128x128_splitk"]
     assert G.gemm_select_config(64, 8192, 8192) == G.CONFIGS["1cta_128x128_splitk"]
     assert G.gemm_select_config(256, 4096, 4096) == G.CONFIGS["1cta_128x128_splitk"]    # 64 tiles
     assert G.gemm_select_config(256, 8192, 8192) == G.CONFIGS["1cta_128x256_splitk"]    # 128; 64 wide
     assert G.gemm_select_config(512, 4096, 4096) == G.CONFIGS["1cta_128x256_splitk"]
-    # a few rows and a long K: the skinny stream-K kernel
+    # a few rows and a long K: the skinny (swapped A/B) kernel
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(32, 2048, 8192) == G.CONFIGS["skinny"]
+    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
+    assert G.gemm_select_config(32, 4096, 2048) == G.CONFIGS["1cta_128x128_splitk"]
     # the 256 x 224 and stream-K configurations are never chosen by shape
     seen = {G.gemm_select_config(m, n, k) for m in (1, 100, 300, 1000, 3000, 8192)
             for n in (64, 1000, 3000, 8192) for k in (16, 1000, 5000, 16384)}

@@ -1,4 +1,4 @@
-"""GPU parity of the skinny path (M <= 256, chosen by shape for M <= 64): A and B swapped so 128 rows of B
+"""GPU parity of the skinny path (M <= 256, chosen by shape for M <= 32): A and B swapped so 128 rows of B
 fill the MMA, stream-K over every SM, split tiles finished by the last
 contributor in contributor order.  Compared with the oracle element by
 element; integer inputs bit-exact."""
@@ -31,10 +31,9 @@ def _check(M, N, K, dist, workload, c_type=F32, lda=None, config="skinny", repea
 def test_auto_selects_skinny_for_small_m():
     assert G.gemm_select_config(16, 8192, 8192) == G.CONFIGS["skinny"]
     assert G.gemm_select_config(32, 2048, 8192) == G.CONFIGS["skinny"]
-    # past 32 rows (or over a shorter K) the skinny kernel's fp32 partials
-    # cost more than the cluster split-K kernel's on-chip sum
+    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["skinny"]
+    # past 32 rows the split-K tile kernel wins
     assert G.gemm_select_config(64, 8192, 8192) == G.CONFIGS["1cta_128x128_splitk"]
-    assert G.gemm_select_config(32, 4096, 4096) == G.CONFIGS["1cta_128x128_splitk"]
 
 
 @pytest.mark.parametrize("c_type", [F32, BF16])
@@ -77,3 +76,57 @@ def test_forcing_skinny_above_256_rows_is_rejected():
     a_bits, b_bits = synth.bf16_operands(300, 64, 64, "uniform", workload=142)
     with pytest.raises(G.GemmError):
         run_gemm(a_bits, b_bits, 300, 64, 64, config="skinny")
+
+
+# ---- the cluster-split form (M <= 64 with enough 128-row tiles of B to keep
+# most SMs streaming): K split over 2 or 4 CTAs per tile, partials summed in
+# member order through distributed shared memory
+
+CLUSTER_SHAPES = [(16, 4096, 1024), (40, 8192, 512), (1, 3100, 2048), (64, 6400, 768)]
+
+
+@pytest.mark.parametrize("shape", CLUSTER_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("c_type", [F32, BF16])
+def test_cluster_split_integers_bit_exact(shape, c_type):
+    M, N, K = shape
+    _check(M, N, K, "ints", workload=600 + M, c_type=c_type)
+
+
+@pytest.mark.parametrize("shape", CLUSTER_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("c_type", [F32, BF16])
+def test_cluster_split_normal(shape, c_type):
+    M, N, K = shape
+    _check(M, N, K, "normal", workload=620 + M, c_type=c_type)
+
+
+def test_cluster_split_deterministic():
+    """Member order, not arrival order, fixes the sum: repeated calls give
+    the same bits."""
+    M, N, K = 24, 4096, 2048
+    a_bits, b_bits = synth.bf16_operands(M, N, K, "normal", workload=640)
+    first = run_gemm(a_bits, b_bits, M, N, K, config="skinny").bits()
+    for _ in range(3):
+        assert (run_gemm(a_bits, b_bits, M, N, K, config="skinny").bits() == first).all()
+
+
+def test_cluster_split_fused_epilogue_and_transposed_b():
+    """alpha, beta, bias and ReLU in the owner's write-back; B stored K x N."""
+    import torch
+
+    from gpu_helpers import to_device_bf16
+    M, N, K = 33, 4096, 1024
+    a, b = synth.bf16_operands(M, N, K, "ints", workload=641)
+    bT = np.ascontiguousarray(b.T)
+    c_old = synth.small_ints(642, (M, N), -8, 8)
+    bias = synth.small_ints(643, (N,), -20, 20).astype(np.float32)
+    C = torch.from_numpy(c_old.astype(np.float32)).cuda()
+    G.gemm_force_config("skinny")
+    try:
+        G.gemm_bf16_fused(to_device_bf16(a), to_device_bf16(bT), C, M, N, K, K, N, N, F32, G.KMAJOR, G.MNMAJOR,
+                          1.0, -1.0, torch.from_numpy(bias).cuda(), G.ACT_RELU)
+    finally:
+        G.gemm_force_config("auto")
+    G.gemm_check_device_status()
+    ab = oracle.gemm_bf16_f64(a, b)
+    want = oracle.epilogue(ab, c_old.astype(np.float64), 1.0, -1.0, bias.astype(np.float64), G.ACT_RELU)
+    assert_exact(C.cpu().numpy().astype(np.float64), want, F32, "cluster skinny fused")
