@@ -676,12 +676,14 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
 // The skinny tile with K split over a cluster of S CTAs per 128-row tile of
 // B (no workspace: the partials meet in shared memory).  S: 4 or 2, the
 // largest whose clusters all fit at once, leave every member two 64-wide K
-// blocks and keep at least 96 SMs streaming; 1 = none qualifies (the caller
-// runs the stream-K kernel).
+// blocks, keep at least 96 SMs streaming, and give no member more than 2048
+// of K (a longer share streams better on all 148 SMs with stream-K:
+// 16 x 8192 x 8192 ran 35.4 us that way against 36.9 split in clusters of
+// two); 1 = none qualifies (the caller runs the stream-K kernel).
 template <class Cfg>
-gemm_status_t launch_skinny_cluster(DeviceState *st, int slot, const void *A, const void *B, void *C, int64_t M,
-                                    int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream,
-                                    const b200::Epilogue &epi, uint32_t layout, bool &launched) {
+gemm_status_t launch_skinny_cluster(DeviceState *st, DeviceStatus *status, int slot, const void *A, const void *B,
+                                    void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                                    cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout, bool &launched) {
     launched = false;
     auto kernel = b200::gemm_bf16_skinny_sm100_kernel<Cfg>;
     cudaError_t e;
@@ -719,7 +721,7 @@ gemm_status_t launch_skinny_cluster(DeviceState *st, int slot, const void *A, co
     int S = 1;
     for (int li = 1; li >= 0; --li) {
         const int cand = 2 << li;
-        if (tiles * cand <= st->skc_ctas[slot][li] && kb >= 2 * cand && tiles * cand >= 96) {
+        if (tiles * cand <= st->skc_ctas[slot][li] && kb >= 2 * cand && tiles * cand >= 96 && K <= 2048 * cand) {
             S = cand;
             break;
         }
@@ -741,7 +743,7 @@ gemm_status_t launch_skinny_cluster(DeviceState *st, int slot, const void *A, co
     float *no_partials = nullptr;
     unsigned long long *no_counters = nullptr;
     e = cudaLaunchKernelEx(&lc, kernel, tmB, tmA, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-                           static_cast<int>(mpad), C, ldc, no_partials, no_counters, 0, 0u, st->status, watchdog_ns(K),
+                           static_cast<int>(mpad), C, ldc, no_partials, no_counters, 0, 0u, status, watchdog_ns(K),
                            epi, layout);
     if (e != cudaSuccess) return cuda_fail(e);
     launched = true;
@@ -757,10 +759,10 @@ gemm_status_t launch_skinny_any(DeviceState *st, bool f32, const void *A, const 
         // enough 128-row tiles of B to keep most SMs streaming with K split
         // over a cluster: the partials stay on chip; otherwise stream-K
         bool launched = false;
-        gemm_status_t s = f32 ? launch_skinny_cluster<CfgSk64F32C>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream,
-                                                                   epi, layout, launched)
-                              : launch_skinny_cluster<CfgSk64B16C>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream,
-                                                                   epi, layout, launched);
+        gemm_status_t s = f32 ? launch_skinny_cluster<CfgSk64F32C>(st, st->status, 0, A, B, C, M, N, K, lda, ldb,
+                                                                   ldc, stream, epi, layout, launched)
+                              : launch_skinny_cluster<CfgSk64B16C>(st, st->status, 1, A, B, C, M, N, K, lda, ldb,
+                                                                   ldc, stream, epi, layout, launched);
         if (s != GEMM_OK || launched) return s;
         return f32 ? launch_skinny<CfgSk64F32>(st, 0, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)
                    : launch_skinny<CfgSk64B16>(st, 1, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
@@ -1206,11 +1208,21 @@ gemm_status_t gemm_bf16_noalloc(const void *A, const void *B, void *C, int64_t M
         return c_type == GEMM_OUT_F32 ? launch_zero<uint32_t>(C, M, N, ldc, st->sm_count, stream)
                                       : launch_zero<uint16_t>(C, M, N, ldc, st->sm_count, stream);
     }
-    // The skinny and stream-K kernels need a workspace; without one, small-M
-    // shapes run on the cluster split-K kernel (its partials meet in shared
-    // memory) and stream-K shapes on the CLC pair kernel instead.
+    // The stream-K kernels need a workspace; without one, small-M shapes run
+    // on the skinny tile split over a cluster where that applies, else on
+    // the split-K tile kernel (both sum their partials in shared memory),
+    // and stream-K shapes on the CLC pair kernel.
     gemm_config_t cfg = select_config(M, N, K);
-    if (cfg == GEMM_CFG_SKINNY) cfg = GEMM_CFG_1CTA_128x128_SPLITK;
+    if (cfg == GEMM_CFG_SKINNY) {
+        bool launched = false;
+        const bool f32 = c_type == GEMM_OUT_F32;
+        s = f32 ? launch_skinny_cluster<CfgSk64F32C>(st, st->noalloc_status, 0, A, B, C, M, N, K, lda, ldb, ldc,
+                                                     stream, b200::plain_epilogue(), 0u, launched)
+                : launch_skinny_cluster<CfgSk64B16C>(st, st->noalloc_status, 1, A, B, C, M, N, K, lda, ldb, ldc,
+                                                     stream, b200::plain_epilogue(), 0u, launched);
+        if (s != GEMM_OK || launched) return s;
+        cfg = GEMM_CFG_1CTA_128x128_SPLITK;
+    }
     if (cfg == GEMM_CFG_2CTA_256x256_SK) cfg = GEMM_CFG_2CTA_256x256_CLC;   // stream-K needs a workspace too
     return launch_dense(st, st->noalloc_status, cfg, c_type == GEMM_OUT_F32, A, B, C, M, N, K, lda, ldb, ldc,
                         stream, b200::plain_epilogue(), 0u);

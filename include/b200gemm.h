@@ -287,11 +287,10 @@ B200GEMM_API gemm_status_t gemm_mxfp8(const void *A, const uint8_t *sfa, const v
  * arguments, checks and kernels, but it allocates nothing: the kernels'
  * scratch (the 16-byte watchdog status block) lives in a static 256-byte
  * device array inside the library, which every GPU that loads the library
- * holds until the process exits.  One difference in kernel choice: the
- * skinny split-K kernel (GEMM_CFG_SKINNY), whose workspace gemm_bf16
- * allocates, is replaced by GEMM_CFG_1CTA_128x128_SPLITK (which needs no
- * workspace: its partials meet in shared memory), so the few shapes that
- * take the skinny kernel (M <= 32, K >= 8192) run somewhat slower here.  A call that would need more scratch than that array is
+ * holds until the process exits.  One difference in kernel choice: where
+ * GEMM_CFG_SKINNY would fall back to its stream-K form, whose workspace
+ * gemm_bf16 allocates, this runs GEMM_CFG_1CTA_128x128_SPLITK instead (no
+ * workspace: its partials meet in shared memory).  A call that would need more scratch than that array is
  * rejected with GEMM_ERR_TOO_LARGE (no shape does today: the scratch does
  * not grow with M, N or K).  Each call queues exactly one kernel.
  *
@@ -338,7 +337,7 @@ B200GEMM_API int gemm_last_cuda_error(void);
  * (GEMM_CFG_AUTO restores shape-based selection).  A bf16 configuration
  * applies to gemm_bf16, gemm_bf16_ex and gemm_bf16_fused (except that an A
  * stored K x M never runs on GEMM_CFG_SKINNY) and to gemm_bf16_noalloc
- * (which runs GEMM_CFG_SKINNY as GEMM_CFG_1CTA_128x128_SPLITK); an MXFP8 one
+ * (which runs GEMM_CFG_SKINNY's stream-K form as GEMM_CFG_1CTA_128x128_SPLITK); an MXFP8 one
  * applies to gemm_mxfp8, and leaves the bf16 entry points choosing by shape.
  * A forced GEMM_CFG_SKINNY with M > 256 fails with GEMM_ERR_INVALID_VALUE.
  * Returns GEMM_ERR_INVALID_VALUE for an unknown configuration. */

@@ -93,12 +93,14 @@ def test_noalloc_runs_the_cluster_launch_control_kernel():
     assert np.all(np.abs(got - c64) <= tolerance(c64, s_abs, G.OUT_BF16))
 
 
-def test_noalloc_small_m_runs_the_split_k_kernel():
-    """Where gemm_bf16 takes the skinny kernel (whose partials live in an
-    allocated workspace), the allocation-free entry point runs the cluster
-    split-K kernel, whose partials meet in shared memory: same result within
-    the tolerance, no device memory taken."""
-    M, N, K = 16, 1024, 8192
+@pytest.mark.parametrize("shape", [(16, 1024, 8192), (16, 8192, 4096)], ids=["split_k_tiles", "skinny_cluster"])
+def test_noalloc_small_m_needs_no_workspace(shape):
+    """Where gemm_bf16 takes the skinny kernel, the allocation-free entry
+    point runs its cluster split (8192 columns: 64 tiles of B) or, where
+    that does not apply (1024 columns), the split-K tile kernel: both sum
+    their partials in shared memory.  Same result within the tolerance, no
+    device memory taken."""
+    M, N, K = shape
     assert G.gemm_select_config(M, N, K) == G.CONFIGS["skinny"]
     a_bits, b_bits = synth.bf16_operands(M, N, K, "normal", workload=74)
     A, B = to_device_bf16(a_bits), to_device_bf16(b_bits)
