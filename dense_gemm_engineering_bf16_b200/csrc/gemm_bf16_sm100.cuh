@@ -452,19 +452,26 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     };
 
     // Work units: K blocks [kb0, kb1) of one tile.  Static and CLC
-    // schedules: whole tiles from next_tile.  Stream-K: the pieces of this
-    // cluster's range [it_begin, it_end) of the (tile, K block) iterations
-    // (K fastest), one piece per tile the range touches.  The split pieces
-    // (a range boundary inside the tile: at most the first and the last)
-    // run first, so the tiles shared with the neighbouring clusters are
-    // complete early and their fix-ups overlap this cluster's whole tiles
-    // instead of ending the launch.
+    // schedules: whole tiles from next_tile.  Stream-K with a data-parallel
+    // head: with W >= 2 full waves of tiles, the first (W - 1) waves are whole
+    // tiles dealt round robin (cluster c: c, c + G, ...); the (tile, K block)
+    // iterations of the remaining tiles (one wave plus the partial one) are
+    // cut into one contiguous range [it_begin, it_end) per cluster, one piece
+    // per tile the range touches.  A cluster runs its split pieces (a range
+    // boundary inside the tile: at most the first and the last) first, then
+    // its data-parallel tiles, then its whole stream-K tiles: the tiles
+    // shared with the neighbouring clusters complete early, so their fix-ups
+    // overlap whole tiles instead of ending the launch.
     struct Unit {
         int tile, kb0, kb1;
     };
-    const int64_t sk_total = static_cast<int64_t>(num_tiles) * num_kb;
-    const int64_t it_begin = Cfg::SK ? (static_cast<int64_t>(cluster_id) * sk_total) / num_clusters : 0;
-    const int64_t it_end = Cfg::SK ? (static_cast<int64_t>(cluster_id + 1) * sk_total) / num_clusters : 0;
+    const int64_t sk_waves = static_cast<int64_t>(num_tiles) / num_clusters;
+    const int64_t dp_tiles = (Cfg::SK && sk_waves >= 2) ? (sk_waves - 1) * num_clusters : 0;
+    const int dp_units = static_cast<int>(dp_tiles / num_clusters);     // data-parallel tiles per cluster
+    const int64_t sk_base = dp_tiles * num_kb;                           // first stream-K iteration
+    const int64_t sk_total = (static_cast<int64_t>(num_tiles) - dp_tiles) * num_kb;
+    const int64_t it_begin = Cfg::SK ? sk_base + (static_cast<int64_t>(cluster_id) * sk_total) / num_clusters : 0;
+    const int64_t it_end = Cfg::SK ? sk_base + (static_cast<int64_t>(cluster_id + 1) * sk_total) / num_clusters : 0;
     const int64_t sk_tile0 = it_begin / num_kb;
     const int sk_units = it_end > it_begin ? static_cast<int>((it_end - 1) / num_kb - sk_tile0 + 1) : 0;
     auto sk_range_unit = [&](int i) -> Unit {        // the i-th piece in range order
@@ -489,10 +496,19 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         return (sk_split_first ? 1 : 0) + j;
     };
+    // the j-th unit this cluster runs: split stream-K pieces, data-parallel
+    // tiles, whole stream-K tiles
+    const int sk_split_units = (sk_split_last ? 1 : 0) + (sk_split_first ? 1 : 0);
+    auto sk_unit = [&](int j) -> Unit {
+        if (j < sk_split_units) return sk_range_unit(sk_order(j));
+        if (j < sk_split_units + dp_units)
+            return Unit{cluster_id + (j - sk_split_units) * num_clusters, 0, num_kb};
+        return sk_range_unit(sk_order(j - dp_units));
+    };
     auto first_unit = [&](Unit &u) -> bool {
         if constexpr (Cfg::SK) {
-            if (sk_units == 0) return false;
-            u = sk_range_unit(sk_order(0));
+            if (sk_units + dp_units == 0) return false;
+            u = sk_unit(0);
             return true;
         } else {
             u = Unit{cluster_id, kb_lo, kb_hi};
@@ -503,8 +519,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     auto next_unit = [&](Unit &u, uint32_t j, bool &ok) -> bool {
         if constexpr (Cfg::SK) {
             (void)ok;
-            if (static_cast<int>(j) + 1 >= sk_units) return false;
-            u = sk_range_unit(sk_order(static_cast<int>(j) + 1));
+            if (static_cast<int>(j) + 1 >= sk_units + dp_units) return false;
+            u = sk_unit(static_cast<int>(j) + 1);
             return true;
         } else {
             const int n = next_tile(u.tile, j, ok);
@@ -897,10 +913,11 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 // clusters.  Write this CTA's fp32 partial (row 32 sub + lane,
                 // all BN columns) to its slot, count the arrival, and let the
                 // last contributor sum every partial in contributor order.
+                // (iterations counted from the first stream-K one)
                 const int64_t G = num_clusters;
-                auto owner = [&](int64_t it) { return ((it + 1) * G + sk_total - 1) / sk_total - 1; };
+                auto owner = [&](int64_t it) { return ((it - sk_base + 1) * G + sk_total - 1) / sk_total - 1; };
                 auto part = [&](int64_t cc) -> float * {
-                    const int64_t first = ((cc * sk_total) / G) / num_kb;   // cc's first tile
+                    const int64_t first = (sk_base + (cc * sk_total) / G) / num_kb;   // cc's first stream-K tile
                     const int64_t slot = (cc * CG + rank) * 2 + (tile == first ? 0 : 1);
                     return sk_partials + slot * (128 * Cfg::BN);
                 };
