@@ -1039,7 +1039,9 @@ gemm_status_t gemm_bf16_fused(const void *A, const void *B, void *C, int64_t M, 
     }
     const uint32_t layout = (a_mn ? b200::kLayoutAMajorM : 0u) | (b_mn ? b200::kLayoutBMajorN : 0u);
     gemm_config_t cfg = select_config(M, N, K);
-    if (cfg == GEMM_CFG_SKINNY && a_mn) cfg = GEMM_CFG_1CTA_128x128;   // skinny reads A K-major only
+    // the skinny kernel reads A K-major only: an A stored K x M takes the
+    // split-K tile kernel, which also spreads a long K over idle SMs
+    if (cfg == GEMM_CFG_SKINNY && a_mn) cfg = GEMM_CFG_1CTA_128x128_SPLITK;
     // The two-consumer tile holds one tile in TMEM, so its epilogue stalls
     // the MMA; with epilogue work beyond the plain store (beta, bias, an
     // activation) the double-buffered 256 x 256 tile hides it instead.

@@ -336,9 +336,10 @@ B200GEMM_API int gemm_last_cuda_error(void);
 /* Force a kernel configuration for subsequent calls in this process
  * (GEMM_CFG_AUTO restores shape-based selection).  A bf16 configuration
  * applies to gemm_bf16, gemm_bf16_ex and gemm_bf16_fused (except that an A
- * stored K x M never runs on GEMM_CFG_SKINNY) and to gemm_bf16_noalloc
- * (which runs GEMM_CFG_SKINNY's stream-K form as GEMM_CFG_1CTA_128x128_SPLITK); an MXFP8 one
- * applies to gemm_mxfp8, and leaves the bf16 entry points choosing by shape.
+ * stored K x M runs GEMM_CFG_SKINNY as GEMM_CFG_1CTA_128x128_SPLITK) and to
+ * gemm_bf16_noalloc (which runs GEMM_CFG_SKINNY's stream-K form as
+ * GEMM_CFG_1CTA_128x128_SPLITK); an MXFP8 one applies to gemm_mxfp8, and
+ * leaves the bf16 entry points choosing by shape.
  * A forced GEMM_CFG_SKINNY with M > 256 fails with GEMM_ERR_INVALID_VALUE.
  * Returns GEMM_ERR_INVALID_VALUE for an unknown configuration. */
 B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
@@ -360,7 +361,8 @@ B200GEMM_API gemm_status_t gemm_force_config(gemm_config_t config);
  * epilogue (beta != 0, alpha != 1, a bias or an activation) they take
  * GEMM_CFG_2CTA_256x256_CLC where this returns GEMM_CFG_2CTA_512x256_CLC
  * (the 256 x 256 tile's second TMEM buffer hides the longer epilogue), and
- * an A stored K x M never takes GEMM_CFG_SKINNY. */
+ * an A stored K x M takes GEMM_CFG_1CTA_128x128_SPLITK where this returns
+ * GEMM_CFG_SKINNY. */
 B200GEMM_API gemm_config_t gemm_select_config(int64_t M, int64_t N, int64_t K);
 
 /* Number of kernels that one call queues for this shape: gemm_bf16 /

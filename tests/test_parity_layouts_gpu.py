@@ -64,7 +64,7 @@ def test_operand_layouts_integers_bit_exact(cfg, layouts, shape):
     a_l, b_l = layouts
     M, N, K = shape
     if cfg == "skinny":                  # the swap-AB path takes at most 256 rows; with A stored
-        M = min(M, 250)                  # K x M the call is routed to the 128 x 128 kernel
+        M = min(M, 250)                  # K x M the call is routed to the 128 x 128 split-K kernel
     got, want, _, _ = _run(M, N, K, "ints", 200 + M, cfg, a_l, b_l)
     assert_exact(got, want, F32, f"{cfg} layouts {layouts} {shape}")
 
