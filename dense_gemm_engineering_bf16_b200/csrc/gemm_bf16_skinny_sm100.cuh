@@ -435,6 +435,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                         wok = 0;
                     }
                     wok = __shfl_sync(0xffffffffu, wok, 0);
+                    __syncwarp();   // lane 0's acquire orders every lane's accesses that follow
                     if (wok) {
                         const uint32_t slot = kr < owner ? kr : kr - 1u;
                         const uint32_t dst_row = map_to_cta(base + slot * slot_bytes + r_in * row_bytes, owner);
@@ -454,6 +455,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                         wok = 0;
                     }
                     wok = __shfl_sync(0xffffffffu, wok, 0);
+                    __syncwarp();   // lane 0's acquire orders every lane's accesses that follow
                 }
                 ok = wok != 0;
             }

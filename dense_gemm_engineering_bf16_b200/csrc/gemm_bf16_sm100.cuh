@@ -819,6 +819,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                         fr = 0;
                     }
                     xok = __shfl_sync(0xffffffffu, fr, 0) != 0;
+                    __syncwarp();   // lane 0's acquire orders every lane's accesses that follow
                     if (xok) {
                         // slice j of this partial, row `arow`, to this member's slot
                         // at member j; 16-byte pieces swizzled by the row, so a
@@ -847,6 +848,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                             rf = 0;
                         }
                         xok = __shfl_sync(0xffffffffu, rf, 0) != 0;
+                        __syncwarp();   // the other members' stores are visible to every lane
                     }
                 }
                 // 32 columns of slice kr (from slice column c * 32): the
