@@ -191,3 +191,29 @@ def test_binding_constants_match_the_header():
     assert (enum["GEMM_OUT_F32"], enum["GEMM_OUT_BF16"]) == (G.OUT_F32, G.OUT_BF16)
     for code, name in G.STATUS_NAMES.items():
         assert enum[name] == code
+
+
+def test_configuration_choice_respects_its_own_rules():
+    """Over a grid of shapes, the shape-based choice keeps to the rules its
+    cost model was fitted under: the skinny kernel only for M <= 32 with a
+    long K, split-K only with K >= 2048 and tiles for at most half the SMs,
+    the single-buffered 512 x 256 tile only for K >= 8192, one-CTA 128 x 256
+    tiles for at most two waves, and never the forced-only kernels."""
+    G.gemm_force_config("auto")
+    C = G.CONFIGS
+    cdiv = lambda a, b: -(-a // b)  # noqa: E731
+    for M in (1, 16, 32, 33, 64, 100, 256, 300, 512, 1000, 2048, 4096, 8192):
+        for N in (64, 256, 1000, 2048, 4096, 8192, 16384):
+            for K in (16, 512, 1024, 2048, 4096, 8192, 16384):
+                c = G.gemm_select_config(M, N, K)
+                assert c in C.values() and c not in (C["auto"], C["2cta_256x224"], C["2cta_256x256_sk"]), (M, N, K)
+                if c == C["skinny"]:
+                    assert M <= 32 and K >= 4096, (M, N, K)
+                if c in (C["1cta_128x128_splitk"], C["1cta_128x256_splitk"]):
+                    assert K >= 2048, (M, N, K)
+                    width = 128 if c == C["1cta_128x128_splitk"] else 256
+                    assert cdiv(M, 128) * cdiv(N, width) <= 74, (M, N, K)
+                if c in (C["2cta_512x256_clc"], C["1cta_128x256_clc"]):
+                    assert K >= 8192, (M, N, K)
+                if c == C["1cta_128x256"]:
+                    assert cdiv(M, 128) * cdiv(N, 256) <= 2 * 148, (M, N, K)
