@@ -142,7 +142,9 @@ typedef enum {
                                        order (deterministic), the partials crossing through
                                        distributed shared memory (no workspace).  S: the largest
                                        whose clusters all fit at once and give every member two
-                                       64-wide K blocks (else the unsplit 1CTA_128x128) */
+                                       64-wide K blocks (else the unsplit 1CTA_128x128); the
+                                       environment variable B200GEMM_KSPLIT = 2, 4 or 8, read
+                                       once, forces it (tests) */
     GEMM_CFG_1CTA_128x256_SPLITK = 13, /* the same with 128 x 256 tiles (else 1CTA_128x256) */
     GEMM_CFG_COUNT_ = 14
 } gemm_config_t;
