@@ -397,6 +397,15 @@ gemm_status_t setup_attrs(DeviceState *st, gemm_config_t cfg_id, cudaStream_t st
     if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES)) !=
         cudaSuccess)
         return cuda_fail(e);
+    // the narrow-tail twin (same shared memory, same co-resident count) is
+    // set up with it, so that a later launch that splits its tail needs no
+    // first-call work (it may be inside a stream capture)
+    if constexpr (Cfg::TAIL_OK) {
+        if ((e = cudaFuncSetAttribute(b200::gemm_bf16_sm100_kernel<typename Cfg::Tail>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::Tail::SMEM_BYTES)) !=
+            cudaSuccess)
+            return cuda_fail(e);
+    }
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = Cfg::CG;
@@ -503,7 +512,25 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
         return GEMM_ERR_INVALID_VALUE;
     cudaError_t e;
     gemm_status_t s;
-    if ((s = setup_attrs<Cfg>(st, cfg_id, stream)) != GEMM_OK) return s;
+    if constexpr (!Cfg::TAIL) {   // (a narrow-tail twin is set up with its whole-tile kernel)
+        if ((s = setup_attrs<Cfg>(st, cfg_id, stream)) != GEMM_OK) return s;
+    }
+    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
+    const int64_t resident = st->max_clusters[cfg_id][oi];
+    const bool b_kmajor = !(layout & b200::kLayoutBMajorN);
+    // Narrow tail: a last wave of R tiles that would leave at least half of
+    // the co-resident clusters idle (0 < 2 R <= resident) runs as 2 R
+    // half-width units on the tile's twin kernel, so that every cluster has
+    // work at the end (measured: 102.0 -> 100.8 us at 4096^3 on 256 x 256
+    // pair tiles, 107.1 -> 103.4 on 128 x 256 one-CTA tiles; the halves
+    // reread A, so the tail shrinks by less than half a tile).
+    const int64_t rem = resident > 0 ? tiles % resident : 0;
+    const bool split_tail = b_kmajor && rem > 0 && 2 * rem <= resident;
+    if constexpr (Cfg::TAIL_OK && !Cfg::TAIL) {
+        if (split_tail)
+            return launch_bf16<typename Cfg::Tail>(st, status, cfg_id, A, B, C, M, N, K, lda, ldb, ldc, stream, epi,
+                                                   layout, peers, ksplit);
+    }
     const int cluster_ctas = Cfg::SPLITK ? ksplit : Cfg::CG;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -518,7 +545,7 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     lc.numAttrs = 1;
     const CUtensorMapDataType cdt = Cfg::OUT == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int64_t ec = Cfg::OUT == 0 ? 4 : 2;
-    alignas(64) CUtensorMap tmA, tmB, tmC;
+    alignas(64) CUtensorMap tmA, tmB, tmC, tmBt;
     // K-major operands: boxes of 64 (K) x rows; MN-major (stored K x M / K x N):
     // boxes of 64 (MN) x 64 (K)
     if (layout & b200::kLayoutAMajorM)
@@ -531,6 +558,14 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     else
         s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::B_ROWS);
     if (s != GEMM_OK) return s;
+    // B for the half-width units of a narrow tail (K-major B only)
+    if (Cfg::TAIL) {
+        if ((s = encode_2d(&tmBt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::B_ROWS / 2)) !=
+            GEMM_OK)
+            return s;
+    } else {
+        tmBt = tmB;
+    }
     // The store map covers the columns that end on a 16-byte granule; the
     // kernel writes the rest of each row ([n_tma, N)) with plain stores.  If
     // no whole granule exists the map is a placeholder the kernel never uses.
@@ -538,14 +573,18 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
     if ((s = encode_2d(&tmC, cdt, C, n_tma > 0 ? n_tma : 16 / ec, M, ldc * ec, Cfg::EPI_COLS, 32)) != GEMM_OK)
         return s;
 
-    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     // Static schedule: as many clusters as fit at once, each striding over
     // the tiles.  CLC: one cluster per tile; running clusters claim the rest.
     // Split-K: one cluster of `ksplit` CTAs per tile.  Stream-K: every
     // co-resident cluster, each with an equal share of the (tile, K block)
     // iterations.
-    const int64_t resident = st->max_clusters[cfg_id][oi];
-    int64_t clusters = (Cfg::CLC || Cfg::SPLITK) ? tiles : (tiles > resident ? resident : tiles);
+    // (the twin runs units [0, tiles - R) as whole tiles, then 2 R halves)
+    int64_t tail_first = tiles, units = tiles;
+    if (Cfg::TAIL && split_tail) {
+        tail_first = tiles - rem;
+        units = tiles + rem;
+    }
+    int64_t clusters = (Cfg::CLC || Cfg::SPLITK) ? units : (units > resident ? resident : units);
     if constexpr (Cfg::SK) {
         // Every cluster's range must hold at least one iteration (the
         // fix-up counts a split tile's contributors as the consecutive range
@@ -576,9 +615,10 @@ gemm_status_t launch_bf16(DeviceState *st, DeviceStatus *status, gemm_config_t c
         epoch = ++st->sk_epoch;
         if (epoch == 0) epoch = ++st->sk_epoch;
     }
-    e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, static_cast<int>(M), static_cast<int>(N),
-                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), wave_tiles, status,
-                           watchdog_ns(K), inject_flags(), epi, layout, sk_partials, sk_counters, epoch, peer_arg);
+    e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmC, tmBt, static_cast<int>(M), static_cast<int>(N),
+                           static_cast<int>(K), C, ldc, static_cast<int>(n_tma), raster_group_m(), wave_tiles,
+                           static_cast<int>(tail_first), units > tiles ? 2 : 1, status, watchdog_ns(K), inject_flags(),
+                           epi, layout, sk_partials, sk_counters, epoch, peer_arg);
     if (e != cudaSuccess) return cuda_fail(e);
     return GEMM_OK;
 }

@@ -45,6 +45,15 @@
 // 执行模型", section "编译与 autotune"), with the reduction on chip: no
 // workspace, no atomics, and a fixed summation order.
 //
+// Narrow tail (TAIL: one consumer, static or CLC schedule, K-major B): when
+// the tiles left for a last wave would occupy at most half of the
+// co-resident clusters, each of them runs as two units of BN / 2 columns
+// (an MMA of N = BN / 2 over half of the B rows), so the clusters that would
+// have idled take the other halves.  This is the wave-tail entry of the
+// pages' autotune search space ("GPU 执行模型", section "编译与 autotune":
+// tile shape and persistent strategy), without a reduction: each half is a
+// whole block of C.
+//
 // Operands may be K-major (A as M x K, B as N x K) or MN-major (A as K x M,
 // B as K x N): MN-major tiles arrive as 64-wide boxes and the MMA reads them
 // through MN-major descriptors.  The epilogue computes
@@ -107,7 +116,7 @@ struct PeerC {
 struct NoPeerC {};
 
 template <int CG_, int BN_, int STAGES_, int OUT_, bool CLC_ = false, int CONSUMERS_ = 1, bool SK_ = false,
-          bool PEERS_ = false, bool SPLITK_ = false>
+          bool PEERS_ = false, bool SPLITK_ = false, bool TAIL_ = false>
 struct GemmBf16Cfg {
     static constexpr bool CLC = CLC_;              // tiles from Cluster Launch Control, not a fixed stride
     // Stream-K: the (tile, K block) iterations are cut into one contiguous
@@ -155,6 +164,16 @@ struct GemmBf16Cfg {
     // after the barriers: TMEM address, abort flag, 2 tile ids, 2 CLC answers
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NUM_BARS * 8 + 64;
     static constexpr int THREADS = CLC ? 224 : 192;        // + one scheduler warp
+    // Narrow tail: when the last wave of tiles would fill at most half of the
+    // co-resident clusters, each of its tiles may run as two half-width units
+    // (BN / 2 columns each) on two clusters, so that every cluster gets work.
+    // TAIL_OK: this tile has such a twin (Tail), a separate instantiation
+    // launched only when the tail splits, so that whole-tile launches run
+    // code without the half-unit logic.
+    static constexpr bool TAIL_OK = CONSUMERS == 1 && !SK && !SPLITK && !PEERS && (BN / 2) % EPI_COLS == 0 &&
+                                    (B_ROWS / 2) % 8 == 0;
+    static constexpr bool TAIL = TAIL_;
+    using Tail = GemmBf16Cfg<CG_, BN_, STAGES_, OUT_, CLC_, CONSUMERS_, SK_, PEERS_, SPLITK_, true>;
     static constexpr int SCHED_CONSUMERS = CG == 1 ? 6 : 11;  // arrivals that free a tile slot
 
     static_assert(CG == 1 || CG == 2, "cta_group is 1 or 2");
@@ -170,6 +189,7 @@ struct GemmBf16Cfg {
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA on sm_100");
     static_assert(SMEM_BYTES < (1 << 18), "descriptor start addresses (18 bits) cannot carry");
+    static_assert(!TAIL || TAIL_OK, "narrow tail: one consumer, whole-tile schedule, whole store chunks per half");
 };
 
 // Tile index -> (tile row, tile column), grouped along M so that CTAs
@@ -334,7 +354,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmBt,   // B, box of B_ROWS / 2 rows (narrow tail)
                        int M, int N, int K, void *C, int64_t ldc, int n_tma, int group_m, int wave_tiles,
+                       int tail_first, int tail_parts,
                        DeviceStatus *status, uint64_t timeout_ns, uint32_t inject,
                        Epilogue epi, uint32_t layout,
                        float *sk_partials, unsigned long long *sk_counters, uint32_t sk_epoch,
@@ -405,6 +427,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmB);
         tma_prefetch_map(&tmC);
+        if constexpr (Cfg::TAIL) tma_prefetch_map(&tmBt);
     }
     if (warp == 1) {
         tmem_alloc<CG>(tmem_slot, Cfg::TMEM_COLS);
@@ -420,6 +443,12 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + Cfg::BK - 1) / Cfg::BK;
+    // Narrow tail (K-major B): units [0, tail_first) are whole tiles; tile
+    // tail_first + i runs as unit tail_first + 2 i (columns [0, BN / 2)) and
+    // unit tail_first + 2 i + 1 (columns [BN / 2, BN)).  Otherwise unit = tile.
+    const int parts = (Cfg::TAIL && !b_mn && tail_parts == 2 && tail_first >= 0 && tail_first < num_tiles) ? 2 : 1;
+    const int t_first = parts == 2 ? tail_first : num_tiles;
+    const int num_units = t_first + (num_tiles - t_first) * parts;
     const int cluster_id = static_cast<int>(blockIdx.x) / cluster_ctas;
     const int num_clusters = static_cast<int>(gridDim.x) / cluster_ctas;
     // K blocks of every tile this CTA works on: all of them, or for split-K
@@ -427,18 +456,18 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     const int kb_lo = Cfg::SPLITK ? static_cast<int>((static_cast<int64_t>(kr) * num_kb) / ksplit) : 0;
     const int kb_hi = Cfg::SPLITK ? static_cast<int>((static_cast<int64_t>(kr + 1) * num_kb) / ksplit) : num_kb;
 
-    // The tile sequence every role of this CTA (and of its pair) walks.
-    // Static: cluster_id, + num_clusters, ...  CLC: the first tile is the
-    // cluster's own; the j-th later tile is read from ring slot j % 2, which
+    // The unit sequence every role of this CTA (and of its pair) walks.
+    // Static: cluster_id, + num_clusters, ...  CLC: the first unit is the
+    // cluster's own; the j-th later unit is read from ring slot j % 2, which
     // the scheduler warp fills, and the slot is handed back to the leader.
-    auto next_tile = [&](int tile, uint32_t j, bool &ok) -> int {
+    auto next_tile = [&](int uid, uint32_t j, bool &ok) -> int {
         if constexpr (!Cfg::CLC) {
             (void)j;
             (void)ok;
-            const int n = tile + num_clusters;
-            return n < num_tiles ? n : -1;
+            const int n = uid + num_clusters;
+            return n < num_units ? n : -1;
         } else {
-            (void)tile;
+            (void)uid;
             const uint32_t slot = j & 1u;
             if (!mbar_wait(sched_full(slot), (j >> 1) & 1u, abort_flag, 3 * timeout_ns)) {
                 ok = false;
@@ -451,8 +480,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         }
     };
 
-    // Work units: K blocks [kb0, kb1) of one tile.  Static and CLC
-    // schedules: whole tiles from next_tile.  Stream-K with a data-parallel
+    // Work units: K blocks [kb0, kb1) of one tile (sub = -1), or of one half
+    // of a narrow-tail tile (sub = 0, 1); uid is the unit's index in the
+    // sequence the schedule hands out.  Static and CLC schedules: the units
+    // from next_tile.  Stream-K with a data-parallel
     // head: with W >= 2 full waves of tiles, the first (W - 1) waves are whole
     // tiles dealt round robin (cluster c: c, c + G, ...); the (tile, K block)
     // iterations of the remaining tiles (one wave plus the partial one) are
@@ -463,7 +494,12 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     // shared with the neighbouring clusters complete early, so their fix-ups
     // overlap whole tiles instead of ending the launch.
     struct Unit {
-        int tile, kb0, kb1;
+        int tile, kb0, kb1, sub, uid;
+    };
+    auto unit_of = [&](int uid) -> Unit {
+        if (!Cfg::TAIL || uid < t_first) return Unit{uid, kb_lo, kb_hi, -1, uid};
+        const int r = uid - t_first;
+        return Unit{t_first + r / parts, kb_lo, kb_hi, r % parts, uid};
     };
     const int64_t sk_waves = static_cast<int64_t>(num_tiles) / num_clusters;
     const int64_t dp_tiles = (Cfg::SK && sk_waves >= 2) ? (sk_waves - 1) * num_clusters : 0;
@@ -480,6 +516,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const int64_t t0 = static_cast<int64_t>(u.tile) * num_kb;
         u.kb0 = static_cast<int>(max(it_begin - t0, int64_t(0)));
         u.kb1 = static_cast<int>(min(it_end - t0, static_cast<int64_t>(num_kb)));
+        u.sub = -1;
+        u.uid = u.tile;
         return u;
     };
     auto whole = [&](const Unit &u) { return u.kb0 == 0 && u.kb1 == num_kb; };
@@ -502,7 +540,10 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     auto sk_unit = [&](int j) -> Unit {
         if (j < sk_split_units) return sk_range_unit(sk_order(j));
         if (j < sk_split_units + dp_units)
-            return Unit{cluster_id + (j - sk_split_units) * num_clusters, 0, num_kb};
+        {
+            const int dt = cluster_id + (j - sk_split_units) * num_clusters;
+            return Unit{dt, 0, num_kb, -1, dt};
+        }
         return sk_range_unit(sk_order(j - dp_units));
     };
     auto first_unit = [&](Unit &u) -> bool {
@@ -511,8 +552,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             u = sk_unit(0);
             return true;
         } else {
-            u = Unit{cluster_id, kb_lo, kb_hi};
-            return cluster_id < num_tiles;
+            u = unit_of(cluster_id);
+            return cluster_id < num_units;
         }
     };
     // j counts the units this role has finished (the CLC ring position)
@@ -523,8 +564,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             u = sk_unit(static_cast<int>(j) + 1);
             return true;
         } else {
-            const int n = next_tile(u.tile, j, ok);
-            u = Unit{n, kb_lo, kb_hi};
+            const int n = next_tile(u.uid, j, ok);
+            u = n >= 0 ? unit_of(n) : Unit{-1, kb_lo, kb_hi, -1, -1};
             return n >= 0;
         }
     };
@@ -543,12 +584,17 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 int tm, tn;
                 raster_tile(tile, num_m, num_n, group_m, tm, tn);
                 const int a_row = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA;   // + c * BM_MMA
-                const int b_row = tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
+                // a narrow-tail half: B_ROWS / 2 rows per CTA, from tmBt
+                const bool half = Cfg::TAIL && u.sub >= 0;
+                const int b_row = half ? tn * Cfg::BN + u.sub * (Cfg::BN / 2) + static_cast<int>(rank) * (Cfg::B_ROWS / 2)
+                                       : tn * Cfg::BN + static_cast<int>(rank) * Cfg::B_ROWS;
+                const uint32_t tx = half ? static_cast<uint32_t>(CG * (Cfg::A_BYTES + Cfg::B_BYTES / 2))
+                                         : static_cast<uint32_t>(Cfg::TX_BYTES);
                 // Serpentine K: tiles of odd waves (tile / wave_tiles) walk K
                 // backwards, so a new wave starts on the K slices of A and B
                 // that the wave before it read last, which are still in L2.
                 // The order is fixed per tile, so results stay deterministic.
-                const bool rev = !Cfg::SK && !Cfg::SPLITK && wave_tiles > 0 && ((tile / wave_tiles) & 1) != 0;
+                const bool rev = !Cfg::SK && !Cfg::SPLITK && wave_tiles > 0 && ((u.uid / wave_tiles) & 1) != 0;
                 for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, 2 * timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleProducer * 16 + kBarEmpty);
@@ -567,16 +613,17 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                     uint32_t bar;
                     if constexpr (CG == 1) {
                         bar = full_bar(stage);
-                        mbar_arrive_expect_tx(bar, Cfg::TX_BYTES);
+                        mbar_arrive_expect_tx(bar, tx);
                     } else {
-                        if (rank == leader_rank) mbar_arrive_expect_tx(full_bar(stage), Cfg::TX_BYTES);
+                        if (rank == leader_rank) mbar_arrive_expect_tx(full_bar(stage), tx);
                         bar = map_to_cta(full_bar(stage), leader_rank);
                     }
 #pragma unroll
                     for (int c = 0; c < Cfg::CONSUMERS; ++c)
                         load_operand_tile<CG>(a_dst + c * Cfg::A_PART_BYTES, &tmA, bar, kx, a_row + c * Cfg::BM_MMA,
                                               Cfg::BM_CTA, a_mn);
-                    load_operand_tile<CG>(b_dst, &tmB, bar, kx, b_row, Cfg::B_ROWS, b_mn);
+                    if (half) load_operand_tile<CG>(b_dst, &tmBt, bar, kx, b_row, Cfg::B_ROWS / 2, false);
+                    else load_operand_tile<CG>(b_dst, &tmB, bar, kx, b_row, Cfg::B_ROWS, b_mn);
                     if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -597,7 +644,8 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
         if (rank == 0 && lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(Cfg::BM_MMA, Cfg::BN, a_mn ? 1u : 0u, b_mn ? 1u : 0u);
+            const uint32_t idesc_whole = idesc_bf16_f32(Cfg::BM_MMA, Cfg::BN, a_mn ? 1u : 0u, b_mn ? 1u : 0u);
+            const uint32_t idesc_half = idesc_bf16_f32(Cfg::BM_MMA, Cfg::BN / 2, a_mn ? 1u : 0u, b_mn ? 1u : 0u);
             // Descriptors of stage 0, K step 0.  A stage, a consumer's A part
             // and a K step add their byte offset >> 4 to the start-address
             // field (bits 0-13), which cannot carry out: shared addresses
@@ -621,6 +669,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + buf * Cfg::CONSUMERS * Cfg::BN;
+                const uint32_t idesc = (Cfg::TAIL && u.sub >= 0) ? idesc_half : idesc_whole;
                 for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, timeout_ns)) {
                         record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleMma * 16 + kBarFull);
@@ -706,9 +755,12 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             if (!ready) break;
             tc_fence_after_sync();
             const int row_base = tm * Cfg::BM + static_cast<int>(rank) * Cfg::BM_CTA + static_cast<int>(sub) * 32;
-            const int col0 = tn * Cfg::BN;
+            // a narrow-tail half: columns [sub BN / 2, (sub + 1) BN / 2) of the
+            // tile, in accumulator columns [0, BN / 2)
+            const bool half = Cfg::TAIL && u.sub >= 0;
+            const int col0 = tn * Cfg::BN + (half ? u.sub * (Cfg::BN / 2) : 0);
             const uint32_t tbase0 = tmem_base + ((sub * 32u) << 16) + buf * Cfg::CONSUMERS * Cfg::BN;
-            constexpr int NQ = Cfg::CONSUMERS * Cfg::EPI_CHUNKS;
+            const int NQ = half ? Cfg::EPI_CHUNKS / 2 : Cfg::CONSUMERS * Cfg::EPI_CHUNKS;
             // chunk q: consumer q / EPI_CHUNKS (its own rows and accumulator),
             // columns (q % EPI_CHUNKS) * EPI_COLS of the tile
             auto chunk_taddr = [&](int q) -> uint32_t {
@@ -1026,11 +1078,11 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                 int nt = -1;
                 if (lane == 0) {
                     bool ok = true;
-                    nt = next_tile(tile, static_cast<uint32_t>(t), ok);
+                    nt = next_tile(u.uid, static_cast<uint32_t>(t), ok);
                     if (!ok) record_timeout(status, abort_flag, abort_slot, cluster_ctas, kRoleEpilogue * 16 + kBarSched);
                 }
                 nt = __shfl_sync(0xffffffffu, nt, 0);
-                u = Unit{nt, kb_lo, kb_hi};
+                u = nt >= 0 ? unit_of(nt) : Unit{-1, kb_lo, kb_hi, -1, -1};
                 more = nt >= 0;
             }
         }
