@@ -106,7 +106,14 @@ typedef enum {
 
 /* Kernel configurations.  GEMM_CFG_AUTO picks by shape (gemm_select_config);
  * the others force a configuration (for tests and benchmarks) through
- * gemm_force_config(). */
+ * gemm_force_config().
+ *
+ * Narrow tail: on 1CTA_128x128, 1CTA_128x256, 2CTA_256x256 and their CLC
+ * forms, with B stored N x K, a last wave of tiles that would occupy at most
+ * half of the co-resident clusters runs as half-width units (BN / 2 columns
+ * each), so that the idle clusters take the other halves.  The result is the
+ * same element by element; only the schedule changes.  ("GPU 执行模型",
+ * section "编译与 autotune": tile shape and persistent strategy.) */
 typedef enum {
     GEMM_CFG_AUTO = 0,
     GEMM_CFG_1CTA_128x256 = 1,      /* one CTA per tile, tile 128 x 256, tcgen05 cta_group::1 */
