@@ -548,6 +548,108 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+class _CublasCall:
+    """cuBLAS (torch.mm) on a bf16 workload's device operands, called like Problem.call."""
+
+    def __init__(self, torch):
+        self.torch = torch
+
+    def call(self, G, dev, C, stream):
+        A, B = dev
+        if C.dtype == self.torch.float32:
+            self.torch.mm(A, B.t(), out_dtype=self.torch.float32, out=C)
+        else:
+            self.torch.mm(A, B.t(), out=C)
+
+
+def cublas_context(args):
+    """cuBLAS (torch.matmul / torch.mm) beside this library on one bf16 workload, in the
+    same process and on the same stream, with bf16 and fp32 C for both: a 20-launch burst
+    of each, then an args.steps-launch run of each, two interleaved rounds, back to back
+    (no L2 flush: meant for shapes above 2 x L2, such as 8192^3).  Context for the reports,
+    not a bench line: the JSON line says "context": "cublas", and the clock record covers
+    the long runs.  The library path is the one `gemm_bf16` takes; cuBLAS is never on it."""
+    import torch
+
+    from dense_gemm_engineering_bf16_b200 import gemm as G
+
+    p = Problem(args.workload, args.shape, 0)
+    if p.kind != "bf16":
+        raise SystemExit("--cublas-context: bf16 workloads only")
+    A, B = p.device_arrays(torch)
+    M, N, K = p.M, p.N, p.K
+    C16 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    C32 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    Bt = B.t()                                   # K x N view of B stored N x K
+    s = torch.cuda.current_stream()
+    ops = {
+        "cublas_bf16_out": lambda: torch.matmul(A, Bt, out=C16),
+        "cublas_fp32_out": lambda: torch.mm(A, Bt, out_dtype=torch.float32, out=C32),
+        "ours_bf16_out": lambda: G.gemm_bf16(A, B, C16, M, N, K, K, K, N, G.OUT_BF16, stream=s),
+        "ours_fp32_out": lambda: G.gemm_bf16(A, B, C32, M, N, K, K, K, N, G.OUT_F32, stream=s),
+    }
+
+    def run(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(steps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return round(p.flops * steps / (e0.elapsed_time(e1) * 1e-3) / 1e12, 1)
+
+    res = {name: {"burst_20": [], f"run_{args.steps}": []} for name in ops}
+    for rnd in range(2):
+        for name in (list(ops) if rnd == 0 else list(ops)[::-1]):
+            res[name]["burst_20"].append(run(ops[name], 20))
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    for rnd in range(2):
+        for name in (list(ops) if rnd == 0 else list(ops)[::-1]):
+            res[name][f"run_{args.steps}"].append(run(ops[name], args.steps))
+    sampler.stop()
+    G.gemm_check_device_status(s)
+    line = {"context": "cublas", "workload": p.desc, "unit": "TFLOP/s", "warmup": args.warmup, "results": res,
+            "clocks": sampler.summary()}
+    del A, B, C16, C32
+    if args.configs and args.shape is None:
+        # the bf16 workloads of the per-config report, each with the bench's
+        # L2 rule: per call, median and mean (us) of args.config_steps calls,
+        # three interleaved rounds
+        scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+        cub = _CublasCall(torch)
+        per = {}
+        for name in CONFIG_SET:
+            q = Problem(name, None, 0)
+            if q.kind != "bf16":
+                continue
+            dev = q.device_arrays(torch)
+            C = q.empty_out(torch)
+            flush = needs_l2_flush(min_bytes(q))
+            r = {"ours": {"median_us": [], "mean_us": []}, "cublas": {"median_us": [], "mean_us": []}}
+            for rnd in range(3):
+                for tag, obj in ((("ours", q), ("cublas", cub)) if rnd % 2 == 0 else (("cublas", cub), ("ours", q))):
+                    for _ in range(5):
+                        obj.call(G, dev, C, s)
+                    t, _ = time_steps(obj, G, dev, C, torch, s, args.config_steps, scratch if flush else None)
+                    r[tag]["median_us"].append(round(statistics.median(t) * 1e3, 1))
+                    r[tag]["mean_us"].append(round(statistics.fmean(t) * 1e3, 1))
+            G.gemm_check_device_status(s)
+            per[name] = {"shape": [q.M, q.N, q.K], "c": "fp32" if C.dtype == torch.float32 else "bf16",
+                         "l2": "flushed before every call" if flush else "no flush", **r}
+            del dev, C
+        line["configs"] = per
+    print(json.dumps(line))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -564,6 +666,8 @@ def main():
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the per-config report (default run: every configuration's workload)")
     ap.add_argument("--config-steps", type=int, default=50)
+    ap.add_argument("--cublas-context", action="store_true",
+                    help="instead of the bench line: cuBLAS beside this library on the workload (context)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -575,6 +679,11 @@ def main():
                          "--nproc-per-node N --master-addr 127.0.0.1 bench.py --gpus N")
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.cublas_context:
+        if world > 1:
+            raise SystemExit("--cublas-context runs on one GPU")
+        cublas_context(args)
         return
 
     import torch
