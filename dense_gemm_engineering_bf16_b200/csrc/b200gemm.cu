@@ -18,6 +18,7 @@
 #include "b200gemm.h"
 #include "gemm_bf16_sm100.cuh"
 #include "gemm_bf16_skinny_sm100.cuh"
+#include "gemm_bf16_small_sm100.cuh"
 #include "gemm_mxfp8_sm100.cuh"
 
 namespace {
@@ -334,6 +335,14 @@ gemm_config_t select_config(int64_t M, int64_t N, int64_t K) {
     const int forced = g_forced.load(std::memory_order_relaxed);
     if (forced != GEMM_CFG_AUTO && forced != GEMM_CFG_MXFP8_1CTA_128x256 && forced != GEMM_CFG_MXFP8_2CTA_256x256)
         return static_cast<gemm_config_t>(forced);
+    // A tiny product: the latency path (no tensor memory, no pipeline to
+    // fill).  Measured against the tcgen05 choice, L2 flushed: 128^3 6.7 vs
+    // 12.1 us, 512^3 10.2 vs 13.3, 128 x 128 x 2048 14.4 vs 20.6,
+    // 16 x 4096 x 2048 16.0 vs 20.1; it ties at 768^3, 1024 x 1024 x 256 and
+    // 1024 x 1024 x 128, and loses at 1024^3, 128 x 256 x 4096 and on wide C
+    // with a tiny K (2048 x 2048 x 32: 18.6 vs 12.5), where its 32 x 32 tiles
+    // are too many.
+    if (M * N * K <= (int64_t(1) << 27) && K <= 2048 && M * N <= (int64_t(1) << 20)) return GEMM_CFG_SMALL;
     // A few rows and a long K: swap A and B, so 128 rows of B fill the MMA,
     // and split K (over a cluster per tile of B, else stream-K over every
     // SM).  Past 32 rows the split-K tile kernels win.
@@ -840,9 +849,34 @@ gemm_status_t launch_zero(void *C, int64_t M, int64_t N, int64_t ldc, int sm_cou
 // The dense bf16 kernels, by configuration.
 // `status`: the watchdog status block (the skinny kernel, which only the
 // allocating entry points run, always uses the device's cudaMalloc'd one).
+// The latency path: one ordinary launch, a 32 x 32 tile of C per CTA.
+gemm_status_t launch_small(bool f32, const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                           int64_t lda, int64_t ldb, int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi,
+                           uint32_t layout) {
+    const dim3 grid(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>((M + 31) / 32), 1);
+    const uint16_t *a = static_cast<const uint16_t *>(A);
+    const uint16_t *b = static_cast<const uint16_t *>(B);
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    if (layout == 0) {   // K-major A and B: staged in shared memory
+        if (f32) b200::gemm_bf16_small_kmajor_kernel<0><<<grid, 128, 0, stream>>>(a, b, C, m, n, k, lda, ldb, ldc, epi);
+        else b200::gemm_bf16_small_kmajor_kernel<1><<<grid, 128, 0, stream>>>(a, b, C, m, n, k, lda, ldb, ldc, epi);
+    } else {
+        if (f32) b200::gemm_bf16_small_kernel<0><<<grid, 128, 0, stream>>>(a, b, C, m, n, k, lda, ldb, ldc, layout, epi);
+        else b200::gemm_bf16_small_kernel<1><<<grid, 128, 0, stream>>>(a, b, C, m, n, k, lda, ldb, ldc, layout, epi);
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
 gemm_status_t launch_dense(DeviceState *st, DeviceStatus *status, gemm_config_t cfg, bool f32, const void *A,
                            const void *B, void *C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
                            int64_t ldc, cudaStream_t stream, const b200::Epilogue &epi, uint32_t layout) {
+    // the latency path's grid holds at most 65535 row blocks of 32
+    if (cfg == GEMM_CFG_SMALL) {
+        if ((M + 31) / 32 <= 65535)
+            return launch_small(f32, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout);
+        cfg = GEMM_CFG_1CTA_128x128;
+    }
     switch (cfg) {
         case GEMM_CFG_1CTA_128x256:
             return f32 ? launch_bf16<Cfg1x256F32>(st, status, cfg, A, B, C, M, N, K, lda, ldb, ldc, stream, epi, layout)

@@ -44,6 +44,7 @@ CONFIGS = {
     "2cta_256x224": 11,
     "1cta_128x128_splitk": 12,
     "1cta_128x256_splitk": 13,
+    "small": 14,
 }
 
 STATUS_NAMES = {

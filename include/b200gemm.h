@@ -153,7 +153,12 @@ typedef enum {
                                        environment variable B200GEMM_KSPLIT = 2, 4 or 8, read
                                        once, forces it (tests) */
     GEMM_CFG_1CTA_128x256_SPLITK = 13, /* the same with 128 x 256 tiles (else 1CTA_128x256) */
-    GEMM_CFG_COUNT_ = 14
+    GEMM_CFG_SMALL = 14,            /* latency path for tiny products: warp-level mma.sync
+                                       (m16n8k16, bf16 in, fp32 accumulate) straight from global
+                                       memory, 32 x 32 of C per CTA; no tensor memory, no shared
+                                       memory, no barriers.  Chosen by shape below a measured work
+                                       bound (gemm_select_config); any size when forced */
+    GEMM_CFG_COUNT_ = 15
 } gemm_config_t;
 
 /*

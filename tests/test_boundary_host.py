@@ -155,10 +155,17 @@ def test_status_strings_and_config_control():
     # up to two waves of one-CTA 128 x 256 tiles: their lower fixed cost wins
     assert G.gemm_select_config(2048, 2048, 2048) == G.CONFIGS["1cta_128x256"]
     assert G.gemm_select_config(2560, 3584, 2048) == G.CONFIGS["1cta_128x256"]
+    # a tiny product (at most 2^27 multiply-adds, K <= 2048, C of at most 2^20
+    # elements): the latency path
+    assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["small"]
+    assert G.gemm_select_config(300, 1000, 64) == G.CONFIGS["small"]
+    assert G.gemm_select_config(512, 512, 512) == G.CONFIGS["small"]
+    assert G.gemm_select_config(128, 128, 2048) == G.CONFIGS["small"]
+    assert G.gemm_select_config(128, 256, 4096) == G.CONFIGS["1cta_128x128_splitk"]   # K > 2048
+    assert G.gemm_select_config(2048, 2048, 32) != G.CONFIGS["small"]                   # C too wide
     # every 128 x 128 tile on an SM of its own
-    assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["1cta_128x128"]
-    assert G.gemm_select_config(300, 1000, 64) == G.CONFIGS["1cta_128x128"]
     assert G.gemm_select_config(1000, 1000, 1000) == G.CONFIGS["1cta_128x128"]   # K < 2048: no split
+    assert G.gemm_select_config(1024, 1024, 256) == G.CONFIGS["1cta_128x128"]    # 2^28: past the latency path
     # tiles for at most half the SMs and K >= 2048: cluster split-K
     assert G.gemm_select_config(64, 4096, 4096) == G.CONFIGS["1cta_128x128_splitk"]
     assert G.gemm_select_config(48, 8192, 4096) == G.CONFIGS["1cta_128x128_splitk"]
@@ -198,7 +205,9 @@ def test_configuration_choice_respects_its_own_rules():
     cost model was fitted under: the skinny kernel only for M <= 32 with a
     long K, split-K only with K >= 2048 and tiles for at most half the SMs,
     the single-buffered 512 x 256 tile only for K >= 8192, one-CTA 128 x 256
-    tiles for at most two waves, and never the forced-only kernels."""
+    tiles for at most two waves, the latency path exactly for the products of
+    at most 2^27 multiply-adds with K <= 2048 and C of at most 2^20 elements,
+    and never the forced-only kernels."""
     G.gemm_force_config("auto")
     C = G.CONFIGS
     cdiv = lambda a, b: -(-a // b)  # noqa: E731
@@ -217,3 +226,4 @@ def test_configuration_choice_respects_its_own_rules():
                     assert K >= 8192, (M, N, K)
                 if c == C["1cta_128x256"]:
                     assert cdiv(M, 128) * cdiv(N, 256) <= 2 * 148, (M, N, K)
+                assert (c == C["small"]) == (M * N * K <= 1 << 27 and K <= 2048 and M * N <= 1 << 20), (M, N, K)

@@ -1,0 +1,93 @@
+"""GPU parity of the latency path (config `small`: warp-level mma.sync
+m16n8k16, fragments loaded straight from global memory, 32 x 32 of C per
+CTA).  Compared with the oracle element by element; integer inputs
+bit-exact.  The configuration is forced, so the shapes reach past the size
+the shape-based choice gives it: ragged M, N and K (K odd, below and past one
+16-wide step), several CTAs in both grid directions, both output types, both
+operand layouts, and the fused epilogue."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dense_gemm_engineering_bf16_b200 import gemm as G
+from dense_gemm_engineering_bf16_b200 import synth
+
+from gpu_helpers import assert_close, assert_exact, run_gemm, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+F32, BF16 = G.OUT_F32, G.OUT_BF16
+SHAPES = [(1, 1, 1), (7, 9, 5), (16, 8, 16), (32, 32, 17), (33, 65, 31), (128, 128, 128), (100, 200, 300),
+          (257, 129, 1000), (512, 96, 64)]
+IDS = ["x".join(map(str, s)) for s in SHAPES]
+
+
+@pytest.mark.parametrize("c_type", [F32, BF16])
+@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
+def test_integers_bit_exact(shape, c_type):
+    M, N, K = shape
+    ld = K + (-K % 8)                  # rows on 16-byte boundaries
+    a_bits, b_bits = synth.bf16_operands(M, N, K, "ints", workload=700 + K % 13, lda=ld, ldb=ld)
+    got, guard_ok = run_gemm(a_bits, b_bits, M, N, K, c_type=c_type, config="small").download()
+    assert guard_ok, "write outside C's M x N window"
+    assert_exact(got, oracle.gemm_bf16_f64(a_bits, b_bits, K=K), c_type, f"small {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
+def test_normal_within_tolerance(shape):
+    M, N, K = shape
+    ld = K + (-K % 8)
+    a_bits, b_bits = synth.bf16_operands(M, N, K, "normal", workload=710 + M % 11, lda=ld, ldb=ld)
+    got, guard_ok = run_gemm(a_bits, b_bits, M, N, K, config="small").download()
+    assert guard_ok
+    c_ref, s_abs = oracle.gemm_bf16_f64(a_bits, b_bits, K=K, with_abs=True)
+    assert_close(got, c_ref, s_abs, F32, f"small {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("layouts", [(G.KMAJOR, G.KMAJOR), (G.MNMAJOR, G.KMAJOR), (G.KMAJOR, G.MNMAJOR),
+                                     (G.MNMAJOR, G.MNMAJOR)], ids=["KK", "A_KxM", "B_KxN", "both"])
+@pytest.mark.parametrize("c_type", [F32, BF16])
+def test_fused_epilogue_and_layouts(layouts, c_type):
+    """alpha, beta, bias and GELU, with each operand stored either way.  M and
+    N are multiples of 8: a transposed operand's rows start on 16-byte
+    boundaries."""
+    M, N, K = 120, 200, 77
+    a_lay, b_lay = layouts
+    a_bits, b_bits = synth.bf16_operands(M, N, K, "normal", workload=720)
+    a_dev = np.ascontiguousarray(a_bits.T) if a_lay == G.MNMAJOR else np.ascontiguousarray(
+        np.pad(a_bits, ((0, 0), (0, -K % 8))))
+    b_dev = np.ascontiguousarray(b_bits.T) if b_lay == G.MNMAJOR else np.ascontiguousarray(
+        np.pad(b_bits, ((0, 0), (0, -K % 8))))
+    lda = M if a_lay == G.MNMAJOR else K + (-K % 8)
+    ldb = N if b_lay == G.MNMAJOR else K + (-K % 8)
+    c_old = synth.normal(721, (M, N)).astype(np.float32)
+    bias = synth.uniform(722, (N,)).astype(np.float32)
+    if c_type == F32:
+        C = torch.from_numpy(c_old).cuda()
+        old = c_old.astype(np.float64)
+    else:
+        C = torch.from_numpy(c_old).to(torch.bfloat16).cuda()
+        old = C.float().cpu().numpy().astype(np.float64)
+    G.gemm_force_config("small")
+    try:
+        G.gemm_bf16_fused(to_device_bf16(a_dev), to_device_bf16(b_dev), C, M, N, K, lda, ldb, N, c_type, a_lay,
+                          b_lay, 0.75, -0.5, torch.from_numpy(bias).cuda(), G.ACT_GELU)
+    finally:
+        G.gemm_force_config("auto")
+    G.gemm_check_device_status()
+    got = C.float().cpu().numpy().astype(np.float64)
+    ab, s = oracle.gemm_bf16_f64(a_bits, b_bits, with_abs=True)
+    want = oracle.epilogue(ab, old, 0.75, -0.5, bias.astype(np.float64), G.ACT_GELU)
+    lin = oracle.axpby(ab, old, 0.75, -0.5) + bias.astype(np.float64)[None, :]
+    tol = 1.13 * (0.75 * (1e-3 * s + 1e-6) + 1e-6 * np.abs(0.5 * old)) + 1e-6 * np.abs(lin) + 1e-6
+    if c_type == BF16:
+        tol = tol + np.abs(want) * 2.0 ** -8
+    bad = np.abs(got - want) > tol
+    assert not bad.any(), f"{layouts} c{c_type}: {int(bad.sum())} elements off, first at {np.argwhere(bad)[0]}"
+
+
+def test_chosen_by_shape_for_tiny_products():
+    """The shape-based choice sends the tiny products to this path and the
+    rest to the tcgen05 kernels."""
+    assert G.gemm_select_config(128, 128, 128) == G.CONFIGS["small"]
+    assert G.gemm_select_config(1024, 1024, 1024) != G.CONFIGS["small"]

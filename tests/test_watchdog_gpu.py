@@ -31,7 +31,7 @@ CHILD = textwrap.dedent(r"""
     import oracle
     from dense_gemm_engineering_bf16_b200 import gemm as G, synth
     from gpu_helpers import to_device_bf16
-    M = N = K = 512
+    M = N = K = 768                   # past the latency path (which has no waits to bound)
     a, b = synth.bf16_operands(M, N, K, "normal", workload=77)
     A, B = to_device_bf16(a), to_device_bf16(b)
     C = torch.zeros((M, N), dtype=torch.float32, device="cuda")

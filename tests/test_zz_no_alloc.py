@@ -19,9 +19,10 @@ from gpu_helpers import tolerance, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
-# two calls in a row: different shapes through the same kernel instantiation,
+# two calls in a row: different shapes through the same kernel instantiation
+# (one-CTA 128 x 128 tiles; both products are past the latency path's bound),
 # so the second call cannot trigger a first-use kernel load
-CASES = [(300, 200, 136, G.OUT_F32), (777, 1030, 1000, G.OUT_F32)]
+CASES = [(600, 400, 1000, G.OUT_F32), (777, 1030, 1000, G.OUT_F32)]
 
 
 def _decode(c, c_type):
