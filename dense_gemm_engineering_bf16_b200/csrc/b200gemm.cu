@@ -1017,7 +1017,7 @@ gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const u
                           int64_t ldb, int64_t ldc, cudaStream_t stream) {
     auto kernel = b200::gemm_mxf8_sm100_kernel<Cfg>;
     cudaError_t e;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = Cfg::CG;
     attr[0].val.clusterDim.y = 1;
@@ -1068,6 +1068,12 @@ gemm_status_t launch_mxf8(DeviceState *st, int attr_slot, const void *A, const u
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     const int64_t clusters = tiles < st->mx_max_clusters[attr_slot] ? tiles : st->mx_max_clusters[attr_slot];
     lc.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CG), 1, 1);
+    // programmatic dependent launch: the GEMM's CTAs may start (barriers,
+    // TMEM, tensor-map prefetch) while the repack finishes; its producer
+    // waits on the repack's grid before the first load
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc.numAttrs = 2;
     e = cudaLaunchKernelEx(&lc, kernel, tmA, tmB, tmSF, static_cast<int64_t>(l.a_blocks * l.kb),
                            static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), C, ldc, raster_group_m(),
                            st->status, watchdog_ns(K));

@@ -105,6 +105,9 @@ __global__ void __launch_bounds__(256)
 mxf8_repack_scales_kernel(const uint8_t *__restrict__ sfa, int64_t M, int64_t a_blocks,
                           const uint8_t *__restrict__ sfb, int64_t N, int64_t b_blocks,
                           int64_t k32, int64_t kblocks, uint32_t *__restrict__ out) {
+    // the GEMM launched after this kernel may start its prologue now; it
+    // waits for this grid's results before its first load (griddepcontrol)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ __align__(16) uint8_t tile[128][4 * kRepackKb];
     const int64_t groups = (kblocks + kRepackKb - 1) / kRepackKb;
     int64_t rb = static_cast<int64_t>(blockIdx.x) / groups;
@@ -227,6 +230,11 @@ gemm_mxf8_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
+            // Launched as a programmatic dependent of the scale repack: the
+            // prologue above ran while the repack finished; its chunks (and
+            // every earlier write in the stream) are visible after this wait.
+            // Without that launch attribute the wait returns at once.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
