@@ -15,6 +15,9 @@
 //       r*16 + q*4 + j holds the scale of row 32q + r for the j-th 32-wide
 //       K step.  Padding rows and K steps get 127 (2^0), so zero-filled
 //       operand tails stay zero.
+//   (The GEMM is launched as a programmatic dependent of the repack: the
+//   repack lets it start at once, and its producer waits for the repack grid
+//   before the first load, so the GEMM's prologue overlaps the repack.)
 //   gemm_mxf8_sm100_kernel  persistent, warp-specialised, one CTA (CG = 1,
 //       128 x 256 tile) or a CTA pair (CG = 2, 256 x 256 tile, cta_group::2)
 //       per tile, BK = 128 (one 128-byte swizzle row of E4M3):
