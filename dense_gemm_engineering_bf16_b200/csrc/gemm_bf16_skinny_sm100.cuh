@@ -500,7 +500,7 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
             const int64_t c_lo = range_owner(t * kb_per_tile, total, g);
             const int64_t c_hi = range_owner((t + 1) * kb_per_tile - 1, total, g);
             const bool shared_tile = c_hi > c_lo;
-            // One thread waits; all 128 epilogue threads take its verdict, so
+            // One thread waits; all 128 epilogue threads take its result, so
             // they stay in step for the named barriers below.
             if (epi_tid == 0) {
                 uint32_t ok = 1;

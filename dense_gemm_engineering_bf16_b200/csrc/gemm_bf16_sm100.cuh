@@ -744,7 +744,7 @@ gemm_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
             raster_tile(tile, num_m, num_n, group_m, tm, tn);
             const uint32_t buf = static_cast<uint32_t>(t) % Cfg::ACC_BUFS;
             const uint32_t acc_phase = (static_cast<uint32_t>(t) / Cfg::ACC_BUFS) & 1u;
-            // One lane waits; the verdict is broadcast so the warp stays
+            // One lane waits; the result is broadcast so the warp stays
             // converged for the .sync.aligned TMEM loads below.
             uint32_t ready = 1;
             if (lane == 0 && !mbar_wait(tfull_bar(buf), acc_phase, abort_flag, 3 * timeout_ns)) {
