@@ -708,7 +708,7 @@ gemm_status_t launch_skinny(DeviceState *st, int attr_slot, const void *A, const
     if (layout & b200::kLayoutBMajorN)
         s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, K, ldb * 2, 64, Cfg::BK);
     else
-        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N);
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N / 2);
     if (s != GEMM_OK) return s;
     if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK,
                        static_cast<uint32_t>(mpad))) != GEMM_OK)
@@ -782,7 +782,7 @@ gemm_status_t launch_skinny_cluster(DeviceState *st, DeviceStatus *status, int s
     if (layout & b200::kLayoutBMajorN)
         s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, K, ldb * 2, 64, Cfg::BK);
     else
-        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N);
+        s = encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, Cfg::BK, Cfg::TILE_N / 2);
     if (s != GEMM_OK) return s;
     if ((s = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, Cfg::BK,
                        static_cast<uint32_t>(mpad))) != GEMM_OK)

@@ -200,7 +200,7 @@ __device__ __forceinline__ void fixup_tile(const float *partials, int64_t slot_e
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
-gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as N x K, box 64 x 128
+gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as N x K, box 64 x 64
                               const __grid_constant__ CUtensorMap tmA,   // A as M x K, box 64 x mpad
                               int M, int N, int K, int mpad, void *C, int64_t ldc,
                               float *partials, unsigned long long *counters, int slots_per_cta,
@@ -306,10 +306,19 @@ gemm_bf16_skinny_sm100_kernel(const __grid_constant__ CUtensorMap tmB,   // B as
                 // boxes wholly past K (the last stage of a tile) are skipped
                 const int nbox = min(Cfg::KBS, k_boxes - kb * Cfg::KBS);
                 mbar_arrive_expect_tx(full_bar(stage), static_cast<uint32_t>(nbox) * box_tx);
-                for (int j = 0; j < nbox; ++j)
-                    load_operand_tile<1, true>(b_dst + j * Cfg::B_BOX, &tmB, full_bar(stage),
-                                               (kb * Cfg::KBS + j) * Cfg::BK, t * Cfg::TILE_N, Cfg::TILE_N, b_mn,
-                                               stream_b);
+                // K-major B arrives as two 64-row boxes per 128-row tile (measured:
+                // 35.3 against 36.1 us at 16 x 8192 x 8192 with one 128-row box)
+                for (int j = 0; j < nbox; ++j) {
+                    const int kx = (kb * Cfg::KBS + j) * Cfg::BK;
+                    if (b_mn) {
+                        load_operand_tile<1, true>(b_dst + j * Cfg::B_BOX, &tmB, full_bar(stage), kx,
+                                                   t * Cfg::TILE_N, Cfg::TILE_N, true, stream_b);
+                    } else {
+                        tma_load_2d_hint(b_dst + j * Cfg::B_BOX, &tmB, full_bar(stage), kx, t * Cfg::TILE_N, stream_b);
+                        tma_load_2d_hint(b_dst + j * Cfg::B_BOX + Cfg::B_BOX / 2, &tmB, full_bar(stage), kx,
+                                         t * Cfg::TILE_N + Cfg::TILE_N / 2, stream_b);
+                    }
+                }
                 for (int j = 0; j < nbox; ++j)
                     tma_load_2d(a_dst + j * Cfg::A_BOX, &tmA, full_bar(stage), (kb * Cfg::KBS + j) * Cfg::BK, 0);
                 if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
