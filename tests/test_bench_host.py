@@ -160,3 +160,16 @@ def test_config_set_covers_every_named_configuration():
     assert bench.WORKLOADS["mxfp8_8192"][3] == "mxfp8" and "mxfp8_8192" in bench.CONFIG_SET
     p = bench.Problem("square4096_bf16", (8, 8, 32), 0)
     assert p.bf16_out and p.out_bytes == 2 * 8 * 8
+
+
+def test_cublas_context_mode_refuses_what_it_cannot_compare():
+    """`--cublas-context` prints context, not a bench line: it runs on one GPU
+    and only on bf16 workloads (the block-scaled one has no torch.mm twin),
+    and it says so before touching a device."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--cublas-context", "--workload",
+                          "mxfp8_8192"], capture_output=True, text=True, timeout=300)
+    assert out.returncode != 0 and "bf16 workloads only" in out.stderr
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--cublas-context"], capture_output=True,
+                         text=True, timeout=300, env=env)
+    assert out.returncode != 0 and "one GPU" in out.stderr
