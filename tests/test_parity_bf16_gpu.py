@@ -101,15 +101,29 @@ def test_empty_m_or_n_touches_nothing():
         assert guard_ok
 
 
-def test_nan_propagates():
+@pytest.mark.parametrize("cfg", ["auto", "1cta_128x128", "2cta_256x256", "2cta_256x256_clc", "2cta_512x256_clc",
+                                 "1cta_128x128_splitk", "skinny"])
+def test_nan_and_inf_propagate(cfg):
+    """A NaN in A (row 17) and in B (column 250) makes that row and column of
+    C NaN; an infinity in A (row 40) makes row 40 an infinity with the sign of
+    the B element it meets, exactly as the oracle's IEEE arithmetic does.
+    ("auto" takes the latency path at this size.)"""
     M, N, K = 200, 300, 256
     a_bits, b_bits = synth.bf16_operands(M, N, K, "uniform", workload=50)
     a_bits[17, 100] = 0x7FC0
     b_bits[250, 3] = 0x7FC0
-    C = run_gemm(a_bits, b_bits, M, N, K)
-    got, _ = C.download()
+    a_bits[40, 7] = 0x7F80
+    C = run_gemm(a_bits, b_bits, M, N, K, config=cfg)
+    got, guard_ok = C.download()
+    assert guard_ok
     c_ref, s_abs = oracle.gemm_bf16_f64(a_bits, b_bits, with_abs=True)
-    assert_close(got, c_ref, s_abs, F32, "nan")
+    assert np.array_equal(np.isinf(got), np.isinf(c_ref)), f"{cfg}: infinity pattern differs"
+    inf = np.isinf(c_ref)
+    assert np.array_equal(np.sign(got[inf]), np.sign(c_ref[inf])), f"{cfg}: infinity signs differ"
+    assert inf[40].sum() > 250, "the infinite row is row 40"
+    fin = ~inf
+    assert_close(np.where(fin, got, 0.0), np.where(fin, c_ref, 0.0), np.where(fin, s_abs, 0.0), F32,
+                 f"{cfg}: nan")
 
 
 @pytest.mark.parametrize("cfg", CFGS)
